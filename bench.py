@@ -1,0 +1,561 @@
+"""Benchmark of the MALA hot path on B200.
+
+One step = the whole hot path on one batch of synthetic input:
+  * long-context training operator, B=1 H=8 L=131072 d=128 bf16, tile 128,
+    tau=1: mala_fwd then mala_bwd;
+  * long-context decode, B=16 Hq=32 Hkv=8 Lc=131072 d=128 bf16 cache, tau=1:
+    one mala_decode step.
+The metric is milliseconds per step (lower is better), with the per-call
+breakdown (fwd ms, bwd ms, decode us), effective TFLOP/s (full legal QK plus
+retained post-score work), retained slots per query and the roofline fraction
+of the dominant kernel. The same kernels at tau=0 (dense) are timed beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mala|reference]
+
+N > 1 runs under torchrun, one rank per GPU; the work shards by (batch, head)
+with no exchange step, so every rank runs its own independent copy of the
+workload (weak scaling) and rank 0 prints the max-over-ranks time.
+Inputs are larger than L2 (805 MB of Q/K/V per prefill pass, 8.6 GB of KV
+cache), so no flush is needed between steps.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+PREFILL = synth.CONFIGS["long_128k"]
+DECODE = synth.CONFIGS["decode_128k"]
+WORKLOAD = "long_128k fwd+bwd (B1 H8 L131072 d128 bf16 tile128 tau=1) + decode_128k (B16 Hq32 Hkv8 Lc131072 d128 bf16 tau=1)"
+
+
+# ---------------------------------------------------------------------------
+# input generation (host, numpy; parallel over sequences with a spawn pool)
+# ---------------------------------------------------------------------------
+def _bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float64 -> bf16 bit patterns (round to nearest even) as uint16."""
+    f = a.astype(np.float32)
+    u = f.view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> 16) & np.uint32(1))) >> 16
+    return r.astype(np.uint16)
+
+
+def _gen_prefill_seq(args):
+    cfg_name, s, shm_names, L, d, seed_shift = args
+    from multiprocessing import shared_memory
+    cfg = synth.CONFIGS[cfg_name]
+    seq = synth.prefill_sequence(cfg.config_seed + seed_shift, s, L, d, cfg.rho, cfg.n_pairs)
+    for n, shm_name in shm_names.items():
+        shm = shared_memory.SharedMemory(name=shm_name)
+        arr = np.ndarray((cfg.B * cfg.H, L, d), dtype=np.uint16, buffer=shm.buf)
+        arr[s] = _bf16_bits(seq[n])
+        del arr
+        shm.close()
+    return s
+
+
+def _gen_decode_group(args):
+    s, shm_names, seed_shift = args
+    from multiprocessing import shared_memory
+    cfg = DECODE
+    if seed_shift:
+        cfg = synth.DecodeConfig(cfg.name, cfg.config_seed + seed_shift, cfg.B, cfg.Hq, cfg.Hkv,
+                                 cfg.Lc, cfg.d, cfg.tile, cfg.rho, cfg.n_pairs, cfg.n_query_targets)
+    b, g = divmod(s, cfg.Hkv)
+    grp = synth.decode_group(cfg, b, g)
+    G = cfg.Hq // cfg.Hkv
+    for n in ("K", "V"):
+        shm = shared_memory.SharedMemory(name=shm_names[n])
+        arr = np.ndarray((cfg.B * cfg.Hkv, cfg.Lc, cfg.d), dtype=np.uint16, buffer=shm.buf)
+        arr[s] = _bf16_bits(grp[n])
+        del arr
+        shm.close()
+    shm = shared_memory.SharedMemory(name=shm_names["q"])
+    arr = np.ndarray((cfg.B * cfg.Hkv, G, cfg.d), dtype=np.uint16, buffer=shm.buf)
+    arr[s] = _bf16_bits(grp["q"])
+    del arr
+    shm.close()
+    return s
+
+
+def generate_inputs(workers: int, seed_shift: int = 0):
+    """Returns dict of uint16 (bf16 bit) numpy arrays; runs before any CUDA
+    call so the spawn pool is safe."""
+    import multiprocessing as mp
+    from multiprocessing import shared_memory
+    ctx = mp.get_context("spawn")
+    P = PREFILL
+    shapes = {n: (P.B * P.H, P.L, P.d) for n in ("Q", "K", "V", "dO")}
+    G = DECODE.Hq // DECODE.Hkv
+    dshapes = {"K": (DECODE.B * DECODE.Hkv, DECODE.Lc, DECODE.d),
+               "V": (DECODE.B * DECODE.Hkv, DECODE.Lc, DECODE.d),
+               "q": (DECODE.B * DECODE.Hkv, G, DECODE.d)}
+    shms = {}
+    try:
+        for n, shp in shapes.items():
+            shms["p" + n] = shared_memory.SharedMemory(create=True, size=int(np.prod(shp)) * 2)
+        for n, shp in dshapes.items():
+            shms["d" + n] = shared_memory.SharedMemory(create=True, size=int(np.prod(shp)) * 2)
+        pre_names = {n: shms["p" + n].name for n in shapes}
+        dec_names = {n: shms["d" + n].name for n in dshapes}
+        jobs_p = [(P.name, s, pre_names, P.L, P.d, seed_shift) for s in range(P.B * P.H)]
+        jobs_d = [(s, dec_names, seed_shift) for s in range(DECODE.B * DECODE.Hkv)]
+        with ctx.Pool(max(1, workers)) as pool:
+            pool.map(_gen_prefill_seq, jobs_p)
+            pool.map(_gen_decode_group, jobs_d)
+        out = {}
+        for n, shp in shapes.items():
+            out["p" + n] = np.ndarray(shp, dtype=np.uint16, buffer=shms["p" + n].buf).copy()
+        for n, shp in dshapes.items():
+            out["d" + n] = np.ndarray(shp, dtype=np.uint16, buffer=shms["d" + n].buf).copy()
+        return out
+    finally:
+        for s in shms.values():
+            s.close()
+            s.unlink()
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# work accounting
+# ---------------------------------------------------------------------------
+def legal_pairs(L: int) -> int:
+    return L * (L + 1) // 2
+
+
+def retained_pairs(kept_bits, L: int, tile: int) -> int:
+    """Sum over query rows of the legal keys inside kept tiles, from the
+    [.., nb, nw] keep bitmask (row = query block, bit = key block)."""
+    import mass_adaptive_causal_b200 as mala
+    nb = (L + tile - 1) // tile
+    keep = mala.unpack_bits(kept_bits, nb)  # [..., nb, nb]
+    keep = keep.reshape(-1, nb, nb).astype(np.int64)
+    rows = np.minimum(L - np.arange(nb) * tile, tile)   # rows per query block
+    cols = np.minimum(L - np.arange(nb) * tile, tile)   # keys per key block
+    full = rows[:, None] * cols[None, :]
+    diag = np.array([r * (r + 1) // 2 for r in rows])
+    w = np.tril(full, -1) + np.diag(diag)
+    return int((keep * w[None]).sum())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def load_profile_traffic():
+    """dram bytes per launch from the committed ncu summary, if it is current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(path):
+        try:
+            return json.load(open(path))
+        except Exception:
+            return {}
+    return {}
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+def run_mala(args, rank, world, local_rank):
+    import torch
+    import mass_adaptive_causal_b200 as mala
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    P, Dc = PREFILL, DECODE
+    G = Dc.Hq // Dc.Hkv
+
+    def to_dev(u16, shape):
+        t = torch.from_numpy(u16.view(np.int16)).view(torch.bfloat16).reshape(shape)
+        return t.to(dev)
+
+    x = args._inputs
+    pshape = (P.B, P.H, P.L, P.d)
+    Q, K, V, dO = (to_dev(x["p" + n], pshape) for n in ("Q", "K", "V", "dO"))
+    q = to_dev(x["dq"], (Dc.B, Dc.Hq, Dc.d))
+    Kc = to_dev(x["dK"], (Dc.B, Dc.Hkv, Dc.Lc, Dc.d))
+    Vc = to_dev(x["dV"], (Dc.B, Dc.Hkv, Dc.Lc, Dc.d))
+    O = torch.empty_like(Q)
+    LSE = torch.empty((P.B, P.H, P.L), dtype=torch.float32, device=dev)
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    o = torch.empty_like(q)
+    ws_b = torch.empty(mala.bwd_workspace_bytes(P.B, P.H, P.L, P.d), dtype=torch.uint8, device=dev)
+    ws_d = torch.empty(mala.decode_workspace_bytes(Dc.B, Dc.Hq, Dc.Hkv, Dc.Lc, Dc.d),
+                       dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(tau, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        mala.mala_fwd(Q, K, V, tau=tau, out=O, lse=LSE)
+        if ev is not None:
+            ev[1].record(stream)
+        mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, workspace=ws_b, grads=(dQ, dK, dV))
+        if ev is not None:
+            ev[2].record(stream)
+        mala.mala_decode(q, Kc, Vc, tau=tau, workspace=ws_d, out=o)
+        if ev is not None:
+            ev[3].record(stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed(tau, steps, warmup):
+        for _ in range(warmup):
+            step(tau)
+        mala.mala_check()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for k in range(steps):
+            step(tau, evs[k])
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        mala.mala_check()
+        total = start.elapsed_time(end)
+        fwd = [e[0].elapsed_time(e[1]) for e in evs]
+        bwd = [e[1].elapsed_time(e[2]) for e in evs]
+        dec = [e[2].elapsed_time(e[3]) for e in evs]
+        return {"ms_per_step": max_over_ranks(total / steps),
+                "fwd_ms": max_over_ranks(sum(fwd) / steps),
+                "bwd_ms": max_over_ranks(sum(bwd) / steps),
+                "decode_us": max_over_ranks(1000 * sum(dec) / steps)}
+
+    # trace pass (untimed): retained work and kept decode tiles at tau=1 and 0
+    def trace(tau):
+        _, _, kept_f, bits_f = mala.mala_fwd(Q, K, V, tau=tau, trace=True)
+        _, _, _, kept_b, bits_b = mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, trace=True)
+        _, kept_d, _ = mala.mala_decode(q, Kc, Vc, tau=tau, trace=True)
+        mala.mala_check()
+        nt = (Dc.Lc + 127) // 128
+        return {"fwd_ret": retained_pairs(bits_f, P.L, P.tile),
+                "bwd_ret": retained_pairs(bits_b, P.L, P.tile),
+                "decode_kept_tiles": int(kept_d.sum().item()),
+                "decode_tiles": Dc.B * Dc.Hkv * nt}
+
+    clock = ClockSampler(local_rank)
+    clock.start()
+    t1 = timed(1.0, args.steps, args.warmup)
+    clocks = clock.stop()
+    work1 = trace(1.0)
+    dense = timed(0.0, max(1, min(args.steps, 3)), 1) if not args.no_dense else None
+    e2e = None if args.no_e2e else run_e2e(args, x, dev, world, max_over_ranks)
+    return t1, work1, dense, clocks, e2e
+
+
+def run_e2e(args, x, dev, world, max_over_ranks):
+    """Same metric through the public API with inputs in pinned HOST memory:
+    each step copies the inputs host->device, runs the three calls and copies
+    the results back (O, LSE, dQ, dK, dV and the decode output)."""
+    import torch
+    import mass_adaptive_causal_b200 as mala
+    P, Dc = PREFILL, DECODE
+
+    def pinned(u16, shape):
+        return torch.from_numpy(u16.view(np.int16)).view(torch.bfloat16).reshape(shape).pin_memory()
+
+    pshape = (P.B, P.H, P.L, P.d)
+    hQ, hK, hV, hdO = (pinned(x["p" + n], pshape) for n in ("Q", "K", "V", "dO"))
+    hq = pinned(x["dq"], (Dc.B, Dc.Hq, Dc.d))
+    hKc = pinned(x["dK"], (Dc.B, Dc.Hkv, Dc.Lc, Dc.d))
+    hVc = pinned(x["dV"], (Dc.B, Dc.Hkv, Dc.Lc, Dc.d))
+    outs_h = {n: torch.empty(pshape, dtype=torch.bfloat16).pin_memory() for n in ("O", "dQ", "dK", "dV")}
+    lse_h = torch.empty((P.B, P.H, P.L), dtype=torch.float32).pin_memory()
+    o_h = torch.empty((Dc.B, Dc.Hq, Dc.d), dtype=torch.bfloat16).pin_memory()
+    dQ_ = {n: torch.empty(pshape, dtype=torch.bfloat16, device=dev) for n in ("Q", "K", "V", "dO")}
+    q_, Kc_, Vc_ = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (hq, hKc, hVc))
+    h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hdO, hq, hKc, hVc))
+    d2h = sum(t.numel() * t.element_size() for t in outs_h.values()) + lse_h.numel() * 4 + \
+        o_h.numel() * 2
+
+    def step():
+        for n, h in zip(("Q", "K", "V", "dO"), (hQ, hK, hV, hdO)):
+            dQ_[n].copy_(h, non_blocking=True)
+        q_.copy_(hq, non_blocking=True)
+        Kc_.copy_(hKc, non_blocking=True)
+        Vc_.copy_(hVc, non_blocking=True)
+        O, LSE = mala.mala_fwd(dQ_["Q"], dQ_["K"], dQ_["V"], tau=1.0)
+        dQ, dK, dV = mala.mala_bwd(dQ_["Q"], dQ_["K"], dQ_["V"], O, dQ_["dO"], LSE, tau=1.0)
+        o = mala.mala_decode(q_, Kc_, Vc_, tau=1.0)
+        for n, t in (("O", O), ("dQ", dQ), ("dK", dK), ("dV", dV)):
+            outs_h[n].copy_(t, non_blocking=True)
+        lse_h.copy_(LSE, non_blocking=True)
+        o_h.copy_(o, non_blocking=True)
+
+    steps = max(1, min(args.steps, 3))
+    for _ in range(max(1, min(args.warmup, 2))):
+        step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    mala.mala_check()
+    ms = max_over_ranks(s.elapsed_time(e) / steps)
+    return {"value": ms, "unit": "ms", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (reported baseline; also the --impl reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(x, budget_s: float):
+    """Time the CPU oracle on a bounded sample of the same workload and
+    extrapolate to milliseconds per step. Returns (ms_per_step, cores, desc)."""
+    import oracle
+    cores = oracle.threads(len(os.sched_getaffinity(0)))
+    P, Dc = PREFILL, DECODE
+    T = P.tile
+    nb = P.L // T
+
+    def f64(u16, shape):
+        return (u16.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(shape)
+
+    h = 0
+    Qh = f64(x["pQ"][h], (P.L, P.d))
+    Kh = f64(x["pK"][h], (P.L, P.d))
+    Vh = f64(x["pV"][h], (P.L, P.d))
+    dOh = f64(x["pdO"][h], (P.L, P.d))
+    # forward: the last `nq` query blocks (each visits every key tile)
+    nq = max(1, cores)
+    t0 = time.perf_counter()
+    fr = oracle.fwd(Qh, Kh, Vh, tile=T, tau=1.0, qblocks=(nb - nq, nb))
+    t_fwd = time.perf_counter() - t0
+    tiles_fwd = sum(i + 1 for i in range(nb - nq, nb))
+    fwd_per_tile = t_fwd / tiles_fwd
+    # backward: dK/dV of the last `nk` key blocks and dQ of the last block
+    nk = max(1, cores)
+    LSE = np.nan_to_num(fr["LSE"])
+    Oh = np.nan_to_num(fr["O"])
+    t0 = time.perf_counter()
+    oracle.bwd(Qh, Kh, Vh, Oh, dOh, LSE, tile=T, tau=1.0, qblocks=[nb - 1],
+               kblocks=list(range(nb - nk, nb)))
+    t_bwd = time.perf_counter() - t0
+    tiles_bwd = nb + sum(nb - j for j in range(nb - nk, nb))
+    bwd_per_tile = t_bwd / tiles_bwd
+    # decode: one group
+    nt = Dc.Lc // 128
+    G = Dc.Hq // Dc.Hkv
+    q0 = f64(x["dq"][0], (G, Dc.d))
+    K0 = f64(x["dK"][0], (1, Dc.Lc, Dc.d))
+    V0 = f64(x["dV"][0], (1, Dc.Lc, Dc.d))
+    t0 = time.perf_counter()
+    oracle.decode(q0, K0, V0, tau=1.0)
+    t_dec = time.perf_counter() - t0
+    total_tiles = P.B * P.H * nb * (nb + 1) // 2
+    ms = 1000 * (fwd_per_tile * total_tiles + bwd_per_tile * total_tiles +
+                 t_dec * Dc.B * Dc.Hkv)
+    desc = (f"fwd: last {nq} query blocks of head 0 ({tiles_fwd} tiles, {t_fwd:.1f}s); "
+            f"bwd: dK/dV of last {nk} key blocks + dQ of last query block ({tiles_bwd} tiles, "
+            f"{t_bwd:.1f}s); decode: 1 of {Dc.B * Dc.Hkv} groups ({t_dec:.1f}s); extrapolated "
+            f"per tile pair / per group to the full step")
+    return ms, cores, desc
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="mala", choices=["mala", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workers", type=int, default=0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    ncpu = len(os.sched_getaffinity(0))
+    workers = args.workers or max(1, min(32, ncpu // max(1, world)))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        x = generate_inputs(workers)
+        per_step = []
+        cores, desc = None, ""
+        for _ in range(args.warmup + args.steps):
+            ms, cores, desc = oracle_sample(x, 30.0)
+            per_step.append(ms)
+        ms = statistics.mean(per_step[args.warmup:])
+        line = {"impl": "reference", "metric": "ms per step (fwd+bwd at 128K + one decode step at 128K)",
+                "value": ms, "unit": "ms", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": WORKLOAD},
+                "cpu_baseline": {"value": ms, "unit": "ms", "cores": cores, "kind": "oracle",
+                                 "sample": desc},
+                "e2e": {"value": ms, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    # generate inputs before any CUDA call (spawn pool)
+    x = generate_inputs(workers, seed_shift=0 if world == 1 else 100 * rank)
+    args._inputs = x
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    t1, work, dense, clocks, e2e = run_mala(args, rank, world, local_rank)
+
+    P, Dc = PREFILL, DECODE
+    peaks = load_peaks()
+    d = P.d
+    P_legal = P.B * P.H * legal_pairs(P.L)
+    fwd_flop = 2 * d * P_legal + 2 * d * work["fwd_ret"]
+    bwd_flop = 2 * d * P_legal + 8 * d * work["bwd_ret"]
+    fwd_tf = fwd_flop / (t1["fwd_ms"] * 1e-3) / 1e12
+    bwd_tf = bwd_flop / (t1["bwd_ms"] * 1e-3) / 1e12
+    kc_bytes = Dc.B * Dc.Hkv * Dc.Lc * Dc.d * 2
+    nt = Dc.Lc // 128
+    tile_bytes = 128 * Dc.d * 2
+    dec_bytes = kc_bytes + 2 * work["decode_kept_tiles"] * tile_bytes + \
+        Dc.B * Dc.Hq * (2 * Dc.d * 2 + nt * 8 * 2)
+    dec_gbs = dec_bytes / (t1["decode_us"] * 1e-6) / 1e9
+    dominant = "fwd" if t1["fwd_ms"] >= t1["bwd_ms"] else "bwd"
+    traffic = load_profile_traffic()
+    if dominant == "fwd":
+        roof = {"bound": "tensor", "kernel": "mala::fwd100::fwd_bf16_kernel", "achieved": fwd_tf,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": fwd_tf / peaks["bf16_tflops"],
+                "traffic": traffic.get("fwd_bf16_kernel")}
+    else:
+        roof = {"bound": "tensor", "kernel": "mala::bwd100::bwd_bf16_kernel", "achieved": bwd_tf,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": bwd_tf / peaks["bf16_tflops"],
+                "traffic": traffic.get("bwd_bf16_kernel")}
+    roof["peak_source"] = peaks["source"] + " (burst bf16 cuBLAS)"
+    roof["frac_of_sustained"] = roof["achieved"] / (peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"])
+
+    line = {
+        "metric": "ms per step (fwd+bwd at 128K + one decode step at 128K)",
+        "value": t1["ms_per_step"], "unit": "ms", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t1["ms_per_step"], "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tau": 1.0, "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"replicas x{world} (independent heads/sequences per rank)"},
+        "fwd_ms": t1["fwd_ms"], "bwd_ms": t1["bwd_ms"], "decode_us": t1["decode_us"],
+        "fwd_tflops_eff": fwd_tf, "bwd_tflops_eff": bwd_tf,
+        "fwd_frac_bf16": fwd_tf / peaks["bf16_tflops"], "bwd_frac_bf16": bwd_tf / peaks["bf16_tflops"],
+        "decode_gbs": dec_gbs, "decode_frac_hbm": dec_gbs / peaks["hbm_gbs"],
+        "decode_bytes": dec_bytes,
+        "fwd_slots_per_query": work["fwd_ret"] / (P.B * P.H * P.L),
+        "bwd_slots_per_query": work["bwd_ret"] / (P.B * P.H * P.L),
+        "decode_kept_tile_frac": work["decode_kept_tiles"] / work["decode_tiles"],
+        "roofline": roof,
+        "clocks": clocks,
+        "gpu_launches": args.steps * (1 + 4 + 4),
+    }
+    if dense is not None:
+        line["dense_tau0"] = {"fwd_ms": dense["fwd_ms"], "bwd_ms": dense["bwd_ms"],
+                              "decode_us": dense["decode_us"],
+                              "fwd_speedup": dense["fwd_ms"] / t1["fwd_ms"],
+                              "bwd_speedup": dense["bwd_ms"] / t1["bwd_ms"],
+                              "decode_speedup": dense["decode_us"] / t1["decode_us"],
+                              "fwd_tflops": 4 * d * P_legal / (dense["fwd_ms"] * 1e-3) / 1e12,
+                              "bwd_tflops": 10 * d * P_legal / (dense["bwd_ms"] * 1e-3) / 1e12}
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ms, cores, desc = oracle_sample(x, 30.0)
+        line["cpu_baseline"] = {"value": ms, "unit": "ms", "cores": cores, "kind": "oracle",
+                                "sample": desc}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,169 @@
+/*
+ * mala.h -- C ABI of the MALA (MassAlloc Attention) library for NVIDIA B200
+ * (sm_100a).
+ *
+ * MALA is causal softmax attention that computes every legal QK tile but
+ * skips the post-score work of a tile when, for every valid query row of the
+ * tile, the tile's largest per-key contribution ratio is below tau / Lq
+ * (Lq = number of keys the query can see). Sources: the pages on arXiv
+ * 2609.32712 "MassAlloc Attention: Let Attention Allocate Its Own Compute" --
+ * agihunt.info summary (rule, forward and backward paragraphs) and the
+ * jaehun.me review, sections "One tolerance governs everything", "Forward:
+ * online sparse softmax" and "Backward: offline sparse probabilities".
+ *
+ * Conventions shared by every call
+ *  - Layout: Q, K, V, O, dO, dQ, dK, dV are [B][H][L][d] contiguous, d
+ *    innermost; LSE is [B][H][L] float32. The decode cache is
+ *    [B][Hkv][Lc][d]; the decode query and output are [B][Hq][d]. Query head
+ *    h uses KV head h / (Hq / Hkv).
+ *  - All data pointers are DEVICE pointers, 16-byte aligned. The caller owns
+ *    every buffer (inputs, outputs, workspace); the library allocates no
+ *    device memory and keeps no state between calls except one device-side
+ *    status word per GPU (see mala_check).
+ *  - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is asynchronous on that stream; none synchronizes.
+ *  - scale <= 0 selects 1/sqrt(d). tau >= 0 and finite; tau = 0 never skips
+ *    (exact FullAttn, the pages' tau -> 0 limit). tau < 0 or NaN is
+ *    MALA_ERR_INVALID_ARG.
+ *  - Argument errors are detected on the host and returned before anything
+ *    is launched. A failed launch returns MALA_ERR_CUDA. A device-side wait
+ *    that exceeds its time limit (about two seconds) records a status that
+ *    mala_check reports as MALA_ERR_TIMEOUT; kernels never trap.
+ *  - Optional trace outputs (pass NULL to skip them; device pointers):
+ *      kept_tiles: int32 counts of kept tiles (layout per call below);
+ *      keep_bits:  uint32 bitmask, bit (j % 32) of word [.., row, j / 32]
+ *                  set iff tile (row, j) was kept. Both are written in full
+ *                  by the call (no pre-zeroing needed).
+ */
+#ifndef MALA_H
+#define MALA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MALA_OK = 0,
+  MALA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned, tau < 0 */
+  MALA_ERR_UNSUPPORTED = 2, /* (dtype, d, tile) combination not built */
+  MALA_ERR_CUDA = 3,        /* CUDA runtime error at launch or check */
+  MALA_ERR_TIMEOUT = 4      /* a device-side wait ran out (see mala_check) */
+} mala_status;
+
+typedef enum { MALA_F32 = 0, MALA_BF16 = 1 } mala_dtype;
+
+/*
+ * Forward pass (training forward / prefill).
+ *
+ * Per (b, h, query block i of `tile` rows) the key tiles j = i, i-1, ..., 0
+ * are visited from the diagonal toward earlier keys. Every legal tile's
+ * scores S = scale * Q_i K_j^T are computed. With the running row max m, the
+ * retained mass l (online softmax over the tiles kept so far) and the tile's
+ * row max mt, the tile is skipped iff every valid row r satisfies
+ *     mt_r - m_r - ln l_r  <  ln tau - ln (r + 1)
+ * (the log form of exp(mt - m) / l < tau / Lq; equality keeps). A skipped
+ * tile leaves m, l and O untouched and its V is never read; a kept tile does
+ * the standard online-softmax update. The diagonal tile is always kept.
+ * Sources: agihunt.info summary, forward paragraph; jaehun.me review,
+ * "Forward: online sparse softmax".
+ *
+ * Inputs  Q, K, V: [B][H][L][d] of dtype dt.
+ * Outputs O: [B][H][L][d] of dtype dt, softmax over the retained tiles;
+ *         LSE: [B][H][L] float32, natural-log normalizer m + ln l over the
+ *         retained keys (the only state backward needs).
+ * Trace   kept_tiles: [B][H][nb] kept key tiles per query block;
+ *         keep_bits: [B][H][nb][ceil(nb/32)], row = query block, bit = key
+ *         block. nb = ceil(L / tile).
+ * Supported: (dt, d, tile) in {(MALA_BF16, 128, 128), (MALA_F32, 32|64|128, 64)};
+ *            any L >= 0 (a ragged last block is masked), B, H >= 1.
+ */
+mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O,
+                     float* LSE, int B, int H, int L, int d, mala_dtype dt,
+                     float tau, int tile, float scale, int32_t* kept_tiles,
+                     uint32_t* keep_bits, void* stream);
+
+/* Bytes of device workspace mala_bwd needs: the row terms D (float32
+ * [B][H][L]) and the float32 dQ accumulator [B][H][L][d], each rounded up to
+ * 256 bytes. */
+size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
+
+/*
+ * Backward pass.
+ *
+ * Uses the forward's final LSE instead of replaying its partial normalizers.
+ * Every legal tile (i, j) has its scores recomputed; the tile is skipped iff
+ * every valid row r satisfies  max_c S_rc - LSE_r  <  ln tau - ln (r + 1).
+ * There is no forced keep and no stored mask; in exact arithmetic the kept
+ * set is inside the forward's. Kept tiles do the standard work with
+ * P = exp(S - LSE), D_r = <dO_r, O_r>: dV_j += P^T dO_i, dP = dO_i V_j^T,
+ * dS = P o (dP - D), dQ_i += scale dS K_j, dK_j += scale dS^T Q_i.
+ * Sources: agihunt.info summary, backward paragraph; jaehun.me review,
+ * "Backward: offline sparse probabilities".
+ *
+ * Inputs  Q, K, V, O, dO: [B][H][L][d] of dtype dt; LSE from mala_fwd.
+ * Outputs dQ, dK, dV: [B][H][L][d] of dtype dt (fully overwritten).
+ * workspace: device buffer of at least mala_bwd_workspace_bytes(B,H,L,d)
+ *         bytes, 256-byte aligned, contents ignored on entry.
+ * Trace   kept_tiles: [B][H][nb] kept query blocks per key block;
+ *         keep_bits: [B][H][nb][ceil(nb/32)], row = query block i, bit = key
+ *         block j.
+ * Supported: as mala_fwd.
+ */
+mala_status mala_bwd(const void* Q, const void* K, const void* V,
+                     const void* O, const void* dO, const float* LSE, void* dQ,
+                     void* dK, void* dV, void* workspace,
+                     size_t workspace_bytes, int B, int H, int L, int d,
+                     mala_dtype dt, float tau, int tile, float scale,
+                     int32_t* kept_tiles, uint32_t* keep_bits, void* stream);
+
+/* Bytes of device workspace mala_decode needs (per-tile statistics, the
+ * kept-tile lists, the final normalizers and a float32 output accumulator),
+ * each part rounded up to 256 bytes. */
+size_t mala_decode_workspace_bytes(int B, int Hq, int Hkv, int Lc, int d);
+
+/*
+ * One decode step with the same rule (agihunt.info summary: one tau for
+ * prefill and decode; the KV cache is kept whole).
+ *
+ * The cache holds Lc keys per (b, kv head) including the current token, so
+ * Lq = Lc. Key tiles of 128 positions are aligned from position 0 and
+ * visited newest first; the newest tile is always kept. The rows of a tile
+ * are the G = Hq / Hkv query heads that share the KV head, and the tile is
+ * skipped iff every one of them is below the threshold (tile granularity is
+ * conservative). Kept tiles update the per-head online softmax; the output is
+ * softmax over the kept tiles.
+ *
+ * Inputs  q: [B][Hq][d] bf16; Kcache, Vcache: [B][Hkv][Lc][d] bf16.
+ * Output  o: [B][Hq][d] bf16.
+ * workspace: at least mala_decode_workspace_bytes(B,Hq,Hkv,Lc,d) bytes.
+ * Trace   kept_tiles: [B][Hkv]; keep_bits: [B][Hkv][ceil(nt/32)], nt =
+ *         ceil(Lc / 128).
+ * Supported: d = 128, Hq % Hkv == 0, 1 <= Hq / Hkv <= 16, Lc >= 1.
+ */
+mala_status mala_decode(const void* q, const void* Kcache, const void* Vcache,
+                        void* o, int B, int Hq, int Hkv, int Lc, int d,
+                        float tau, float scale, void* workspace,
+                        size_t workspace_bytes, int32_t* kept_tiles,
+                        uint32_t* keep_bits, void* stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears this GPU's device status word.
+ * Returns MALA_ERR_CUDA if the stream reported an error, MALA_ERR_TIMEOUT if
+ * a kernel gave up on a wait since the last check, MALA_OK otherwise.
+ */
+mala_status mala_check(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* mala_status_string(mala_status s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int mala_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MALA_H */

@@ -1,0 +1,223 @@
+"""MALA (MassAlloc Attention) for NVIDIA B200 -- Python binding of the C ABI.
+
+This module only marshals arguments: torch tensors supply device memory and
+the current CUDA stream; every step of the computation runs in the kernels of
+``libmala.so`` (built from ``csrc/`` for sm_100a). There is no fallback: if
+the library is missing or fails to load, every call raises.
+
+Entry points (same names as the C ABI in ``include/mala.h``):
+
+* :func:`mala_fwd`    -- forward / prefill: O, LSE
+* :func:`mala_bwd`    -- backward: dQ, dK, dV
+* :func:`mala_decode` -- one decode step over a KV cache: o
+* :func:`mala_check`  -- synchronize and read the device status word
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = ["mala_fwd", "mala_bwd", "mala_decode", "mala_check", "MalaError", "lib",
+           "LIB_PATH", "MALA_F32", "MALA_BF16", "STATUS"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmala.so")
+
+MALA_F32, MALA_BF16 = 0, 1
+STATUS = {0: "MALA_OK", 1: "MALA_ERR_INVALID_ARG", 2: "MALA_ERR_UNSUPPORTED",
+          3: "MALA_ERR_CUDA", 4: "MALA_ERR_TIMEOUT"}
+
+
+class MalaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+
+
+_lib = None
+_vp, _i32p, _u32p, _fp = (ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m mass_adaptive_causal_b200.build`"
+                " (or __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        ci, cf, cs = ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.mala_fwd.argtypes = [_vp, _vp, _vp, _vp, _fp, ci, ci, ci, ci, ci, cf, ci, cf, _i32p,
+                               _u32p, _vp]
+        L.mala_fwd.restype = ci
+        L.mala_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
+        L.mala_bwd_workspace_bytes.restype = cs
+        L.mala_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, cs, ci, ci, ci, ci,
+                               ci, cf, ci, cf, _i32p, _u32p, _vp]
+        L.mala_bwd.restype = ci
+        L.mala_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
+        L.mala_decode_workspace_bytes.restype = cs
+        L.mala_decode.argtypes = [_vp, _vp, _vp, _vp, ci, ci, ci, ci, ci, cf, cf, _vp, cs, _i32p,
+                                  _u32p, _vp]
+        L.mala_decode.restype = ci
+        L.mala_check.argtypes = [_vp]
+        L.mala_check.restype = ci
+        L.mala_status_string.argtypes = [ci]
+        L.mala_status_string.restype = ctypes.c_char_p
+        L.mala_version.argtypes = []
+        L.mala_version.restype = ci
+        _lib = L
+    return _lib
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return MALA_F32
+    if t.dtype == torch.bfloat16:
+        return MALA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _check_prefill(*ts):
+    torch = _torch()
+    ref = ts[0]
+    for t in ts:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+        if t.shape != ref.shape or t.dtype != ref.dtype:
+            raise ValueError("Q, K, V (, O, dO) must share shape and dtype")
+    if ref.dim() != 4:
+        raise ValueError("expected [B, H, L, d]")
+    return torch
+
+
+def _raise(code, where):
+    if code != 0:
+        raise MalaError(code, where)
+
+
+def default_tile(dtype) -> int:
+    torch = _torch()
+    return 128 if dtype == torch.bfloat16 else 64
+
+
+def n_blocks(L: int, tile: int) -> int:
+    return (L + tile - 1) // tile
+
+
+def mala_fwd(q, k, v, tau: float = 1.0, tile: int | None = None, scale: float = 0.0,
+             trace: bool = False, out=None, lse=None, stream=None):
+    """Forward pass. q, k, v: [B, H, L, d] (bf16 with d = 128, or float32).
+
+    Returns (O, LSE) or, with ``trace=True``, (O, LSE, kept_tiles, keep_bits)
+    where kept_tiles is int32 [B, H, nb] and keep_bits int32 [B, H, nb, nw]."""
+    torch = _check_prefill(q, k, v)
+    B, H, L, d = q.shape
+    tile = default_tile(q.dtype) if tile is None else tile
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if lse is None else lse
+    kept = bits = None
+    if trace:
+        nb = n_blocks(L, tile)
+        kept = torch.empty((B, H, nb), dtype=torch.int32, device=q.device)
+        bits = torch.empty((B, H, nb, (nb + 31) // 32), dtype=torch.int32, device=q.device)
+    code = lib().mala_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, H, L, d,
+                          _dtype_code(q), float(tau), int(tile), float(scale), _ptr(kept),
+                          _ptr(bits), _stream(stream))
+    _raise(code, "mala_fwd")
+    return (o, lse_t, kept, bits) if trace else (o, lse_t)
+
+
+def bwd_workspace_bytes(B, H, L, d) -> int:
+    return int(lib().mala_bwd_workspace_bytes(B, H, L, d))
+
+
+def mala_bwd(q, k, v, o, do, lse, tau: float = 1.0, tile: int | None = None,
+             scale: float = 0.0, trace: bool = False, workspace=None, grads=None, stream=None):
+    """Backward pass. Returns (dQ, dK, dV) or, with ``trace=True``,
+    (dQ, dK, dV, kept_tiles [B, H, nb] per key block, keep_bits [B, H, nb, nw])."""
+    torch = _check_prefill(q, k, v, o, do)
+    B, H, L, d = q.shape
+    tile = default_tile(q.dtype) if tile is None else tile
+    if grads is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = grads
+    nbytes = bwd_workspace_bytes(B, H, L, d)
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device) if workspace is None \
+        else workspace
+    kept = bits = None
+    if trace:
+        nb = n_blocks(L, tile)
+        kept = torch.empty((B, H, nb), dtype=torch.int32, device=q.device)
+        bits = torch.empty((B, H, nb, (nb + 31) // 32), dtype=torch.int32, device=q.device)
+    code = lib().mala_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                          _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), B, H, L, d, _dtype_code(q),
+                          float(tau), int(tile), float(scale), _ptr(kept), _ptr(bits),
+                          _stream(stream))
+    _raise(code, "mala_bwd")
+    return (dq, dk, dv, kept, bits) if trace else (dq, dk, dv)
+
+
+def decode_workspace_bytes(B, Hq, Hkv, Lc, d) -> int:
+    return int(lib().mala_decode_workspace_bytes(B, Hq, Hkv, Lc, d))
+
+
+def mala_decode(q, k_cache, v_cache, tau: float = 1.0, scale: float = 0.0, trace: bool = False,
+                workspace=None, out=None, stream=None):
+    """One decode step. q: [B, Hq, d] bf16; caches: [B, Hkv, Lc, d] bf16.
+    Returns o [B, Hq, d] or, with ``trace=True``, (o, kept_tiles [B, Hkv],
+    keep_bits [B, Hkv, nw])."""
+    torch = _torch()
+    for t in (q, k_cache, v_cache):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("decode tensors must be contiguous bf16 CUDA tensors")
+    B, Hq, d = q.shape
+    _, Hkv, Lc, _ = k_cache.shape
+    o = torch.empty_like(q) if out is None else out
+    nbytes = decode_workspace_bytes(B, Hq, Hkv, Lc, d)
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device) if workspace is None \
+        else workspace
+    kept = bits = None
+    if trace:
+        nt = n_blocks(Lc, 128)
+        kept = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+        bits = torch.empty((B, Hkv, (nt + 31) // 32), dtype=torch.int32, device=q.device)
+    code = lib().mala_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), B, Hq, Hkv, Lc, d,
+                             float(tau), float(scale), _ptr(ws), ws.numel(), _ptr(kept),
+                             _ptr(bits), _stream(stream))
+    _raise(code, "mala_decode")
+    return (o, kept, bits) if trace else o
+
+
+def mala_check(stream=None):
+    """Synchronize the stream and raise MalaError if a kernel reported a
+    timeout or the stream holds a CUDA error."""
+    _raise(lib().mala_check(_stream(stream)), "mala_check")
+
+
+def unpack_bits(bits, n: int):
+    """[..., nw] int32 keep bitmask -> [..., n] uint8 (host numpy)."""
+    import numpy as np
+    b = bits.cpu().numpy().astype(np.uint32)
+    shifts = np.arange(32, dtype=np.uint32)
+    out = ((b[..., :, None] >> shifts) & 1).astype(np.uint8)
+    return out.reshape(*b.shape[:-1], -1)[..., :n]

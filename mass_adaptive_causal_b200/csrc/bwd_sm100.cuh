@@ -1,0 +1,347 @@
+// bwd_sm100.cuh -- MALA backward for bf16, d = 128, 128 x 128 tiles on the
+// 5th-generation tensor cores (tcgen05 + TMEM), operands staged by TMA.
+//
+// Rule (MassAlloc Attention; agihunt.info summary, backward paragraph;
+// jaehun.me review, "Backward: offline sparse probabilities"): the backward
+// reuses the forward's final log-normalizer LSE. For every legal tile (query
+// block i, key block j) the scores are recomputed and the tile is skipped iff
+// every valid query row r has  max_c S_rc - LSE_r < ln tau - ln(r+1).
+// Only kept tiles load dO_i and do the post-score work
+//   P = exp(S - LSE), dV_j += P^T dO_i, dP = dO_i V_j^T, dS = P o (dP - D),
+//   dK_j += scale dS^T Q_i, dQ_i += scale dS K_j.
+//
+// The test "every row below its threshold" is evaluated per key instead of
+// per query: keep iff some (query q, key k) has S_qk >= LSE_q + ln tau -
+// ln(q+1). With the scores transposed (keys in TMEM lanes) each thread checks
+// its own key against the 128 per-query thresholds, then the CTA votes.
+//
+// CTA (128 threads) = one key block j, looping over query blocks i >= j.
+// Thread t owns key row t = TMEM lane t for the key-major products:
+//   TMEM [  0,128): S^T = K_j Q_i^T, later reused for dQ_i = dS K_j
+//   TMEM [128,256): dP^T = V_j dO_i^T
+//   TMEM [256,384): dK_j accumulator      TMEM [384,512): dV_j accumulator
+// Shared memory: K_j, V_j, Q_i, dO_i, P^T, dS^T (32 KB each, 128-byte
+// swizzle) + the per-query thresholds and D terms.
+// dQ_i is read back from TMEM (query rows in lanes) and added with float4
+// atomics into a float32 workspace; a separate kernel converts it to bf16.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace mala {
+namespace bwd100 {
+
+using namespace sm100;
+
+constexpr int T = 128;
+constexpr int D = 128;
+constexpr int NT = 128;
+constexpr uint32_t TILE_BYTES = T * D * 2;
+constexpr uint32_t HALF_BYTES = T * 64 * 2;
+constexpr uint32_t SMEM_BYTES = 6 * TILE_BYTES + 1024 /*align*/ + 2048 /*thresholds*/ + 256;
+constexpr uint32_t TMEM_COLS = 512;
+// S^T, dP^T: A = K_j or V_j (K-major over d), B = Q_i or dO_i (K-major over d)
+constexpr uint32_t IDESC_KQ = idesc_bf16(128, 128, false, false);
+// dV, dK: A = P^T or dS^T (K-major over queries), B = dO_i or Q_i (MN-major: d contiguous)
+constexpr uint32_t IDESC_ACC = idesc_bf16(128, 128, false, true);
+// dQ: A = dS (queries contiguous in dS^T rows: MN-major), B = K_j (MN-major)
+constexpr uint32_t IDESC_DQ = idesc_bf16(128, 128, true, true);
+
+struct Params {
+  const float* LSE;
+  const float* Dterm;
+  float* dQacc;
+  __nv_bfloat16* dK;
+  __nv_bfloat16* dV;
+  int L;
+  int nb;
+  float scale;       // softmax scale (dS is scaled before the bf16 cast)
+  float scale_log2;  // scale * log2(e)
+  float log2_tau;
+  int never_skip;
+  int32_t* kept_tiles;
+  uint32_t* keep_bits;  // pre-zeroed by the host
+};
+
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, uint32_t taddr) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 w;
+      w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+      w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+      w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+      w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+      d4[q] = w;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(NT, 1)
+    bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                    const Params p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t ka = smem_u32(base);
+  const uint32_t va = ka + TILE_BYTES;
+  const uint32_t qa = ka + 2 * TILE_BYTES;
+  const uint32_t da = ka + 3 * TILE_BYTES;   // dO_i
+  const uint32_t pta = ka + 4 * TILE_BYTES;  // P^T
+  const uint32_t sta = ka + 5 * TILE_BYTES;  // dS^T
+  float* thr_s = reinterpret_cast<float*>(base + 6 * TILE_BYTES);  // [128] LSE2 + log2 thr
+  float* lse_s = thr_s + T;                                        // [128] LSE2
+  float* dd_s = lse_s + T;                                         // [128] D
+  uint64_t* bars = reinterpret_cast<uint64_t*>(dd_s + T + 128);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int j = blockIdx.x;  // key block 0 has the most query blocks: first
+  const int z = blockIdx.y;
+  const uint32_t bar_kv = smem_u32(&bars[0]);
+  const uint32_t bar_q = smem_u32(&bars[1]);
+  const uint32_t bar_do = smem_u32(&bars[2]);
+  const uint32_t bar_mma = smem_u32(&bars[3]);
+
+  if (tid == 0) {
+    mbar_init(bar_kv, 1);
+    mbar_init(bar_q, 1);
+    mbar_init(bar_do, 1);
+    mbar_init(bar_mma, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const uint32_t t_st = tmem + lane_base;         // S^T, then dQ
+  const uint32_t t_dpt = tmem + lane_base + 128;  // dP^T
+  const uint32_t t_dk = tmem + lane_base + 256;
+  const uint32_t t_dv = tmem + lane_base + 384;
+
+  if (tid == 0) {
+    mbar_expect_tx(bar_kv, 2 * TILE_BYTES);
+    tma_load_3d(ka, &tmK, 0, j * T, z, bar_kv);
+    tma_load_3d(ka + HALF_BYTES, &tmK, 64, j * T, z, bar_kv);
+    tma_load_3d(va, &tmV, 0, j * T, z, bar_kv);
+    tma_load_3d(va + HALF_BYTES, &tmV, 64, j * T, z, bar_kv);
+    mbar_expect_tx(bar_q, TILE_BYTES);
+    tma_load_3d(qa, &tmQ, 0, j * T, z, bar_q);
+    tma_load_3d(qa + HALF_BYTES, &tmQ, 64, j * T, z, bar_q);
+  }
+  uint32_t ph_q = 0, ph_do = 0, ph_mma = 0;
+  int kept_count = 0;
+  bool ok = mbar_wait(bar_kv, 0, abort, 0x201);
+  const int nw = (p.nb + 31) >> 5;
+
+  for (int i = j; i < p.nb && ok; ++i) {
+    // per-query thresholds of this block (log2 domain)
+    {
+      const int q = i * T + tid;
+      const bool qv = q < p.L;
+      const float lse2 = qv ? p.LSE[(size_t)z * p.L + q] * kLog2e : 0.f;
+      lse_s[tid] = lse2;
+      dd_s[tid] = qv ? p.Dterm[(size_t)z * p.L + q] : 0.f;
+      thr_s[tid] = !qv ? __int_as_float(0x7f800000)
+                       : (p.never_skip ? kNegInf : lse2 + p.log2_tau - __log2f((float)(q + 1)));
+    }
+    if (!mbar_wait(bar_q, ph_q, abort, 0x202)) ok = false;
+    ph_q ^= 1;
+    if (__syncthreads_or(!ok)) { ok = false; break; }
+    // ---- S^T = K_j Q_i^T -----------------------------------------------------
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+        mma_bf16(tmem, sdesc_sw128(ka + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024),
+                 IDESC_KQ, kk > 0);
+      }
+      mma_commit(bar_mma);
+    }
+    if (!mbar_wait(bar_mma, ph_mma, abort, 0x203)) ok = false;
+    ph_mma ^= 1;
+    if (__syncthreads_or(!ok)) { ok = false; break; }
+    tc_fence_after();
+    // ---- offline test: does this key reach any query's threshold? ----------
+    const bool diag = (i == j);
+    int want = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float s[32];
+      tmem_ld32(t_st + c * 32, s);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int qc = c * 32 + e;
+        const bool legal = !diag || qc >= tid;
+        want |= (legal && s[e] * p.scale_log2 >= thr_s[qc]);
+      }
+    }
+    tc_fence_before();
+    const int keep = __syncthreads_or(want);
+    if (tid == 0 && keep && p.keep_bits)
+      atomicOr(&p.keep_bits[((size_t)z * p.nb + i) * nw + (j >> 5)], 1u << (j & 31));
+    if (keep) {
+      if (tid == 0) {
+        mbar_expect_tx(bar_do, TILE_BYTES);
+        tma_load_3d(da, &tmdO, 0, i * T, z, bar_do);
+        tma_load_3d(da + HALF_BYTES, &tmdO, 64, i * T, z, bar_do);
+      }
+      // P^T row (key tid) over the block's queries, fp32 kept for dS
+      float pr[T];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float s[32];
+        tmem_ld32(t_st + c * 32, s);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int qc = c * 32 + e;
+          const bool legal = (!diag || qc >= tid) && (i * T + qc) < p.L;
+          pr[qc] = legal ? exp2f(s[e] * p.scale_log2 - lse_s[qc]) : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int q0 = c * 32 + q * 8;
+          st_shared_v4(pta + sw128_chunk_off(tid, q0, T), pack_bf16(pr[q0], pr[q0 + 1]),
+                       pack_bf16(pr[q0 + 2], pr[q0 + 3]), pack_bf16(pr[q0 + 4], pr[q0 + 5]),
+                       pack_bf16(pr[q0 + 6], pr[q0 + 7]));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (!mbar_wait(bar_do, ph_do, abort, 0x204)) ok = false;
+      ph_do ^= 1;
+      if (__syncthreads_or(!ok)) { ok = false; break; }
+      // ---- dP^T = V_j dO_i^T ; dV += P^T dO_i ---------------------------------
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          mma_bf16(tmem + 128, sdesc_sw128(va + off, 16, 1024), sdesc_sw128(da + off, 16, 1024),
+                   IDESC_KQ, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < T / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          mma_bf16(tmem + 384, sdesc_sw128(pta + aoff, 16, 1024),
+                   sdesc_sw128(da + kk * 2048, HALF_BYTES, 1024), IDESC_ACC,
+                   (kept_count > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar_mma);
+      }
+      if (!mbar_wait(bar_mma, ph_mma, abort, 0x205)) ok = false;
+      ph_mma ^= 1;
+      if (__syncthreads_or(!ok)) { ok = false; break; }
+      tc_fence_after();
+      // ---- dS^T = P^T o (dP^T - D) * scale -> bf16 ----------------------------
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float dp[32];
+        tmem_ld32(t_dpt + c * 32, dp);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const int q0 = c * 32 + q * 8 + e;
+            const float a = pr[q0] * (dp[q * 8 + e] - dd_s[q0]) * p.scale;
+            const float b = pr[q0 + 1] * (dp[q * 8 + e + 1] - dd_s[q0 + 1]) * p.scale;
+            w[e >> 1] = pack_bf16(a, b);
+          }
+          st_shared_v4(sta + sw128_chunk_off(tid, c * 32 + q * 8, T), w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      // ---- dK += dS^T Q_i ; dQ_i = dS K_j (into the S^T columns) -------------
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < T / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          mma_bf16(tmem + 256, sdesc_sw128(sta + aoff, 16, 1024),
+                   sdesc_sw128(qa + kk * 2048, HALF_BYTES, 1024), IDESC_ACC,
+                   (kept_count > 0 || kk > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < T / 16; ++kk) {
+          mma_bf16(tmem, sdesc_sw128(sta + kk * 2048, HALF_BYTES, 1024),
+                   sdesc_sw128(ka + kk * 2048, HALF_BYTES, 1024), IDESC_DQ, kk > 0);
+        }
+        mma_commit(bar_mma);
+      }
+      if (!mbar_wait(bar_mma, ph_mma, abort, 0x206)) ok = false;
+      ph_mma ^= 1;
+      if (__syncthreads_or(!ok)) { ok = false; break; }
+      tc_fence_after();
+      ++kept_count;
+      // ---- dQ_i rows (lane = query) added into the float32 workspace ----------
+      const int q = i * T + tid;
+      if (q < p.L) {
+        float4* dst = reinterpret_cast<float4*>(p.dQacc + ((size_t)z * p.L + q) * D);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(t_st + c * 32, v);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            atomicAdd(dst + c * 8 + e, make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]));
+        }
+      }
+    }
+    // next query block: Q_i is free once every MMA that read it completed
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && i + 1 < p.nb) {
+      mbar_expect_tx(bar_q, TILE_BYTES);
+      tma_load_3d(qa, &tmQ, 0, (i + 1) * T, z, bar_q);
+      tma_load_3d(qa + HALF_BYTES, &tmQ, 64, (i + 1) * T, z, bar_q);
+    }
+  }
+
+  // ---- epilogue: dK_j, dV_j (bf16); zero if no tile was kept ----------------
+  const int key = j * T + tid;
+  if (ok && key < p.L) {
+    __nv_bfloat16* dk = p.dK + ((size_t)z * p.L + key) * D;
+    __nv_bfloat16* dv = p.dV + ((size_t)z * p.L + key) * D;
+    if (kept_count > 0) {
+      tc_fence_after();
+      store_row_bf16(dk, t_dk);
+      store_row_bf16(dv, t_dv);
+    } else {
+      uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        reinterpret_cast<uint4*>(dk)[c] = zero;
+        reinterpret_cast<uint4*>(dv)[c] = zero;
+      }
+    }
+  }
+  if (tid == 0 && p.kept_tiles) p.kept_tiles[(size_t)z * p.nb + j] = kept_count;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace bwd100
+}  // namespace mala

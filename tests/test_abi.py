@@ -1,0 +1,89 @@
+"""The C ABI without a GPU: the library loads, exports every call that
+include/mala.h declares, and rejects bad arguments on the host before any
+CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import mass_adaptive_causal_b200 as mala
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mala.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mala_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mass_adaptive_causal_b200 import build
+    build.build()
+    return mala.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert {"mala_fwd", "mala_bwd", "mala_decode", "mala_check"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code, name in mala.STATUS.items():
+        assert lib.mala_status_string(code).decode() == name
+    assert lib.mala_version() >= 100
+
+
+def _fwd(lib, ptrs=(16, 16, 16, 16, 16), B=1, H=1, L=256, d=128, dt=1, tau=1.0, tile=128):
+    p = [ctypes.c_void_p(x) if x else None for x in ptrs]
+    return lib.mala_fwd(*p, B, H, L, d, dt, tau, tile, 0.0, None, None, None)
+
+
+def test_fwd_argument_checks(lib):
+    assert _fwd(lib, tau=-1.0) == 1
+    assert _fwd(lib, tau=float("nan")) == 1
+    assert _fwd(lib, tau=float("inf")) == 1
+    assert _fwd(lib, B=0) == 1
+    assert _fwd(lib, L=-1) == 1
+    assert _fwd(lib, d=64) == 2                 # bf16 needs d = 128
+    assert _fwd(lib, tile=64) == 2              # bf16 needs tile 128
+    assert _fwd(lib, dt=0, d=64, tile=128) == 2  # f32 tile is 64
+    assert _fwd(lib, dt=0, d=48, tile=64) == 2
+    assert _fwd(lib, dt=7) == 2
+    assert _fwd(lib, ptrs=(0, 16, 16, 16, 16)) == 1
+    assert _fwd(lib, ptrs=(16, 16, 8, 16, 16)) == 1  # misaligned
+    assert _fwd(lib, L=0) == 0                   # empty input: nothing to do
+    assert _fwd(lib, B=300, H=300) == 1          # grid limit
+
+
+def test_bwd_and_decode_argument_checks(lib):
+    v = ctypes.c_void_p(256)
+    need = lib.mala_bwd_workspace_bytes(1, 2, 1000, 128)
+    assert need == (((2 * 1000 * 4 + 255) // 256) * 256 + ((2 * 1000 * 128 * 4 + 255) // 256) * 256)
+    args = [v] * 10
+    assert lib.mala_bwd(*args, need - 1, 1, 2, 1000, 128, 1, 1.0, 128, 0.0, None, None, None) == 1
+    assert lib.mala_bwd(*args, need, 1, 2, 1000, 128, 1, -0.5, 128, 0.0, None, None, None) == 1
+    assert lib.mala_bwd(*args, need, 1, 2, 0, 128, 1, 1.0, 128, 0.0, None, None, None) == 0
+    ws = lib.mala_decode_workspace_bytes(2, 8, 2, 1000, 128)
+    assert ws > 0
+    dec = lambda Hq, Hkv, d, tau, nbytes: lib.mala_decode(v, v, v, v, 2, Hq, Hkv, 1000, d, tau,
+                                                          0.0, v, nbytes, None, None, None)
+    assert dec(8, 3, 128, 1.0, ws) == 1    # Hq % Hkv
+    assert dec(8, 2, 64, 1.0, ws) == 2     # d
+    assert dec(32, 2, 128, 1.0, 1 << 30) == 2  # group of 16 heads > 8
+    assert dec(8, 2, 128, -1.0, ws) == 1
+    assert dec(8, 2, 128, 1.0, ws - 1) == 1
+
+
+def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import importlib
+    monkeypatch.setattr(mala, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(mala, "_lib", None)
+    with pytest.raises(RuntimeError):
+        mala.lib()

@@ -1,0 +1,233 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs. Every test here needs a B200 and the built library."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.parity import (TOL, as_f64, compare_bwd_keep, compare_decode_keep, compare_fwd_keep,
+                          rel_l2, row_mask)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - CPU container
+    pytest.skip("needs a GPU", allow_module_level=True)
+
+import mass_adaptive_causal_b200 as mala  # noqa: E402
+
+
+def dev_tensor(a, dtype):
+    return torch.tensor(np.ascontiguousarray(a), dtype=torch.float64).to(dtype).cuda()
+
+
+def rounded(t):
+    """The exact values the GPU sees (bf16/f32 -> float64)."""
+    return as_f64(t)
+
+
+def prefill_case(cfg, L=None, heads=None, dtype=torch.bfloat16):
+    x = synth.prefill_inputs(cfg, L=L, heads=heads)
+    t = {n: dev_tensor(x[n], dtype) for n in ("Q", "K", "V", "dO")}
+    return t
+
+
+def check_fwd_slice(Qd, Kd, Vd, O_gpu, LSE_gpu, bits_gpu, tile, tau, tol, qblocks=None):
+    """One (b, h) slice; returns (rows_compared, near_flips)."""
+    L = Qd.shape[0]
+    nb = oracle.n_blocks(L, tile)
+    ref = oracle.fwd(Qd, Kd, Vd, tile=tile, tau=tau, want_margin=True, qblocks=qblocks)
+    lo, hi = (0, nb) if qblocks is None else qblocks
+    gk = mala.unpack_bits(bits_gpu, nb)
+    n_near, bad = compare_fwd_keep(gk[lo:hi], ref["keep"][lo:hi], ref["margin"][lo:hi])
+    bad = [b + lo for b in bad]
+    rows = row_mask(L, tile, bad)
+    sel = np.zeros(L, bool)
+    sel[lo * tile:min(L, hi * tile)] = True
+    rows &= sel
+    assert rel_l2(O_gpu[rows], ref["O"][rows]) <= tol["O"]
+    assert rel_l2(LSE_gpu[rows], ref["LSE"][rows]) <= tol["LSE"]
+    return int(rows.sum()), n_near, ref
+
+
+# ----------------------------------------------------------------------------
+# float32 path (64 x 64 tiles)
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("tau", [1.0, 0.0])
+def test_f32_tiny_config_fwd_bwd(tau):
+    """B=1 H=1 L=1024 d=64 float32, tile 64: the tiny configuration."""
+    cfg = synth.CONFIGS["tiny_f32"]
+    t = prefill_case(cfg, dtype=torch.float32)
+    O, LSE, kept, bits = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True)
+    dQ, dK, dV, kept_b, bits_b = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
+                                               trace=True)
+    mala.mala_check()
+    Qd, Kd, Vd, dOd = (rounded(t[n][0, 0]) for n in ("Q", "K", "V", "dO"))
+    _, n_near, ref = check_fwd_slice(Qd, Kd, Vd, as_f64(O[0, 0]), as_f64(LSE[0, 0]), bits[0, 0],
+                                     64, tau, TOL["f32"])
+    assert n_near == 0
+    nb = 16
+    assert np.array_equal(kept[0, 0].cpu().numpy(), ref["keep"].sum(axis=1))
+    g = oracle.bwd(Qd, Kd, Vd, ref["O"], dOd, ref["LSE"], tile=64, tau=tau, want_margin=True)
+    assert compare_bwd_keep(mala.unpack_bits(bits_b[0, 0], nb), g["keep"], g["margin"]) == 0
+    assert np.array_equal(kept_b[0, 0].cpu().numpy(), g["keep"].sum(axis=0))
+    for n, a in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        assert rel_l2(as_f64(a[0, 0]), g[n]) <= TOL["f32"]["grad"], n
+    if tau == 0.0:
+        dense = oracle.dense_fwd(Qd, Kd, Vd)
+        assert rel_l2(as_f64(O[0, 0]), dense["O"]) <= 1e-5
+
+
+@pytest.mark.parametrize("L,d,B,H", [(1, 64, 1, 1), (63, 32, 2, 1), (65, 64, 1, 3),
+                                     (200, 128, 2, 2), (512, 64, 1, 1)])
+def test_f32_ragged_shapes(L, d, B, H):
+    rng = np.random.default_rng(L * 7 + d)
+    Q = rng.standard_normal((B, H, L, d)) * 2.0
+    K = rng.standard_normal((B, H, L, d)) * 2.0
+    V = rng.standard_normal((B, H, L, d))
+    dO = rng.standard_normal((B, H, L, d))
+    t = {n: dev_tensor(a, torch.float32) for n, a in zip(("Q", "K", "V", "dO"), (Q, K, V, dO))}
+    O, LSE, kept, bits = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, trace=True)
+    dQ, dK, dV = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=1.0)
+    mala.mala_check()
+    for b in range(B):
+        for h in range(H):
+            Qd, Kd, Vd, dOd = (rounded(t[n][b, h]) for n in ("Q", "K", "V", "dO"))
+            _, n_near, ref = check_fwd_slice(Qd, Kd, Vd, as_f64(O[b, h]), as_f64(LSE[b, h]),
+                                             bits[b, h], 64, 1.0, TOL["f32"])
+            assert n_near == 0
+            g = oracle.bwd(Qd, Kd, Vd, ref["O"], dOd, ref["LSE"], tile=64, tau=1.0)
+            for n, a in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+                assert rel_l2(as_f64(a[b, h]), g[n]) <= TOL["f32"]["grad"], n
+
+
+# ----------------------------------------------------------------------------
+# bf16 tcgen05 path (128 x 128 tiles, d = 128)
+# ----------------------------------------------------------------------------
+def run_bf16_prefill(t, tau):
+    O, LSE, kept, bits = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True)
+    dQ, dK, dV, kept_b, bits_b = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
+                                               trace=True)
+    mala.mala_check()
+    return O, LSE, kept, bits, dQ, dK, dV, kept_b, bits_b
+
+
+def check_bf16_slice(t, outs, b, h, tau, grads=True):
+    O, LSE, kept, bits, dQ, dK, dV, kept_b, bits_b = outs
+    Qd, Kd, Vd, dOd = (rounded(t[n][b, h]) for n in ("Q", "K", "V", "dO"))
+    L = Qd.shape[0]
+    nb = oracle.n_blocks(L, 128)
+    _, n_near, ref = check_fwd_slice(Qd, Kd, Vd, as_f64(O[b, h]), as_f64(LSE[b, h]), bits[b, h],
+                                     128, tau, TOL["bf16"])
+    if not grads:
+        return n_near, 0
+    gk = mala.unpack_bits(bits[b, h], nb)
+    _, bad = compare_fwd_keep(gk, ref["keep"], ref["margin"])
+    g = oracle.bwd(Qd, Kd, Vd, ref["O"], dOd, ref["LSE"], tile=128, tau=tau, want_margin=True)
+    n_near_b = compare_bwd_keep(mala.unpack_bits(bits_b[b, h], nb), g["keep"], g["margin"],
+                                skip_blocks=bad)
+    if not bad:
+        for n, a in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+            assert rel_l2(as_f64(a[b, h]), g[n]) <= TOL["bf16"]["grad"], n
+    return n_near, n_near_b
+
+
+@pytest.mark.parametrize("L", [128, 1000, 1536])
+@pytest.mark.parametrize("tau", [1.0, 0.0])
+def test_bf16_small_fwd_bwd(L, tau):
+    cfg = synth.CONFIGS["matched_8k"]
+    t = prefill_case(cfg, L=L, heads=[0, 1])
+    t = {n: v[:, :2].contiguous() for n, v in t.items()}
+    outs = run_bf16_prefill(t, tau)
+    for h in range(2):
+        check_bf16_slice(t, outs, 0, h, tau)
+
+
+def test_bf16_random_inputs_multi_batch():
+    rng = np.random.default_rng(5)
+    B, H, L, d = 2, 2, 700, 128
+    arrs = [rng.standard_normal((B, H, L, d)) * s for s in (1.5, 1.5, 1.0, 1.0)]
+    t = {n: dev_tensor(a, torch.bfloat16) for n, a in zip(("Q", "K", "V", "dO"), arrs)}
+    outs = run_bf16_prefill(t, 1.0)
+    for b in range(B):
+        for h in range(H):
+            check_bf16_slice(t, outs, b, h, 1.0)
+
+
+def test_bf16_matched_work_config_full():
+    """B=1 H=8 L=8192 d=128 bf16 tile 128 tau=1: every head, every output."""
+    cfg = synth.CONFIGS["matched_8k"]
+    t = prefill_case(cfg)
+    outs = run_bf16_prefill(t, 1.0)
+    for h in range(cfg.H):
+        check_bf16_slice(t, outs, 0, h, 1.0)
+
+
+@pytest.mark.parametrize("L", [2048, 16384])
+def test_bf16_sweep_config_sampled_heads(L):
+    """Length-sweep configuration (H=16), tau=1 and tau=0, two heads checked."""
+    cfg = synth.CONFIGS[f"sweep_L{L}"]
+    t = prefill_case(cfg, heads=[0, 9])
+    for tau in (1.0, 0.0):
+        outs = run_bf16_prefill(t, tau)
+        for h in (0, 9):
+            check_bf16_slice(t, outs, 0, h, tau, grads=(L <= 4096 or tau == 1.0))
+
+
+# ----------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------
+def check_decode(q, Kc, Vc, o, kept, bits, tau, groups):
+    B, Hq, d = q.shape
+    Hkv, Lc = Kc.shape[1], Kc.shape[2]
+    G = Hq // Hkv
+    nt = oracle.n_blocks(Lc, 128)
+    for b in sorted(set(g // Hkv for g in groups)):
+        ref = oracle.decode(rounded(q[b]), rounded(Kc[b]), rounded(Vc[b]), tau=tau,
+                            want_margin=True)
+        gk = mala.unpack_bits(bits[b], nt)
+        for g in range(Hkv):
+            if b * Hkv + g not in groups:
+                continue
+            if compare_decode_keep(gk[g], ref["keep"][g], ref["margin"][g]):
+                continue
+            assert kept[b, g].item() == int(ref["keep"][g].sum())
+            sl = slice(g * G, (g + 1) * G)
+            assert rel_l2(as_f64(o[b, sl]), ref["o"][sl]) <= TOL["bf16"]["decode"]
+
+
+@pytest.mark.parametrize("Lc", [1, 127, 128, 1000, 5000])
+@pytest.mark.parametrize("tau", [1.0, 0.0])
+def test_decode_small(Lc, tau):
+    cfg = synth.DecodeConfig("small", 4, 2, 8, 2, Lc, 128, 128, 0.98, max(0, Lc // 256), 4 if Lc > 300 else 0)
+    x = synth.decode_inputs(cfg)
+    q = dev_tensor(x["q"], torch.bfloat16)
+    Kc = dev_tensor(x["K"], torch.bfloat16)
+    Vc = dev_tensor(x["V"], torch.bfloat16)
+    o, kept, bits = mala.mala_decode(q, Kc, Vc, tau=tau, trace=True)
+    mala.mala_check()
+    check_decode(q, Kc, Vc, o, kept, bits, tau, set(range(cfg.B * cfg.Hkv)))
+
+
+def test_decode_group_sizes():
+    rng = np.random.default_rng(3)
+    for Hq, Hkv in ((4, 4), (8, 1), (16, 2)):
+        B, Lc = 1, 3000
+        q = dev_tensor(rng.standard_normal((B, Hq, 128)) * 2, torch.bfloat16)
+        Kc = dev_tensor(rng.standard_normal((B, Hkv, Lc, 128)) * 2, torch.bfloat16)
+        Vc = dev_tensor(rng.standard_normal((B, Hkv, Lc, 128)), torch.bfloat16)
+        o, kept, bits = mala.mala_decode(q, Kc, Vc, tau=1.0, trace=True)
+        mala.mala_check()
+        check_decode(q, Kc, Vc, o, kept, bits, 1.0, set(range(B * Hkv)))
+
+
+def test_empty_and_status():
+    z = torch.empty((1, 1, 0, 128), dtype=torch.bfloat16, device="cuda")
+    O, LSE = mala.mala_fwd(z, z, z)
+    assert O.numel() == 0
+    mala.mala_check()
