@@ -63,11 +63,15 @@ struct Params {
   uint32_t* keep_bits;  // pre-zeroed by the host
 };
 
-__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, uint32_t taddr) {
+// Row of a TMEM accumulator (this thread's lane) -> bf16 global row. Every
+// lane of the warp must call it (tcgen05.ld is warp-collective); `store`
+// masks the global write.
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, uint32_t taddr, bool store) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     float v[32];
     tmem_ld32(taddr + c * 32, v);
+    if (!store) continue;
     uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -249,41 +253,59 @@ __global__ void __launch_bounds__(NT, 1)
       ph_mma ^= 1;
       if (__syncthreads_or(!ok)) { ok = false; break; }
       tc_fence_after();
-      // ---- dS^T = P^T o (dP^T - D) * scale -> bf16 ----------------------------
+      // ---- dS^T = P^T o (dP^T - D) * scale as a bf16 pair hi + lo --------------
+      // dQ sums dS K over keys whose rows of dS cancel (each full row of dS
+      // sums to zero), so a single bf16 rounding of dS costs several percent
+      // of dQ; hi + lo carries ~16 significant bits. lo goes into the P^T
+      // buffer, free now that the dV product has completed.
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float dp[32];
         tmem_ld32(t_dpt + c * 32, dp);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint32_t w[4];
+          uint32_t whi[4], wlo[4];
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
             const int q0 = c * 32 + q * 8 + e;
             const float a = pr[q0] * (dp[q * 8 + e] - dd_s[q0]) * p.scale;
             const float b = pr[q0 + 1] * (dp[q * 8 + e + 1] - dd_s[q0 + 1]) * p.scale;
-            w[e >> 1] = pack_bf16(a, b);
+            const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+            const float2 hf = __bfloat1622float2(h);
+            whi[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+            wlo[e >> 1] = pack_bf16(a - hf.x, b - hf.y);
           }
-          st_shared_v4(sta + sw128_chunk_off(tid, c * 32 + q * 8, T), w[0], w[1], w[2], w[3]);
+          const uint32_t off = sw128_chunk_off(tid, c * 32 + q * 8, T);
+          st_shared_v4(sta + off, whi[0], whi[1], whi[2], whi[3]);
+          st_shared_v4(pta + off, wlo[0], wlo[1], wlo[2], wlo[3]);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
-      // ---- dK += dS^T Q_i ; dQ_i = dS K_j (into the S^T columns) -------------
+      // ---- dK += (hi + lo)^T Q_i ; dQ_i = (hi + lo) K_j (into the S^T columns)
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < T / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          mma_bf16(tmem + 256, sdesc_sw128(sta + aoff, 16, 1024),
-                   sdesc_sw128(qa + kk * 2048, HALF_BYTES, 1024), IDESC_ACC,
-                   (kept_count > 0 || kk > 0) ? 1u : 0u);
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t src = part == 0 ? sta : pta;
+#pragma unroll
+          for (int kk = 0; kk < T / 16; ++kk) {
+            const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+            mma_bf16(tmem + 256, sdesc_sw128(src + aoff, 16, 1024),
+                     sdesc_sw128(qa + kk * 2048, HALF_BYTES, 1024), IDESC_ACC,
+                     (kept_count > 0 || part > 0 || kk > 0) ? 1u : 0u);
+          }
         }
 #pragma unroll
-        for (int kk = 0; kk < T / 16; ++kk) {
-          mma_bf16(tmem, sdesc_sw128(sta + kk * 2048, HALF_BYTES, 1024),
-                   sdesc_sw128(ka + kk * 2048, HALF_BYTES, 1024), IDESC_DQ, kk > 0);
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t src = part == 0 ? sta : pta;
+#pragma unroll
+          for (int kk = 0; kk < T / 16; ++kk) {
+            mma_bf16(tmem, sdesc_sw128(src + kk * 2048, HALF_BYTES, 1024),
+                     sdesc_sw128(ka + kk * 2048, HALF_BYTES, 1024), IDESC_DQ,
+                     (part > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         mma_commit(bar_mma);
       }
@@ -293,13 +315,14 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_after();
       ++kept_count;
       // ---- dQ_i rows (lane = query) added into the float32 workspace ----------
+      // tcgen05.ld is warp-collective: every lane loads, only valid rows add.
       const int q = i * T + tid;
-      if (q < p.L) {
-        float4* dst = reinterpret_cast<float4*>(p.dQacc + ((size_t)z * p.L + q) * D);
+      float4* dst = reinterpret_cast<float4*>(p.dQacc + ((size_t)z * p.L + (q < p.L ? q : 0)) * D);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(t_st + c * 32, v);
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(t_st + c * 32, v);
+        if (q < p.L) {
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             atomicAdd(dst + c * 8 + e, make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]));
@@ -317,15 +340,16 @@ __global__ void __launch_bounds__(NT, 1)
   }
 
   // ---- epilogue: dK_j, dV_j (bf16); zero if no tile was kept ----------------
+  // (TMEM loads are warp-collective: all lanes load, valid key rows store)
   const int key = j * T + tid;
-  if (ok && key < p.L) {
-    __nv_bfloat16* dk = p.dK + ((size_t)z * p.L + key) * D;
-    __nv_bfloat16* dv = p.dV + ((size_t)z * p.L + key) * D;
+  if (ok) {
+    __nv_bfloat16* dk = p.dK + ((size_t)z * p.L + (key < p.L ? key : 0)) * D;
+    __nv_bfloat16* dv = p.dV + ((size_t)z * p.L + (key < p.L ? key : 0)) * D;
     if (kept_count > 0) {
       tc_fence_after();
-      store_row_bf16(dk, t_dk);
-      store_row_bf16(dv, t_dv);
-    } else {
+      store_row_bf16(dk, t_dk, key < p.L);
+      store_row_bf16(dv, t_dv, key < p.L);
+    } else if (key < p.L) {
       uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
