@@ -440,6 +440,41 @@ def oracle_sample(x, budget_s: float):
 
 
 # ---------------------------------------------------------------------------
+def profile_case(args):
+    """A small case of one call for ncu: long_128k recipe at length --L
+    (B=1, H=8; Q/K/V larger than L2 from L=32768), or a decode step with
+    B=4 over a 131072-key cache. Runs `--warmup` untimed launches then
+    `--launches` more and prints their mean time."""
+    import torch
+    import mass_adaptive_causal_b200 as mala
+    torch.cuda.set_device(0)
+    if args.profile in ("fwd", "bwd"):
+        x = synth.prefill_inputs(PREFILL, L=args.L)
+        t = {n: torch.tensor(x[n]).to(torch.bfloat16).cuda() for n in ("Q", "K", "V", "dO")}
+        O, LSE = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0)
+        run = (lambda: mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, out=O, lse=LSE)) \
+            if args.profile == "fwd" else \
+            (lambda: mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=1.0))
+    else:
+        cfg = synth.DecodeConfig("profile", 4, 4, DECODE.Hq, DECODE.Hkv, DECODE.Lc, DECODE.d,
+                                 128, DECODE.rho, DECODE.n_pairs, DECODE.n_query_targets)
+        x = synth.decode_inputs(cfg)
+        q, Kc, Vc = (torch.tensor(x[n]).to(torch.bfloat16).cuda() for n in ("q", "K", "V"))
+        run = lambda: mala.mala_decode(q, Kc, Vc, tau=1.0)
+    for _ in range(args.warmup):
+        run()
+    mala.mala_check()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.launches):
+        run()
+    e.record()
+    torch.cuda.synchronize()
+    mala.mala_check()
+    print(json.dumps({"profile": args.profile, "L": args.L,
+                      "ms_per_launch": s.elapsed_time(e) / args.launches}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -450,7 +485,13 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workers", type=int, default=0)
+    ap.add_argument("--profile", choices=["fwd", "bwd", "decode"], default=None,
+                    help="run only a small case of one call (for ncu captures)")
+    ap.add_argument("--L", type=int, default=32768, help="sequence length of --profile")
+    ap.add_argument("--launches", type=int, default=2, help="timed launches of --profile")
     args = ap.parse_args()
+    if args.profile:
+        return profile_case(args)
     args.warmup = max(3, args.warmup)
 
     rank = int(os.environ.get("RANK", "0"))

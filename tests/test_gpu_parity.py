@@ -117,7 +117,15 @@ def run_bf16_prefill(t, tau):
     return O, LSE, kept, bits, dQ, dK, dV, kept_b, bits_b
 
 
+def bf16_round(a):
+    return torch.tensor(a).to(torch.bfloat16).double().numpy()
+
+
 def check_bf16_slice(t, outs, b, h, tau, grads=True):
+    """Forward against the oracle; backward against the oracle fed the
+    forward output in the path's dtype. The backward's row term
+    D_r = <dO_r, O_r> is defined on the O it is given, and the bf16 path gives
+    it a bf16 O: the oracle's own O rounded to bf16 is that input."""
     O, LSE, kept, bits, dQ, dK, dV, kept_b, bits_b = outs
     Qd, Kd, Vd, dOd = (rounded(t[n][b, h]) for n in ("Q", "K", "V", "dO"))
     L = Qd.shape[0]
@@ -128,7 +136,8 @@ def check_bf16_slice(t, outs, b, h, tau, grads=True):
         return n_near, 0
     gk = mala.unpack_bits(bits[b, h], nb)
     _, bad = compare_fwd_keep(gk, ref["keep"], ref["margin"])
-    g = oracle.bwd(Qd, Kd, Vd, ref["O"], dOd, ref["LSE"], tile=128, tau=tau, want_margin=True)
+    g = oracle.bwd(Qd, Kd, Vd, bf16_round(ref["O"]), dOd, ref["LSE"], tile=128, tau=tau,
+                   want_margin=True)
     n_near_b = compare_bwd_keep(mala.unpack_bits(bits_b[b, h], nb), g["keep"], g["margin"],
                                 skip_blocks=bad)
     if not bad:
