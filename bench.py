@@ -247,6 +247,7 @@ def run_mala(args, rank, world, local_rank):
     Kc = to_dev(x["dK"], (Dc.B, Dc.Hkv, Dc.Lc, Dc.d))
     Vc = to_dev(x["dV"], (Dc.B, Dc.Hkv, Dc.Lc, Dc.d))
     O = torch.empty_like(Q)
+    O32 = torch.empty(Q.shape, dtype=torch.float32, device=dev)
     LSE = torch.empty((P.B, P.H, P.L), dtype=torch.float32, device=dev)
     dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
     o = torch.empty_like(q)
@@ -258,10 +259,10 @@ def run_mala(args, rank, world, local_rank):
     def step(tau, ev=None):
         if ev is not None:
             ev[0].record(stream)
-        mala.mala_fwd(Q, K, V, tau=tau, out=O, lse=LSE)
+        mala.mala_fwd(Q, K, V, tau=tau, out=O, lse=LSE, o32=O32)
         if ev is not None:
             ev[1].record(stream)
-        mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, workspace=ws_b, grads=(dQ, dK, dV))
+        mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, workspace=ws_b, grads=(dQ, dK, dV), o32=O32)
         if ev is not None:
             ev[2].record(stream)
         mala.mala_decode(q, Kc, Vc, tau=tau, workspace=ws_d, out=o)
@@ -308,8 +309,8 @@ def run_mala(args, rank, world, local_rank):
 
     # trace pass (untimed): retained work and kept decode tiles at tau=1 and 0
     def trace(tau):
-        _, _, kept_f, bits_f = mala.mala_fwd(Q, K, V, tau=tau, trace=True)
-        _, _, _, kept_b, bits_b = mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, trace=True)
+        _, _, kept_f, bits_f = mala.mala_fwd(Q, K, V, tau=tau, trace=True, out=O, lse=LSE, o32=O32)[:4]
+        _, _, _, kept_b, bits_b = mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, trace=True, o32=O32)
         _, kept_d, _ = mala.mala_decode(q, Kc, Vc, tau=tau, trace=True)
         mala.mala_check()
         nt = (Dc.Lc + 127) // 128
@@ -359,8 +360,8 @@ def run_e2e(args, x, dev, world, max_over_ranks):
         q_.copy_(hq, non_blocking=True)
         Kc_.copy_(hKc, non_blocking=True)
         Vc_.copy_(hVc, non_blocking=True)
-        O, LSE = mala.mala_fwd(dQ_["Q"], dQ_["K"], dQ_["V"], tau=1.0)
-        dQ, dK, dV = mala.mala_bwd(dQ_["Q"], dQ_["K"], dQ_["V"], O, dQ_["dO"], LSE, tau=1.0)
+        O, LSE, O32 = mala.mala_fwd(dQ_["Q"], dQ_["K"], dQ_["V"], tau=1.0, o32=True)
+        dQ, dK, dV = mala.mala_bwd(dQ_["Q"], dQ_["K"], dQ_["V"], O, dQ_["dO"], LSE, tau=1.0, o32=O32)
         o = mala.mala_decode(q_, Kc_, Vc_, tau=1.0)
         for n, t in (("O", O), ("dQ", dQ), ("dK", dK), ("dV", dV)):
             outs_h[n].copy_(t, non_blocking=True)
@@ -451,10 +452,10 @@ def profile_case(args):
     if args.profile in ("fwd", "bwd"):
         x = synth.prefill_inputs(PREFILL, L=args.L)
         t = {n: torch.tensor(x[n]).to(torch.bfloat16).cuda() for n in ("Q", "K", "V", "dO")}
-        O, LSE = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0)
-        run = (lambda: mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, out=O, lse=LSE)) \
+        O, LSE, O32 = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, o32=True)
+        run = (lambda: mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, out=O, lse=LSE, o32=O32)) \
             if args.profile == "fwd" else \
-            (lambda: mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=1.0))
+            (lambda: mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=1.0, o32=O32))
     else:
         cfg = synth.DecodeConfig("profile", 4, 4, DECODE.Hq, DECODE.Hkv, DECODE.Lc, DECODE.d,
                                  128, DECODE.rho, DECODE.n_pairs, DECODE.n_query_targets)

@@ -73,7 +73,12 @@ typedef enum { MALA_F32 = 0, MALA_BF16 = 1 } mala_dtype;
  * Inputs  Q, K, V: [B][H][L][d] of dtype dt.
  * Outputs O: [B][H][L][d] of dtype dt, softmax over the retained tiles;
  *         LSE: [B][H][L] float32, natural-log normalizer m + ln l over the
- *         retained keys (the only state backward needs).
+ *         retained keys (with O, the only state backward needs);
+ *         O_f32 (may be NULL): [B][H][L][d] float32, the same output before
+ *         rounding to dt. Pass it to mala_bwd: the backward's row terms
+ *         D = <dO, O> feed dQ through a sum over keys whose rows cancel, so
+ *         D computed from a bf16-rounded O costs dQ percents of accuracy when
+ *         keys share a large common component.
  * Trace   kept_tiles: [B][H][nb] kept key tiles per query block;
  *         keep_bits: [B][H][nb][ceil(nb/32)], row = query block, bit = key
  *         block. nb = ceil(L / tile).
@@ -81,7 +86,7 @@ typedef enum { MALA_F32 = 0, MALA_BF16 = 1 } mala_dtype;
  *            any L >= 0 (a ragged last block is masked), B, H >= 1.
  */
 mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O,
-                     float* LSE, int B, int H, int L, int d, mala_dtype dt,
+                     float* LSE, float* O_f32, int B, int H, int L, int d, mala_dtype dt,
                      float tau, int tile, float scale, int32_t* kept_tiles,
                      uint32_t* keep_bits, void* stream);
 
@@ -103,7 +108,9 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
  * Sources: agihunt.info summary, backward paragraph; jaehun.me review,
  * "Backward: offline sparse probabilities".
  *
- * Inputs  Q, K, V, O, dO: [B][H][L][d] of dtype dt; LSE from mala_fwd.
+ * Inputs  Q, K, V, O, dO: [B][H][L][d] of dtype dt; LSE from mala_fwd;
+ *         O_f32 (may be NULL): the float32 output of mala_fwd, used for the
+ *         row terms D instead of O when given.
  * Outputs dQ, dK, dV: [B][H][L][d] of dtype dt (fully overwritten).
  * workspace: device buffer of at least mala_bwd_workspace_bytes(B,H,L,d)
  *         bytes, 256-byte aligned, contents ignored on entry.
@@ -113,7 +120,8 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
  * Supported: as mala_fwd.
  */
 mala_status mala_bwd(const void* Q, const void* K, const void* V,
-                     const void* O, const void* dO, const float* LSE, void* dQ,
+                     const void* O, const float* O_f32, const void* dO,
+                     const float* LSE, void* dQ,
                      void* dK, void* dV, void* workspace,
                      size_t workspace_bytes, int B, int H, int L, int d,
                      mala_dtype dt, float tau, int tile, float scale,
@@ -141,7 +149,8 @@ size_t mala_decode_workspace_bytes(int B, int Hq, int Hkv, int Lc, int d);
  * workspace: at least mala_decode_workspace_bytes(B,Hq,Hkv,Lc,d) bytes.
  * Trace   kept_tiles: [B][Hkv]; keep_bits: [B][Hkv][ceil(nt/32)], nt =
  *         ceil(Lc / 128).
- * Supported: d = 128, Hq % Hkv == 0, 1 <= Hq / Hkv <= 16, Lc >= 1.
+ * Supported: d = 128, Hq % Hkv == 0, 1 <= Hq / Hkv <= 8, B * Hkv <= 4095,
+ *            Lc >= 1.
  */
 mala_status mala_decode(const void* q, const void* Kcache, const void* Vcache,
                         void* o, int B, int Hq, int Hkv, int Lc, int d,

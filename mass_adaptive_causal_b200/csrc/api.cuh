@@ -101,13 +101,14 @@ inline mala_status fwd_f32(const float* Q, const float* K, const float* V, float
 }
 
 inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O, float* LSE,
-                            int Z, int L, float scale, float tau, int32_t* kept, uint32_t* bits,
-                            cudaStream_t s) {
+                            float* O32, int Z, int L, float scale, float tau, int32_t* kept,
+                            uint32_t* bits, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, Q, L, Z) || !make_map(&mk, K, L, Z) || !make_map(&mv, V, L, Z))
     return MALA_ERR_CUDA;
   fwd100::Params p;
   p.O = reinterpret_cast<__nv_bfloat16*>(O);
+  p.O32 = O32;
   p.LSE = LSE;
   p.L = L;
   p.nb = (L + fwd100::T - 1) / fwd100::T;
@@ -143,11 +144,18 @@ inline int blocks_for(size_t n, int per_block, int cap) {
   return (int)(b > (size_t)cap ? cap : (b == 0 ? 1 : b));
 }
 
-inline mala_status bwd_common_pre(const void* O, const void* dO, mala_dtype dt, BwdWorkspace w,
-                                  size_t Z, int L, int d, uint32_t* bits, int nb, cudaStream_t s) {
+inline mala_status bwd_common_pre(const void* O, const float* O32, const void* dO, mala_dtype dt,
+                                  BwdWorkspace w, size_t Z, int L, int d, uint32_t* bits, int nb,
+                                  cudaStream_t s) {
   const size_t rows = Z * (size_t)L;
   const int blocks = blocks_for(rows, 8, 1 << 20);
-  if (dt == MALA_BF16)
+  if (O32 && dt == MALA_BF16)
+    aux::row_dot_mixed_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(dO),
+                                                      O32, w.D, rows, d);
+  else if (O32)
+    aux::row_dot_kernel<float><<<blocks, 256, 0, s>>>(reinterpret_cast<const float*>(dO), O32,
+                                                      w.D, rows, d);
+  else if (dt == MALA_BF16)
     aux::row_dot_bf16_v8_kernel<<<blocks, 256, 0, s>>>(
         reinterpret_cast<const __nv_bfloat16*>(dO), reinterpret_cast<const __nv_bfloat16*>(O),
         w.D, rows, d);
@@ -365,23 +373,29 @@ static mala_status check_prefill_shape(int B, int H, int L, int d, mala_dtype dt
   return MALA_OK;
 }
 
-mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
-                     int H, int L, int d, mala_dtype dt, float tau, int tile, float scale,
-                     int32_t* kept_tiles, uint32_t* keep_bits, void* stream) {
+mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                     float* O_f32, int B, int H, int L, int d, mala_dtype dt, float tau, int tile,
+                     float scale, int32_t* kept_tiles, uint32_t* keep_bits, void* stream) {
   mala_status st = check_prefill_shape(B, H, L, d, dt, tau, tile);
   if (st != MALA_OK) return st;
   if (L == 0) return MALA_OK;
   if (!Q || !K || !V || !O || !LSE) return MALA_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) ||
+      !aligned16(O_f32))
     return MALA_ERR_INVALID_ARG;
   const int Z = B * H;
   const float sc = resolve_scale(scale, d);
   cudaStream_t s = as_stream(stream);
-  if (dt == MALA_F32)
-    return fwd_f32(reinterpret_cast<const float*>(Q), reinterpret_cast<const float*>(K),
-                   reinterpret_cast<const float*>(V), reinterpret_cast<float*>(O), LSE, Z, L, d,
-                   sc, tau, kept_tiles, keep_bits, s);
-  return fwd_bf16(Q, K, V, O, LSE, Z, L, sc, tau, kept_tiles, keep_bits, s);
+  if (dt == MALA_F32) {
+    mala_status st = fwd_f32(reinterpret_cast<const float*>(Q), reinterpret_cast<const float*>(K),
+                             reinterpret_cast<const float*>(V), reinterpret_cast<float*>(O), LSE,
+                             Z, L, d, sc, tau, kept_tiles, keep_bits, s);
+    if (st == MALA_OK && O_f32 && O_f32 != O)
+      MALA_CUDA_TRY(cudaMemcpyAsync(O_f32, O, (size_t)Z * L * d * sizeof(float),
+                                    cudaMemcpyDeviceToDevice, s));
+    return st;
+  }
+  return fwd_bf16(Q, K, V, O, LSE, O_f32, Z, L, sc, tau, kept_tiles, keep_bits, s);
 }
 
 size_t mala_bwd_workspace_bytes(int B, int H, int L, int d) {
@@ -389,8 +403,9 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d) {
   return bwd_ws_bytes((size_t)B * H, (size_t)L, (size_t)d);
 }
 
-mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
-                     const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
+                     const float* O_f32, const void* dO, const float* LSE, void* dQ, void* dK,
+                     void* dV, void* workspace,
                      size_t workspace_bytes, int B, int H, int L, int d, mala_dtype dt, float tau,
                      int tile, float scale, int32_t* kept_tiles, uint32_t* keep_bits,
                      void* stream) {
@@ -402,6 +417,7 @@ mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
   const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV};
   for (const void* p : ptrs)
     if (!aligned16(p)) return MALA_ERR_INVALID_ARG;
+  if (!aligned16(O_f32)) return MALA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MALA_ERR_INVALID_ARG;
   if (workspace_bytes < mala_bwd_workspace_bytes(B, H, L, d)) return MALA_ERR_INVALID_ARG;
   const int Z = B * H;
@@ -409,7 +425,7 @@ mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
   cudaStream_t s = as_stream(stream);
   BwdWorkspace w = bwd_ws_carve(workspace, Z, L);
   const int nb = (L + tile - 1) / tile;
-  st = bwd_common_pre(O, dO, dt, w, Z, L, d, keep_bits, nb, s);
+  st = bwd_common_pre(O, O_f32, dO, dt, w, Z, L, d, keep_bits, nb, s);
   if (st != MALA_OK) return st;
   if (dt == MALA_F32)
     return bwd_f32(reinterpret_cast<const float*>(Q), reinterpret_cast<const float*>(K),

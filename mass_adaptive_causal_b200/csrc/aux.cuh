@@ -56,6 +56,31 @@ __global__ void row_dot_bf16_v8_kernel(const __nv_bfloat16* __restrict__ dO,
   if (lane == 0) D[warp] = s;
 }
 
+// D from the float32 output and a bf16 dO (one warp per row, d % 4 == 0).
+__global__ void row_dot_mixed_kernel(const __nv_bfloat16* __restrict__ dO,
+                                     const float* __restrict__ O32, float* __restrict__ D,
+                                     size_t rows, int d) {
+  const size_t warp = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const uint2* a = reinterpret_cast<const uint2*>(dO + warp * d);
+  const float4* b = reinterpret_cast<const float4*>(O32 + warp * d);
+  float s = 0.f;
+  for (int c = lane; c < d / 4; c += 32) {
+    const uint2 x = a[c];
+    const float4 y = b[c];
+    const float2 x0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
+    const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.y));
+    s = fmaf(x0.x, y.x, s);
+    s = fmaf(x0.y, y.y, s);
+    s = fmaf(x1.x, y.z, s);
+    s = fmaf(x1.y, y.w, s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) D[warp] = s;
+}
+
 template <typename TOut>
 __global__ void convert_kernel(const float* __restrict__ src, TOut* __restrict__ dst, size_t n) {
   for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;

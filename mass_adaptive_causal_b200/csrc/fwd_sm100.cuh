@@ -21,7 +21,11 @@
 // touches neither TMEM's PV columns nor O.
 //
 // Shared memory (1024-byte aligned, 128-byte swizzle, 64-column blocks):
-//   Q_i (32 KB), K_j (32 KB), V_j (32 KB), P (32 KB), barriers.
+//   Q_i (32 KB), K_j (32 KB), V_j (32 KB), P_hi and P_lo (32 KB each).
+// P goes to the tensor cores as a bf16 pair hi + lo (PV = P_hi V + P_lo V),
+// so the float32 output carries P to ~16 significant bits: the backward's
+// row terms D = <dO, O> are computed from that float32 output, and dQ is
+// sensitive to their error.
 // K_{j-1} is prefetched by TMA as soon as the S MMA of tile j has consumed
 // K_j, so its load overlaps the row-max / test of tile j. V_j is requested
 // only after the CTA-wide vote says "keep".
@@ -39,13 +43,14 @@ constexpr int D = 128;
 constexpr int NT = 128;
 constexpr uint32_t TILE_BYTES = T * D * 2;  // 32 KB
 constexpr uint32_t HALF_BYTES = T * 64 * 2; // one 64-column swizzled block
-constexpr uint32_t SMEM_BYTES = 4 * TILE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t SMEM_BYTES = 5 * TILE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, false, true);
 
 struct Params {
   __nv_bfloat16* O;
+  float* O32;  // optional float32 copy of O (nullptr: not written)
   float* LSE;
   int L;
   int nb;
@@ -66,7 +71,8 @@ __global__ void __launch_bounds__(NT, 1)
   unsigned char* k_s = base + TILE_BYTES;
   unsigned char* v_s = base + 2 * TILE_BYTES;
   unsigned char* p_s = base + 3 * TILE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + 4 * TILE_BYTES);
+  unsigned char* pl_s = base + 4 * TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + 5 * TILE_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -78,6 +84,7 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t bar_v = smem_u32(&bars[1]);
   const uint32_t bar_mma = smem_u32(&bars[2]);
   const uint32_t qa = smem_u32(q_s), ka = smem_u32(k_s), va = smem_u32(v_s), pa = smem_u32(p_s);
+  const uint32_t pla = smem_u32(pl_s);
 
   if (tid == 0) {
     mbar_init(bar_qk, 1);
@@ -185,20 +192,24 @@ __global__ void __launch_bounds__(NT, 1)
     for (int c = 0; c < 4; ++c) {
       float s[32];
       tmem_ld32(t_s + c * 32, s);
-      uint32_t pk[16];
+      uint32_t pk[16], pl[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
         const int col = c * 32 + e;
         const float v0 = (diag && col > tid) ? 0.f : exp2f(s[e] * p.scale_log2 - mnew);
         const float v1 = (diag && col + 1 > tid) ? 0.f : exp2f(s[e + 1] * p.scale_log2 - mnew);
         lsum += v0 + v1;
-        pk[e >> 1] = pack_bf16(v0, v1);
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+        const float2 hf = __bfloat1622float2(h);
+        pk[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+        pl[e >> 1] = pack_bf16(v0 - hf.x, v1 - hf.y);
       }
-      // P row tid, keys c*32 .. c*32+31: four 16-byte chunks
+      // P row tid, keys c*32 .. c*32+31: four 16-byte chunks of hi and of lo
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const uint32_t addr = pa + sw128_chunk_off(tid, c * 32 + q * 8, T);
-        st_shared_v4(addr, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        const uint32_t off = sw128_chunk_off(tid, c * 32 + q * 8, T);
+        st_shared_v4(pa + off, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        st_shared_v4(pla + off, pl[4 * q], pl[4 * q + 1], pl[4 * q + 2], pl[4 * q + 3]);
       }
     }
     l = l * alpha + lsum;
@@ -213,11 +224,15 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < T / 16; ++kk) {
-        const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-        const uint32_t boff = kk * 16 * 128;
-        mma_bf16(tmem + 128, sdesc_sw128(pa + aoff, 16, 1024),
-                 sdesc_sw128(va + boff, HALF_BYTES, 1024), IDESC_PV, kk > 0);
+      for (int part = 0; part < 2; ++part) {
+        const uint32_t src = part == 0 ? pa : pla;
+#pragma unroll
+        for (int kk = 0; kk < T / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          const uint32_t boff = kk * 16 * 128;
+          mma_bf16(tmem + 128, sdesc_sw128(src + aoff, 16, 1024),
+                   sdesc_sw128(va + boff, HALF_BYTES, 1024), IDESC_PV, (part > 0 || kk > 0) ? 1u : 0u);
+        }
       }
       mma_commit(bar_mma);
     }
@@ -248,6 +263,12 @@ __global__ void __launch_bounds__(NT, 1)
       w.z = pack_bf16(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
       w.w = pack_bf16(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
       dst[c] = w;
+    }
+    if (p.O32) {
+      float4* d32 = reinterpret_cast<float4*>(p.O32 + ((size_t)z * p.L + row) * D);
+#pragma unroll
+      for (int c = 0; c < D / 4; ++c)
+        d32[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv, o[4 * c + 3] * inv);
     }
     p.LSE[(size_t)z * p.L + row] = (m + __log2f(l)) * kLn2;
   }

@@ -40,7 +40,7 @@ def test_status_strings(lib):
     assert lib.mala_version() >= 100
 
 
-def _fwd(lib, ptrs=(16, 16, 16, 16, 16), B=1, H=1, L=256, d=128, dt=1, tau=1.0, tile=128):
+def _fwd(lib, ptrs=(16, 16, 16, 16, 16, 0), B=1, H=1, L=256, d=128, dt=1, tau=1.0, tile=128):
     p = [ctypes.c_void_p(x) if x else None for x in ptrs]
     return lib.mala_fwd(*p, B, H, L, d, dt, tau, tile, 0.0, None, None, None)
 
@@ -56,8 +56,9 @@ def test_fwd_argument_checks(lib):
     assert _fwd(lib, dt=0, d=64, tile=128) == 2  # f32 tile is 64
     assert _fwd(lib, dt=0, d=48, tile=64) == 2
     assert _fwd(lib, dt=7) == 2
-    assert _fwd(lib, ptrs=(0, 16, 16, 16, 16)) == 1
-    assert _fwd(lib, ptrs=(16, 16, 8, 16, 16)) == 1  # misaligned
+    assert _fwd(lib, ptrs=(0, 16, 16, 16, 16, 0)) == 1
+    assert _fwd(lib, ptrs=(16, 16, 8, 16, 16, 0)) == 1  # misaligned
+    assert _fwd(lib, ptrs=(16, 16, 16, 16, 16, 8)) == 1  # misaligned float32 output
     assert _fwd(lib, L=0) == 0                   # empty input: nothing to do
     assert _fwd(lib, B=300, H=300) == 1          # grid limit
 
@@ -66,7 +67,7 @@ def test_bwd_and_decode_argument_checks(lib):
     v = ctypes.c_void_p(256)
     need = lib.mala_bwd_workspace_bytes(1, 2, 1000, 128)
     assert need == (((2 * 1000 * 4 + 255) // 256) * 256 + ((2 * 1000 * 128 * 4 + 255) // 256) * 256)
-    args = [v] * 10
+    args = [v] * 11
     assert lib.mala_bwd(*args, need - 1, 1, 2, 1000, 128, 1, 1.0, 128, 0.0, None, None, None) == 1
     assert lib.mala_bwd(*args, need, 1, 2, 1000, 128, 1, -0.5, 128, 0.0, None, None, None) == 1
     assert lib.mala_bwd(*args, need, 1, 2, 0, 128, 1, 1.0, 128, 0.0, None, None, None) == 0

@@ -109,11 +109,17 @@ def test_f32_ragged_shapes(L, d, B, H):
 # ----------------------------------------------------------------------------
 # bf16 tcgen05 path (128 x 128 tiles, d = 128)
 # ----------------------------------------------------------------------------
-def run_bf16_prefill(t, tau):
-    O, LSE, kept, bits = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True)
+def run_bf16_prefill(t, tau, use_o32=True):
+    """The training chain: forward (with its float32 output when use_o32),
+    then backward."""
+    O, LSE, kept, bits, *rest = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True,
+                                              o32=use_o32)
+    o32 = rest[0] if use_o32 else None
     dQ, dK, dV, kept_b, bits_b = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
-                                               trace=True)
+                                               trace=True, o32=o32)
     mala.mala_check()
+    if use_o32:  # the float32 output is the bf16 output before rounding
+        assert torch.equal(o32.to(torch.bfloat16), O)
     return O, LSE, kept, bits, dQ, dK, dV, kept_b, bits_b
 
 
@@ -121,11 +127,12 @@ def bf16_round(a):
     return torch.tensor(a).to(torch.bfloat16).double().numpy()
 
 
-def check_bf16_slice(t, outs, b, h, tau, grads=True):
-    """Forward against the oracle; backward against the oracle fed the
-    forward output in the path's dtype. The backward's row term
-    D_r = <dO_r, O_r> is defined on the O it is given, and the bf16 path gives
-    it a bf16 O: the oracle's own O rounded to bf16 is that input."""
+def check_bf16_slice(t, outs, b, h, tau, grads=True, o_rounded=False):
+    """Forward against the oracle; backward against the oracle's backward fed
+    the oracle's own forward output. With ``o_rounded`` (the chain without
+    the float32 output) the backward's row terms D_r = <dO_r, O_r> are
+    defined on the bf16 O it is given, so the oracle is fed its own O rounded
+    to bf16."""
     O, LSE, kept, bits, dQ, dK, dV, kept_b, bits_b = outs
     Qd, Kd, Vd, dOd = (rounded(t[n][b, h]) for n in ("Q", "K", "V", "dO"))
     L = Qd.shape[0]
@@ -136,8 +143,8 @@ def check_bf16_slice(t, outs, b, h, tau, grads=True):
         return n_near, 0
     gk = mala.unpack_bits(bits[b, h], nb)
     _, bad = compare_fwd_keep(gk, ref["keep"], ref["margin"])
-    g = oracle.bwd(Qd, Kd, Vd, bf16_round(ref["O"]), dOd, ref["LSE"], tile=128, tau=tau,
-                   want_margin=True)
+    O_in = bf16_round(ref["O"]) if o_rounded else ref["O"]
+    g = oracle.bwd(Qd, Kd, Vd, O_in, dOd, ref["LSE"], tile=128, tau=tau, want_margin=True)
     n_near_b = compare_bwd_keep(mala.unpack_bits(bits_b[b, h], nb), g["keep"], g["margin"],
                                 skip_blocks=bad)
     if not bad:
@@ -155,6 +162,17 @@ def test_bf16_small_fwd_bwd(L, tau):
     outs = run_bf16_prefill(t, tau)
     for h in range(2):
         check_bf16_slice(t, outs, 0, h, tau)
+
+
+@pytest.mark.parametrize("L", [1000])
+def test_bf16_chain_without_float32_output(L):
+    """Backward with D from the bf16 output (no float32 copy)."""
+    cfg = synth.CONFIGS["matched_8k"]
+    t = prefill_case(cfg, L=L, heads=[0, 1])
+    t = {n: v[:, :2].contiguous() for n, v in t.items()}
+    outs = run_bf16_prefill(t, 1.0, use_o32=False)
+    for h in range(2):
+        check_bf16_slice(t, outs, 0, h, 1.0, o_rounded=True)
 
 
 def test_bf16_random_inputs_multi_batch():
