@@ -112,6 +112,7 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
   p.LSE = LSE;
   p.L = L;
   p.nb = (L + fwd100::T - 1) / fwd100::T;
+  p.npairs = (p.nb + 1) / 2;
   p.scale_log2 = scale * kLog2e;
   p.never_skip = tau == 0.f;
   p.log2_tau = tau > 0.f ? log2f(tau) : 0.f;
@@ -120,7 +121,8 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
   MALA_CUDA_TRY(cudaFuncSetAttribute(fwd100::fwd_bf16_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)fwd100::SMEM_BYTES));
-  fwd100::fwd_bf16_kernel<<<dim3(p.nb, Z), fwd100::NT, fwd100::SMEM_BYTES, s>>>(mq, mk, mv, p);
+  fwd100::fwd_bf16_kernel<<<dim3(p.npairs, Z), fwd100::NT, fwd100::SMEM_BYTES, s>>>(mq, mk, mv,
+                                                                                    p);
   return launch_status();
 }
 

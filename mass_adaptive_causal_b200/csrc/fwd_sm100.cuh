@@ -5,30 +5,35 @@
 // jaehun.me review, "Forward: online sparse softmax"): per query block i the
 // key tiles j = i, i-1, ..., 0 are visited from the diagonal back. Every
 // tile's scores S = Q_i K_j^T are computed on the tensor cores; the tile is
-// skipped iff every valid row r has  mt_r - m_r - ln l_r < ln tau - ln(r+1).
-// Only kept tiles load V_j, update (m, l) and accumulate P V_j. The diagonal
-// tile is always kept; the final log-normalizer goes to LSE.
+// skipped iff every valid row r has  mt_r - m_r - ln l_r < ln tau - ln(r+1),
+// i.e. exp(mt - m) / l < tau / Lq. Only kept tiles load V_j, update (m, l)
+// and accumulate P V_j. The diagonal tile is always kept; the final
+// log-normalizer goes to LSE. Work is in log2 units (s2 = s * scale * log2 e).
 //
-// Work is in the log2 domain (s2 = s * scale * log2 e) so that every
-// exponential is one ex2; the test is the same inequality divided by ln 2.
+// CTA = two query blocks A = 2c and B = 2c + 1 of one (b, h) slice that
+// share every K tile: K_{2c+1} (B's diagonal, B only), then K_{2c} ... K_0
+// for both. Sharing halves the L2 -> SM traffic per tensor-core FLOP.
 //
-// CTA layout (128 threads, one query block): thread t owns query row t, which
-// is TMEM lane t of both accumulators:
-//   TMEM cols [  0,128): S = Q_i K_j^T          (fp32)
-//   TMEM cols [128,256): PV = P_j V_j of the current kept tile (fp32)
-// The output accumulator O lives in the thread's registers (128 floats), so
-// rescaling by exp(m_old - m_new) is a register multiply, and a skipped tile
-// touches neither TMEM's PV columns nor O.
+// Warp roles (320 threads):
+//   warps 0-3  softmax/test warpgroup of A (thread r owns query row r = TMEM lane r)
+//   warps 4-7  softmax/test warpgroup of B
+//   warp  8    TMA producer: Q_A, Q_B, then the K ring (3 stages)
+//   warp  9    MMA issuer (one thread): QK^T and PV, ping-ponging A and B so
+//              the tensor pipe computes one block's scores while the other
+//              block's warpgroup runs its test
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// A kept tile's P = exp2(s2 - m) is written back over its own S columns as
+// bf16 pairs: each 32-column chunk holds 16 columns of P_hi and 16 of P_lo
+// (P = P_hi + P_lo to ~16 bits), and PV = P_hi V + P_lo V reads P from TMEM.
+// O accumulates in TMEM; it is rescaled only when the running max grows by
+// more than 2^8 (the ratio test is exact for any reference max, since
+// exp(mt - m)/l is unchanged by a common shift of m and l).
+// V_j is loaded (by the warpgroup's first thread) only after the warpgroup's
+// vote says "keep"; skipped tiles cost one QK^T and a row max.
 //
-// Shared memory (1024-byte aligned, 128-byte swizzle, 64-column blocks):
-//   Q_i (32 KB), K_j (32 KB), V_j (32 KB), P_hi and P_lo (32 KB each).
-// P goes to the tensor cores as a bf16 pair hi + lo (PV = P_hi V + P_lo V),
-// so the float32 output carries P to ~16 significant bits: the backward's
-// row terms D = <dO, O> are computed from that float32 output, and dQ is
-// sensitive to their error.
-// K_{j-1} is prefetched by TMA as soon as the S MMA of tile j has consumed
-// K_j, so its load overlaps the row-max / test of tile j. V_j is requested
-// only after the CTA-wide vote says "keep".
+// Every mbarrier wait is bounded; a wait that runs out records a timeout in
+// the device status word and the thread carries on, so that no warp is left
+// behind at a named barrier: the kernel always terminates.
 #pragma once
 
 #include "sm100.cuh"
@@ -40,26 +45,84 @@ using namespace sm100;
 
 constexpr int T = 128;
 constexpr int D = 128;
-constexpr int NT = 128;
-constexpr uint32_t TILE_BYTES = T * D * 2;  // 32 KB
-constexpr uint32_t HALF_BYTES = T * 64 * 2; // one 64-column swizzled block
-constexpr uint32_t SMEM_BYTES = 5 * TILE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-constexpr uint32_t TMEM_COLS = 256;
+constexpr int NT = 320;
+constexpr int WARP_PRODUCER = 8;
+constexpr int WARP_MMA = 9;
+constexpr int NSTAGE = 3;
+constexpr uint32_t TILE_BYTES = T * D * 2;   // 32 KB
+constexpr uint32_t HALF_BYTES = T * 64 * 2;  // one 64-column swizzled block
+constexpr uint32_t OFF_Q = 0;                            // Q_A, Q_B
+constexpr uint32_t OFF_K = 2 * TILE_BYTES;               // K ring
+constexpr uint32_t OFF_V = OFF_K + NSTAGE * TILE_BYTES;  // V_A, V_B
+constexpr uint32_t OFF_BAR = OFF_V + 2 * TILE_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
+constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, false, true);
+constexpr float kRescaleLog2 = 8.f;  // lazy O rescale threshold (log2 units)
 
 struct Params {
   __nv_bfloat16* O;
   float* O32;  // optional float32 copy of O (nullptr: not written)
   float* LSE;
   int L;
-  int nb;
-  float scale_log2;  // scale * log2(e)
-  float log2_tau;    // log2(tau); unused when never_skip
-  int never_skip;    // tau == 0
+  int nb;      // query / key blocks
+  int npairs;  // ceil(nb / 2)
+  float scale_log2;
+  float log2_tau;
+  int never_skip;
   int32_t* kept_tiles;
   uint32_t* keep_bits;
 };
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t k_full[NSTAGE];
+  uint64_t k_empty[NSTAGE];
+  uint64_t s_full[2];
+  uint64_t decision[2];
+  uint64_t v_full[2];
+  uint64_t pv_done[2];
+  int keepflag[2];
+  uint32_t tmem_slot;
+  int abort;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
+// OR-vote over one 128-thread warpgroup on named barrier `id`.
+__device__ __forceinline__ int wg_vote_or(int pred, int id) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "barrier.cta.red.or.pred po, %2, 128, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(out)
+      : "r"(pred), "r"(id)
+      : "memory");
+  return (int)out;
+}
+__device__ __forceinline__ void wg_sync(int id) {
+  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
+
+// S_X = Q_X K_t^T (8 MMAs of K = 16), completion signalled on s_full[X].
+__device__ __forceinline__ void issue_qk(Bars& bars, uint32_t sbase, uint32_t tmem, int X, int t) {
+  const uint32_t qa = sbase + OFF_Q + X * TILE_BYTES;
+  const uint32_t ka = sbase + OFF_K + (t % NSTAGE) * TILE_BYTES;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+    mma_bf16(tmem + X * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
+             IDESC_QK, kk > 0);
+  }
+  mma_commit(smem_u32(&bars.s_full[X]));
+}
+
+__device__ __forceinline__ void wait_k_full(Bars& bars, int t, volatile int* abort) {
+  mbar_wait(smem_u32(&bars.k_full[t % NSTAGE]), (t / NSTAGE) & 1, abort, 0x113);
+  tc_fence_after();
+}
 
 __global__ void __launch_bounds__(NT, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -67,218 +130,276 @@ __global__ void __launch_bounds__(NT, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* q_s = base;
-  unsigned char* k_s = base + TILE_BYTES;
-  unsigned char* v_s = base + 2 * TILE_BYTES;
-  unsigned char* p_s = base + 3 * TILE_BYTES;
-  unsigned char* pl_s = base + 4 * TILE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + 5 * TILE_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
-  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
+  Bars& bars = *reinterpret_cast<Bars*>(base + OFF_BAR);
+  volatile int* abort = &bars.abort;
+  const uint32_t sbase = smem_u32(base);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
-  const int i = p.nb - 1 - (int)blockIdx.x;  // longest query blocks first
-  const int z = blockIdx.y;                  // (b, h) slice
-  const uint32_t bar_qk = smem_u32(&bars[0]);
-  const uint32_t bar_v = smem_u32(&bars[1]);
-  const uint32_t bar_mma = smem_u32(&bars[2]);
-  const uint32_t qa = smem_u32(q_s), ka = smem_u32(k_s), va = smem_u32(v_s), pa = smem_u32(p_s);
-  const uint32_t pla = smem_u32(pl_s);
+  const int lane = tid & 31;
+
+  const int c = p.npairs - 1 - (int)blockIdx.x;  // longest pairs first
+  const int z = blockIdx.y;
+  const int iA = 2 * c, iB = 2 * c + 1;
+  const bool hasB = iB < p.nb;
+  const int jtop = hasB ? iB : iA;
+  const int ntiles = jtop + 1;  // tile t <-> key block jtop - t
+  // block X (0 = A, 1 = B) works on tile t iff its query block >= key block
+#define MALA_PART(X, t) ((X) == 0 ? (jtop - (t) <= iA) : hasB)
 
   if (tid == 0) {
-    mbar_init(bar_qk, 1);
-    mbar_init(bar_v, 1);
-    mbar_init(bar_mma, 1);
-    *abort = 0;
+    mbar_init(smem_u32(&bars.q_full), 1);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(smem_u32(&bars.k_full[s]), 1);
+      mbar_init(smem_u32(&bars.k_empty[s]), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(smem_u32(&bars.s_full[x]), 1);
+      mbar_init(smem_u32(&bars.decision[x]), 1);
+      mbar_init(smem_u32(&bars.v_full[x]), 1);
+      mbar_init(smem_u32(&bars.pv_done[x]), 1);
+    }
+    bars.abort = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
   }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+  if (warp == WARP_MMA) {
+    tmem_alloc(smem_u32(&bars.tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const uint32_t t_s = tmem + lane_base;        // this warp's lanes, S columns
-  const uint32_t t_pv = tmem + lane_base + 128; // this warp's lanes, PV columns
+  const uint32_t tmem = bars.tmem_slot;
 
-  if (tid == 0) {
-    mbar_expect_tx(bar_qk, 2 * TILE_BYTES);
-    tma_load_3d(qa, &tmQ, 0, i * T, z, bar_qk);
-    tma_load_3d(qa + HALF_BYTES, &tmQ, 64, i * T, z, bar_qk);
-    tma_load_3d(ka, &tmK, 0, i * T, z, bar_qk);
-    tma_load_3d(ka + HALF_BYTES, &tmK, 64, i * T, z, bar_qk);
-  }
+  if (warp == WARP_PRODUCER) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const uint32_t qb = smem_u32(&bars.q_full);
+      mbar_expect_tx(qb, (hasB ? 2 : 1) * TILE_BYTES);
+      tma_load_3d(sbase + OFF_Q, &tmQ, 0, iA * T, z, qb);
+      tma_load_3d(sbase + OFF_Q + HALF_BYTES, &tmQ, 64, iA * T, z, qb);
+      if (hasB) {
+        tma_load_3d(sbase + OFF_Q + TILE_BYTES, &tmQ, 0, iB * T, z, qb);
+        tma_load_3d(sbase + OFF_Q + TILE_BYTES + HALF_BYTES, &tmQ, 64, iB * T, z, qb);
+      }
+      for (int t = 0; t < ntiles; ++t) {
+        const int s = t % NSTAGE;
+        if (t >= NSTAGE)
+          mbar_wait(smem_u32(&bars.k_empty[s]), ((t / NSTAGE) - 1) & 1, abort, 0x111);
+        const uint32_t kb = smem_u32(&bars.k_full[s]);
+        const uint32_t dst = sbase + OFF_K + s * TILE_BYTES;
+        mbar_expect_tx(kb, TILE_BYTES);
+        tma_load_3d(dst, &tmK, 0, (jtop - t) * T, z, kb);
+        tma_load_3d(dst + HALF_BYTES, &tmK, 64, (jtop - t) * T, z, kb);
+      }
+    }
+    __syncwarp();
+  } else if (warp == WARP_MMA) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      mbar_wait(smem_u32(&bars.q_full), 0, abort, 0x112);
+      uint32_t dec_ph[2] = {0, 0}, v_ph[2] = {0, 0};
+      int pv_count[2] = {0, 0};
+      wait_k_full(bars, 0, abort);
+#pragma unroll
+      for (int X = 0; X < 2; ++X)
+        if (MALA_PART(X, 0)) issue_qk(bars, sbase, tmem, X, 0);
+      mma_commit(smem_u32(&bars.k_empty[0]));
+      for (int t = 0; t < ntiles; ++t) {
+        bool k_next_ready = false;
+#pragma unroll
+        for (int X = 0; X < 2; ++X) {
+          if (MALA_PART(X, t)) {
+            mbar_wait(smem_u32(&bars.decision[X]), dec_ph[X], abort, 0x114);
+            dec_ph[X] ^= 1;
+            if (*reinterpret_cast<volatile int*>(&bars.keepflag[X])) {
+              mbar_wait(smem_u32(&bars.v_full[X]), v_ph[X], abort, 0x115);
+              v_ph[X] ^= 1;
+              tc_fence_after();
+              const uint32_t va = sbase + OFF_V + X * TILE_BYTES;
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                for (int kk = 0; kk < T / 16; ++kk) {
+                  const uint32_t a_t = tmem + X * 128 + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half;
+                  mma_bf16_ts(tmem + 256 + X * 128, a_t,
+                              sdesc_sw128(va + kk * 2048, HALF_BYTES, 1024), IDESC_PV,
+                              (pv_count[X] > 0 || half > 0 || kk > 0) ? 1u : 0u);
+                }
+              }
+              mma_commit(smem_u32(&bars.pv_done[X]));
+              ++pv_count[X];
+            }
+          }
+          if (t + 1 < ntiles && MALA_PART(X, t + 1)) {
+            if (!k_next_ready) {
+              wait_k_full(bars, t + 1, abort);
+              k_next_ready = true;
+            }
+            issue_qk(bars, sbase, tmem, X, t + 1);
+          }
+        }
+        if (t + 1 < ntiles) mma_commit(smem_u32(&bars.k_empty[(t + 1) % NSTAGE]));
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------- softmax / test groups
+    const int X = warp >> 2;  // 0 = A, 1 = B
+    const int r = tid & 127;
+    const int iX = X == 0 ? iA : iB;
+    if (X == 0 || hasB) {
+      const int bar_id = 1 + X;
+      const int row = iX * T + r;
+      const bool row_valid = row < p.L;
+      const float thr = p.never_skip ? 0.f : (p.log2_tau - __log2f((float)(row + 1)));
+      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t t_s = tmem + lane_base + X * 128;
+      const uint32_t t_o = tmem + lane_base + 256 + X * 128;
+      const uint32_t vdst = sbase + OFF_V + X * TILE_BYTES;
+      float m_ref = kNegInf, l = 0.f;
+      int n_kept = 0;
+      uint32_t s_ph = 0;
+      const int nw = (p.nb + 31) >> 5;
+      KeepBits kb;
+      kb.init(r == 0 ? p.keep_bits : nullptr, ((size_t)z * p.nb + iX) * nw);
+      if (r == 0 && p.keep_bits)
+        for (int w = iX / 32 + 1; w < nw; ++w) p.keep_bits[((size_t)z * p.nb + iX) * nw + w] = 0u;
 
-  const int row = i * T + tid;
-  const bool row_valid = row < p.L;
-  const float thr = p.never_skip ? 0.f : (p.log2_tau - __log2f((float)(row + 1)));
-  float m = kNegInf, l = 0.f;
-  float o[D];
+      for (int t = 0; t < ntiles; ++t) {
+        if (!MALA_PART(X, t)) continue;
+        const int j = jtop - t;
+        const bool diag = (j == iX);
+        mbar_wait(smem_u32(&bars.s_full[X]), s_ph, abort, 0x116);
+        s_ph ^= 1;
+        tc_fence_after();
+        // ---- row max of the tile (raw scores: the positive scale commutes)
+        float mraw = kNegInf;
 #pragma unroll
-  for (int e = 0; e < D; ++e) o[e] = 0.f;
-  uint32_t ph_qk = 0, ph_v = 0, ph_mma = 0;
-  int kept_count = 0;
-  const int nw = (p.nb + 31) >> 5;
-  KeepBits kb;
-  kb.init(tid == 0 ? p.keep_bits : nullptr, ((size_t)z * p.nb + i) * nw);
-  if (tid == 0 && p.keep_bits)
-    for (int w = i / 32 + 1; w < nw; ++w) p.keep_bits[((size_t)z * p.nb + i) * nw + w] = 0u;
-
-  bool ok = true;
-  for (int j = i; j >= 0; --j) {
-    // ---- S = Q_i K_j^T on the tensor cores --------------------------------
-    if (!mbar_wait(bar_qk, ph_qk, abort, 0x101)) ok = false;
-    ph_qk ^= 1;
-    if (__syncthreads_or(!ok)) { ok = false; break; }
-    if (tid == 0) {
-      tc_fence_after();
+        for (int ch = 0; ch < 4; ++ch) {
+          float s[32];
+          tmem_ld32(t_s + ch * 32, s);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-        mma_bf16(tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
-                 IDESC_QK, kk > 0);
-      }
-      mma_commit(bar_mma);
-    }
-    if (!mbar_wait(bar_mma, ph_mma, abort, 0x102)) ok = false;
-    ph_mma ^= 1;
-    if (__syncthreads_or(!ok)) { ok = false; break; }
-    tc_fence_after();
-    // K_j consumed: start loading K_{j-1} now
-    if (tid == 0 && j > 0) {
-      mbar_expect_tx(bar_qk, TILE_BYTES);
-      tma_load_3d(ka, &tmK, 0, (j - 1) * T, z, bar_qk);
-      tma_load_3d(ka + HALF_BYTES, &tmK, 64, (j - 1) * T, z, bar_qk);
-    }
-    // ---- row max of the tile and the online test -------------------------
-    const bool diag = (j == i);
-    float mt = kNegInf;
+          for (int e = 0; e < 32; ++e) mraw = fmaxf(mraw, (diag && ch * 32 + e > r) ? kNegInf : s[e]);
+        }
+        const float mt = mraw * p.scale_log2;
+        int want = diag || p.never_skip;
+        if (!want && row_valid) want = (mt - m_ref - __log2f(l)) >= thr;
+        tc_fence_before();
+        const int keep = wg_vote_or(want, bar_id);
+        kb.set(j, keep != 0);
+        if (!keep) {
+          if (r == 0) {
+            bars.keepflag[X] = 0;
+            mbar_arrive(smem_u32(&bars.decision[X]));
+          }
+          continue;
+        }
+        // ---- kept tile ----------------------------------------------------
+        if (n_kept > 0) {  // the previous PV of this block reads V_X and O_X
+          mbar_wait(smem_u32(&bars.pv_done[X]), (n_kept - 1) & 1, abort, 0x117);
+          tc_fence_after();
+        }
+        if (r == 0) {
+          const uint32_t vb = smem_u32(&bars.v_full[X]);
+          mbar_expect_tx(vb, TILE_BYTES);
+          tma_load_3d(vdst, &tmV, 0, j * T, z, vb);
+          tma_load_3d(vdst + HALF_BYTES, &tmV, 64, j * T, z, vb);
+        }
+        const float m_new = fmaxf(m_ref, mt);
+        const bool first = (n_kept == 0);
+        const bool need = !first && (m_new > m_ref + kRescaleLog2);
+        if (first) {
+          m_ref = m_new;
+        } else if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? exp2f(m_ref - m_new) : 1.f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float s[32];
-      tmem_ld32(t_s + c * 32, s);
+          for (int ch = 0; ch < 4; ++ch) {
+            float o[32];
+            tmem_ld32(t_o + ch * 32, o);
+            uint32_t w[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int col = c * 32 + e;
-        const float v = (diag && col > tid) ? kNegInf : s[e] * p.scale_log2;
-        mt = fmaxf(mt, v);
-      }
-    }
-    int want = diag || p.never_skip;
-    if (!want && row_valid) want = (mt - m - __log2f(l)) >= thr;
-    tc_fence_before();
-    const int keep = __syncthreads_or(want);
-    kb.set(j, keep != 0);
-    if (!keep) continue;  // skipped: no V load, no softmax update, no PV
-    ++kept_count;
-    if (tid == 0) {
-      mbar_expect_tx(bar_v, TILE_BYTES);
-      tma_load_3d(va, &tmV, 0, j * T, z, bar_v);
-      tma_load_3d(va + HALF_BYTES, &tmV, 64, j * T, z, bar_v);
-    }
-    // ---- retained tile: P = exp2(s2 - m_new), l and m update -------------
-    const float mnew = fmaxf(m, mt);
-    const float alpha = (m == kNegInf) ? 0.f : exp2f(m - mnew);
-    float lsum = 0.f;
+            for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(o[e] * alpha);
+            tmem_st32(t_o + ch * 32, w);
+          }
+          if (need) {
+            l *= alpha;
+            m_ref = m_new;
+          }
+        }
+        // ---- P = exp2(s2 - m_ref) as hi + lo bf16 pairs over the S columns
+        float lsum = 0.f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float s[32];
-      tmem_ld32(t_s + c * 32, s);
-      uint32_t pk[16], pl[16];
+        for (int ch = 0; ch < 4; ++ch) {
+          float s[32];
+          tmem_ld32(t_s + ch * 32, s);
+          uint32_t w[32];
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const int col = c * 32 + e;
-        const float v0 = (diag && col > tid) ? 0.f : exp2f(s[e] * p.scale_log2 - mnew);
-        const float v1 = (diag && col + 1 > tid) ? 0.f : exp2f(s[e + 1] * p.scale_log2 - mnew);
-        lsum += v0 + v1;
-        const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-        const float2 hf = __bfloat1622float2(h);
-        pk[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
-        pl[e >> 1] = pack_bf16(v0 - hf.x, v1 - hf.y);
-      }
-      // P row tid, keys c*32 .. c*32+31: four 16-byte chunks of hi and of lo
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t off = sw128_chunk_off(tid, c * 32 + q * 8, T);
-        st_shared_v4(pa + off, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        st_shared_v4(pla + off, pl[4 * q], pl[4 * q + 1], pl[4 * q + 2], pl[4 * q + 3]);
-      }
-    }
-    l = l * alpha + lsum;
-    m = mnew;
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // ---- PV = P V_j on the tensor cores ------------------------------------
-    if (!mbar_wait(bar_v, ph_v, abort, 0x103)) ok = false;
-    ph_v ^= 1;
-    if (__syncthreads_or(!ok)) { ok = false; break; }
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t src = part == 0 ? pa : pla;
-#pragma unroll
-        for (int kk = 0; kk < T / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          const uint32_t boff = kk * 16 * 128;
-          mma_bf16(tmem + 128, sdesc_sw128(src + aoff, 16, 1024),
-                   sdesc_sw128(va + boff, HALF_BYTES, 1024), IDESC_PV, (part > 0 || kk > 0) ? 1u : 0u);
+          for (int e = 0; e < 32; e += 2) {
+            const int col = ch * 32 + e;
+            const float p0 = (diag && col > r) ? 0.f : exp2f(s[e] * p.scale_log2 - m_ref);
+            const float p1 = (diag && col + 1 > r) ? 0.f : exp2f(s[e + 1] * p.scale_log2 - m_ref);
+            lsum += p0 + p1;
+            const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+            const float2 hf = __bfloat1622float2(h);
+            w[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+            w[16 + (e >> 1)] = pack_bf16(p0 - hf.x, p1 - hf.y);
+          }
+          tmem_st32(t_s + ch * 32, w);
+        }
+        l += lsum;
+        ++n_kept;
+        tc_fence_before();
+        wg_sync(bar_id);
+        if (r == 0) {
+          bars.keepflag[X] = 1;
+          mbar_arrive(smem_u32(&bars.decision[X]));
         }
       }
-      mma_commit(bar_mma);
-    }
-    if (!mbar_wait(bar_mma, ph_mma, abort, 0x104)) ok = false;
-    ph_mma ^= 1;
-    if (__syncthreads_or(!ok)) { ok = false; break; }
-    tc_fence_after();
+      kb.flush();
+      // ---- epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2 -------------------
+      mbar_wait(smem_u32(&bars.pv_done[X]), (n_kept - 1) & 1, abort, 0x118);
+      tc_fence_after();
+      const float inv = 1.f / l;
+      const size_t orow = ((size_t)z * p.L + (row_valid ? row : 0)) * D;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float pv[32];
-      tmem_ld32(t_pv + c * 32, pv);
+      for (int ch = 0; ch < 4; ++ch) {
+        float o[32];
+        tmem_ld32(t_o + ch * 32, o);
+        if (row_valid) {
+          uint4* d4 = reinterpret_cast<uint4*>(p.O + orow + ch * 32);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) o[c * 32 + e] = fmaf(o[c * 32 + e], alpha, pv[e]);
+          for (int q = 0; q < 4; ++q) {
+            uint4 w;
+            w.x = pack_bf16(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+            w.y = pack_bf16(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+            w.z = pack_bf16(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+            w.w = pack_bf16(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+            d4[q] = w;
+          }
+          if (p.O32) {
+            float4* d32 = reinterpret_cast<float4*>(p.O32 + orow + ch * 32);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              d32[q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv,
+                                   o[4 * q + 3] * inv);
+          }
+        }
+      }
+      if (row_valid) p.LSE[(size_t)z * p.L + row] = (m_ref + __log2f(l)) * kLn2;
+      if (r == 0 && p.kept_tiles) p.kept_tiles[(size_t)z * p.nb + iX] = n_kept;
     }
-    tc_fence_before();
   }
-  kb.flush();
-
-  // ---- epilogue: O = acc / l (bf16), LSE = (m + log2 l) ln 2 ----------------
-  if (ok && row_valid) {
-    const float inv = 1.f / l;
-    uint4* dst = reinterpret_cast<uint4*>(p.O + ((size_t)z * p.L + row) * D);
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      uint4 w;
-      w.x = pack_bf16(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
-      w.y = pack_bf16(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
-      w.z = pack_bf16(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
-      w.w = pack_bf16(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
-      dst[c] = w;
-    }
-    if (p.O32) {
-      float4* d32 = reinterpret_cast<float4*>(p.O32 + ((size_t)z * p.L + row) * D);
-#pragma unroll
-      for (int c = 0; c < D / 4; ++c)
-        d32[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv, o[4 * c + 3] * inv);
-    }
-    p.LSE[(size_t)z * p.L + row] = (m + __log2f(l)) * kLn2;
-  }
-  if (tid == 0 && p.kept_tiles) p.kept_tiles[(size_t)z * p.nb + i] = kept_count;
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+#undef MALA_PART
 }
 
 }  // namespace fwd100
