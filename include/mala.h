@@ -91,8 +91,9 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O,
                      uint32_t* keep_bits, void* stream);
 
 /* Bytes of device workspace mala_bwd needs: the row terms D (float32
- * [B][H][L]) and the float32 dQ accumulator [B][H][L][d], each rounded up to
- * 256 bytes. */
+ * [B][H][L]), the float32 dQ accumulator [B][H][L][d] and the per-tile keep
+ * bits of the backward's test pass (B*H*nb*ceil(nb/32) words for nb =
+ * ceil(L/64)), each rounded up to 256 bytes. */
 size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
 
 /*

@@ -9,6 +9,7 @@
 
 #include "aux.cuh"
 #include "bwd_sm100.cuh"
+#include "bwd_test_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "mala.h"
@@ -130,14 +131,24 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
 struct BwdWorkspace {
   float* D;
   float* dQacc;
+  uint32_t* bits;  // per-tile keep bits of the test pass (sized for 64-row tiles)
 };
-inline size_t bwd_ws_bytes(size_t Z, size_t L, size_t d) {
-  return round256(Z * L * sizeof(float)) + round256(Z * L * d * sizeof(float));
+inline size_t bwd_bits_words(size_t Z, size_t L) {
+  const size_t nb = (L + 63) / 64;
+  return Z * nb * ((nb + 31) / 32);
 }
-inline BwdWorkspace bwd_ws_carve(void* ws, size_t Z, size_t L) {
+inline size_t bwd_ws_bytes(size_t Z, size_t L, size_t d) {
+  return round256(Z * L * sizeof(float)) + round256(Z * L * d * sizeof(float)) +
+         round256(bwd_bits_words(Z, L) * sizeof(uint32_t));
+}
+inline BwdWorkspace bwd_ws_carve(void* ws, size_t Z, size_t L, size_t d) {
   BwdWorkspace w;
-  w.D = reinterpret_cast<float*>(ws);
-  w.dQacc = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round256(Z * L * sizeof(float)));
+  char* c = reinterpret_cast<char*>(ws);
+  w.D = reinterpret_cast<float*>(c);
+  c += round256(Z * L * sizeof(float));
+  w.dQacc = reinterpret_cast<float*>(c);
+  c += round256(Z * L * d * sizeof(float));
+  w.bits = reinterpret_cast<uint32_t*>(c);
   return w;
 }
 
@@ -209,6 +220,29 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
   if (!make_map(&mq, Q, L, Z) || !make_map(&mk, K, L, Z) || !make_map(&mv, V, L, Z) ||
       !make_map(&mdo, dO, L, Z))
     return MALA_ERR_CUDA;
+  const int nb = (L + bwd100::T - 1) / bwd100::T;
+  const int never = tau == 0.f;
+  uint32_t* tile_bits = bits ? bits : w.bits;
+  if (!never) {
+    // pass 1: the offline test of every legal tile -> one bit per tile
+    bwdtest::Params tp;
+    tp.LSE = LSE;
+    tp.L = L;
+    tp.nb = nb;
+    tp.npairs = (nb + 1) / 2;
+    tp.scale_log2 = scale * kLog2e;
+    tp.log2_tau = log2f(tau);
+    tp.bits = tile_bits;
+    MALA_CUDA_TRY(cudaFuncSetAttribute(bwdtest::test_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bwdtest::SMEM_BYTES));
+    bwdtest::test_kernel<<<dim3(tp.npairs, Z), bwdtest::NT, bwdtest::SMEM_BYTES, s>>>(mq, mk, tp);
+  } else if (bits) {
+    const size_t nwords = (size_t)Z * nb * ((nb + 31) / 32);
+    aux::lower_bits_kernel<<<blocks_for(nwords, 256, 4 * sm_count()), 256, 0, s>>>(bits, nb,
+                                                                                 nwords);
+  }
+  // pass 2: post-score work of the kept tiles, one CTA per key block
   bwd100::Params p;
   p.LSE = LSE;
   p.Dterm = w.D;
@@ -216,13 +250,12 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
   p.dK = reinterpret_cast<__nv_bfloat16*>(dK);
   p.dV = reinterpret_cast<__nv_bfloat16*>(dV);
   p.L = L;
-  p.nb = (L + bwd100::T - 1) / bwd100::T;
+  p.nb = nb;
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
-  p.never_skip = tau == 0.f;
-  p.log2_tau = tau > 0.f ? log2f(tau) : 0.f;
+  p.never_skip = never;
   p.kept_tiles = kept;
-  p.keep_bits = bits;
+  p.bits = tile_bits;
   MALA_CUDA_TRY(cudaFuncSetAttribute(bwd100::bwd_bf16_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)bwd100::SMEM_BYTES));
@@ -425,7 +458,7 @@ mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
   const int Z = B * H;
   const float sc = resolve_scale(scale, d);
   cudaStream_t s = as_stream(stream);
-  BwdWorkspace w = bwd_ws_carve(workspace, Z, L);
+  BwdWorkspace w = bwd_ws_carve(workspace, Z, L, d);
   const int nb = (L + tile - 1) / tile;
   st = bwd_common_pre(O, O_f32, dO, dt, w, Z, L, d, keep_bits, nb, s);
   if (st != MALA_OK) return st;

@@ -107,6 +107,21 @@ __global__ void zero_kernel(float4* __restrict__ p, size_t n4) {
     p[e] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
+// Keep bits when every legal tile is kept: row i has bits j = 0..i set.
+__global__ void lower_bits_kernel(uint32_t* __restrict__ bits, int nb, size_t nwords) {
+  const int nw = (nb + 31) / 32;
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < nwords;
+       e += (size_t)gridDim.x * blockDim.x) {
+    const int w = (int)(e % nw);
+    const int i = (int)((e / nw) % nb);
+    const int lo = w * 32;
+    uint32_t v = 0u;
+    if (i >= lo + 31) v = 0xffffffffu;
+    else if (i >= lo) v = (uint32_t)((1ull << (i - lo + 1)) - 1ull);
+    bits[e] = v;
+  }
+}
+
 __global__ void zero_u32_kernel(uint32_t* __restrict__ p, size_t n) {
   for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
        e += (size_t)gridDim.x * blockDim.x)

@@ -1,29 +1,28 @@
-// bwd_sm100.cuh -- MALA backward for bf16, d = 128, 128 x 128 tiles on the
-// 5th-generation tensor cores (tcgen05 + TMEM), operands staged by TMA.
+// bwd_sm100.cuh -- MALA backward work pass for bf16, d = 128, 128 x 128
+// tiles on the 5th-generation tensor cores (tcgen05 + TMEM), operands staged
+// by TMA.
 //
 // Rule (MassAlloc Attention; agihunt.info summary, backward paragraph;
 // jaehun.me review, "Backward: offline sparse probabilities"): the backward
-// reuses the forward's final log-normalizer LSE. For every legal tile (query
-// block i, key block j) the scores are recomputed and the tile is skipped iff
-// every valid query row r has  max_c S_rc - LSE_r < ln tau - ln(r+1).
-// Only kept tiles load dO_i and do the post-score work
+// reuses the forward's final log-normalizer LSE; a tile whose every valid row
+// has max_c S_rc - LSE_r < ln tau - ln(r+1) is skipped. The test of every
+// legal tile runs first (bwd_test_sm100.cuh) and leaves one bit per tile;
+// this pass does the post-score work of the kept tiles only:
 //   P = exp(S - LSE), dV_j += P^T dO_i, dP = dO_i V_j^T, dS = P o (dP - D),
 //   dK_j += scale dS^T Q_i, dQ_i += scale dS K_j.
 //
-// The test "every row below its threshold" is evaluated per key instead of
-// per query: keep iff some (query q, key k) has S_qk >= LSE_q + ln tau -
-// ln(q+1). With the scores transposed (keys in TMEM lanes) each thread checks
-// its own key against the 128 per-query thresholds, then the CTA votes.
-//
-// CTA (128 threads) = one key block j, looping over query blocks i >= j.
-// Thread t owns key row t = TMEM lane t for the key-major products:
-//   TMEM [  0,128): S^T = K_j Q_i^T, later reused for dQ_i = dS K_j
+// CTA (128 threads) = one key block j: it lists the kept query blocks
+// i >= j of its column of the bit matrix, then for each: loads Q_i and dO_i,
+// recomputes S^T = K_j Q_i^T with keys in TMEM lanes (thread t owns key t),
+// and accumulates dK_j, dV_j in TMEM:
+//   TMEM [  0,128): S^T, later reused for dQ_i = dS K_j
 //   TMEM [128,256): dP^T = V_j dO_i^T
 //   TMEM [256,384): dK_j accumulator      TMEM [384,512): dV_j accumulator
 // Shared memory: K_j, V_j, Q_i, dO_i, P^T, dS^T (32 KB each, 128-byte
-// swizzle) + the per-query thresholds and D terms.
-// dQ_i is read back from TMEM (query rows in lanes) and added with float4
-// atomics into a float32 workspace; a separate kernel converts it to bf16.
+// swizzle) + per-query LSE and D, and the list of kept query blocks.
+// dS goes to the tensor cores as a bf16 pair hi + lo (dQ sums rows of dS
+// that cancel); dQ_i is read back from TMEM (query rows in lanes) and added
+// with float4 atomics into a float32 workspace, converted afterwards.
 #pragma once
 
 #include "sm100.cuh"
@@ -38,7 +37,9 @@ constexpr int D = 128;
 constexpr int NT = 128;
 constexpr uint32_t TILE_BYTES = T * D * 2;
 constexpr uint32_t HALF_BYTES = T * 64 * 2;
-constexpr uint32_t SMEM_BYTES = 6 * TILE_BYTES + 1024 /*align*/ + 2048 /*thresholds*/ + 256;
+constexpr int LIST_CHUNK = 1024;  // query blocks listed per round
+constexpr uint32_t SMEM_BYTES = 6 * TILE_BYTES + 1024 /*align*/ + 2048 /*LSE, D*/ + 256 +
+                                LIST_CHUNK * 4 + 64;
 constexpr uint32_t TMEM_COLS = 512;
 // S^T, dP^T: A = K_j or V_j (K-major over d), B = Q_i or dO_i (K-major over d)
 constexpr uint32_t IDESC_KQ = idesc_bf16(128, 128, false, false);
@@ -57,10 +58,9 @@ struct Params {
   int nb;
   float scale;       // softmax scale (dS is scaled before the bf16 cast)
   float scale_log2;  // scale * log2(e)
-  float log2_tau;
-  int never_skip;
+  int never_skip;    // tau == 0: every legal tile is kept (no bits read)
   int32_t* kept_tiles;
-  uint32_t* keep_bits;  // pre-zeroed by the host
+  const uint32_t* bits;  // [Z][nb][nw] from the test pass
 };
 
 // Row of a TMEM accumulator (this thread's lane) -> bf16 global row. Every
@@ -98,12 +98,13 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t da = ka + 3 * TILE_BYTES;   // dO_i
   const uint32_t pta = ka + 4 * TILE_BYTES;  // P^T
   const uint32_t sta = ka + 5 * TILE_BYTES;  // dS^T
-  float* thr_s = reinterpret_cast<float*>(base + 6 * TILE_BYTES);  // [128] LSE2 + log2 thr
-  float* lse_s = thr_s + T;                                        // [128] LSE2
-  float* dd_s = lse_s + T;                                         // [128] D
-  uint64_t* bars = reinterpret_cast<uint64_t*>(dd_s + T + 128);
+  float* lse_s = reinterpret_cast<float*>(base + 6 * TILE_BYTES);  // [128] LSE2
+  float* dd_s = lse_s + T;                                          // [128] D
+  uint64_t* bars = reinterpret_cast<uint64_t*>(dd_s + T + 256);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* list = reinterpret_cast<int*>(bars + 8);  // [LIST_CHUNK]
+  int* wcount = list + LIST_CHUNK;               // [4]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -111,13 +112,11 @@ __global__ void __launch_bounds__(NT, 1)
   const int z = blockIdx.y;
   const uint32_t bar_kv = smem_u32(&bars[0]);
   const uint32_t bar_q = smem_u32(&bars[1]);
-  const uint32_t bar_do = smem_u32(&bars[2]);
   const uint32_t bar_mma = smem_u32(&bars[3]);
 
   if (tid == 0) {
     mbar_init(bar_kv, 1);
     mbar_init(bar_q, 1);
-    mbar_init(bar_do, 1);
     mbar_init(bar_mma, 1);
     *abort = 0;
     fence_mbar_init();
@@ -143,25 +142,45 @@ __global__ void __launch_bounds__(NT, 1)
     tma_load_3d(ka + HALF_BYTES, &tmK, 64, j * T, z, bar_kv);
     tma_load_3d(va, &tmV, 0, j * T, z, bar_kv);
     tma_load_3d(va + HALF_BYTES, &tmV, 64, j * T, z, bar_kv);
-    mbar_expect_tx(bar_q, TILE_BYTES);
-    tma_load_3d(qa, &tmQ, 0, j * T, z, bar_q);
-    tma_load_3d(qa + HALF_BYTES, &tmQ, 64, j * T, z, bar_q);
   }
-  uint32_t ph_q = 0, ph_do = 0, ph_mma = 0;
+  uint32_t ph_q = 0, ph_mma = 0;
   int kept_count = 0;
   bool ok = mbar_wait(bar_kv, 0, abort, 0x201);
   const int nw = (p.nb + 31) >> 5;
+  const int lane = tid & 31;
 
-  for (int i = j; i < p.nb && ok; ++i) {
-    // per-query thresholds of this block (log2 domain)
+  for (int i0 = j; i0 < p.nb && ok; i0 += LIST_CHUNK) {
+    // ---- list the kept query blocks i in [i0, i0 + LIST_CHUNK), ascending
+    int n_list = 0;
+    for (int k = 0; k < LIST_CHUNK / NT; ++k) {
+      const int i = i0 + k * NT + tid;
+      bool f = false;
+      if (i < p.nb)
+        f = p.never_skip ||
+            ((p.bits[((size_t)z * p.nb + i) * nw + (j >> 5)] >> (j & 31)) & 1u);
+      const unsigned bal = __ballot_sync(0xffffffffu, f);
+      if (lane == 0) wcount[warp] = __popc(bal);
+      __syncthreads();
+      int off = n_list;
+      for (int w = 0; w < warp; ++w) off += wcount[w];
+      if (f) list[off + __popc(bal & ((1u << lane) - 1u))] = i;
+      n_list += wcount[0] + wcount[1] + wcount[2] + wcount[3];
+      __syncthreads();
+    }
+    for (int li = 0; li < n_list && ok; ++li) {
+    const int i = list[li];
     {
       const int q = i * T + tid;
       const bool qv = q < p.L;
-      const float lse2 = qv ? p.LSE[(size_t)z * p.L + q] * kLog2e : 0.f;
-      lse_s[tid] = lse2;
+      lse_s[tid] = qv ? p.LSE[(size_t)z * p.L + q] * kLog2e : 0.f;
       dd_s[tid] = qv ? p.Dterm[(size_t)z * p.L + q] : 0.f;
-      thr_s[tid] = !qv ? __int_as_float(0x7f800000)
-                       : (p.never_skip ? kNegInf : lse2 + p.log2_tau - __log2f((float)(q + 1)));
+    }
+    if (tid == 0) {
+      mbar_expect_tx(bar_q, 2 * TILE_BYTES);
+      tma_load_3d(qa, &tmQ, 0, i * T, z, bar_q);
+      tma_load_3d(qa + HALF_BYTES, &tmQ, 64, i * T, z, bar_q);
+      tma_load_3d(da, &tmdO, 0, i * T, z, bar_q);
+      tma_load_3d(da + HALF_BYTES, &tmdO, 64, i * T, z, bar_q);
     }
     if (!mbar_wait(bar_q, ph_q, abort, 0x202)) ok = false;
     ph_q ^= 1;
@@ -181,30 +200,8 @@ __global__ void __launch_bounds__(NT, 1)
     ph_mma ^= 1;
     if (__syncthreads_or(!ok)) { ok = false; break; }
     tc_fence_after();
-    // ---- offline test: does this key reach any query's threshold? ----------
     const bool diag = (i == j);
-    int want = 0;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float s[32];
-      tmem_ld32(t_st + c * 32, s);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int qc = c * 32 + e;
-        const bool legal = !diag || qc >= tid;
-        want |= (legal && s[e] * p.scale_log2 >= thr_s[qc]);
-      }
-    }
-    tc_fence_before();
-    const int keep = __syncthreads_or(want);
-    if (tid == 0 && keep && p.keep_bits)
-      atomicOr(&p.keep_bits[((size_t)z * p.nb + i) * nw + (j >> 5)], 1u << (j & 31));
-    if (keep) {
-      if (tid == 0) {
-        mbar_expect_tx(bar_do, TILE_BYTES);
-        tma_load_3d(da, &tmdO, 0, i * T, z, bar_do);
-        tma_load_3d(da + HALF_BYTES, &tmdO, 64, i * T, z, bar_do);
-      }
+    {
       // P^T row (key tid) over the block's queries, fp32 kept for dS
       float pr[T];
 #pragma unroll
@@ -228,9 +225,6 @@ __global__ void __launch_bounds__(NT, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
-      if (!mbar_wait(bar_do, ph_do, abort, 0x204)) ok = false;
-      ph_do ^= 1;
-      if (__syncthreads_or(!ok)) { ok = false; break; }
       // ---- dP^T = V_j dO_i^T ; dV += P^T dO_i ---------------------------------
       if (tid == 0) {
         tc_fence_after();
@@ -329,13 +323,9 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
     }
-    // next query block: Q_i is free once every MMA that read it completed
+    // Q_i, dO_i and the TMEM columns are free once every MMA above completed
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && i + 1 < p.nb) {
-      mbar_expect_tx(bar_q, TILE_BYTES);
-      tma_load_3d(qa, &tmQ, 0, (i + 1) * T, z, bar_q);
-      tma_load_3d(qa + HALF_BYTES, &tmQ, 64, (i + 1) * T, z, bar_q);
     }
   }
 
