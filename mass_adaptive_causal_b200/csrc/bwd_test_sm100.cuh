@@ -187,14 +187,7 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_wait(smem_u32(&bars.s_full[X]), s_ph, abort, 0x215);
         s_ph ^= 1;
         tc_fence_after();
-        float mraw = kNegInf;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          float s[32];
-          tmem_ld32(t_s + ch * 32, s);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mraw = fmaxf(mraw, (diag && ch * 32 + e > r) ? kNegInf : s[e]);
-        }
+        const float mraw = tmem_rowmax128(t_s, diag, r);
         tc_fence_before();
         const int keep = wg_vote_or(mraw >= craw, bar_id);
         kb.set(j, keep != 0);

@@ -31,7 +31,7 @@ using namespace sm100;
 constexpr int T = 128;
 constexpr int D = 128;
 constexpr int NT = 128;  // 4 warps x 32 keys
-constexpr int NST = 4;   // TMA ring depth of the stats pass
+constexpr int NST = 6;   // TMA ring depth of the stats pass
 constexpr int GMAX = 8;  // heads per KV group (the mma N dimension)
 constexpr uint32_t TILE_BYTES = T * D * 2;
 constexpr uint32_t HALF_BYTES = T * 64 * 2;
@@ -78,12 +78,15 @@ __device__ __forceinline__ void warp_scores(uint32_t tile, const uint32_t (&bq)[
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int mb = 0; mb < 2; ++mb) {
+  for (int mb = 0; mb < 2; ++mb)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[mb][e] = 0.f;
-    const int r = warp * 32 + mb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  // two independent accumulation chains (mb = 0, 1) interleaved over ks
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
+  for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+    for (int mb = 0; mb < 2; ++mb) {
+      const int r = warp * 32 + mb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
       const int c = ks * 16 + (lane >> 4) * 8;
       uint32_t a0, a1, a2, a3;
       ldsm_x4(tile + sw128_chunk_off(r, c, T), a0, a1, a2, a3);

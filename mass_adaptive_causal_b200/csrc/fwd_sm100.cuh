@@ -277,14 +277,7 @@ __global__ void __launch_bounds__(NT, 1)
         s_ph ^= 1;
         tc_fence_after();
         // ---- row max of the tile (raw scores: the positive scale commutes)
-        float mraw = kNegInf;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          float s[32];
-          tmem_ld32(t_s + ch * 32, s);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mraw = fmaxf(mraw, (diag && ch * 32 + e > r) ? kNegInf : s[e]);
-        }
+        const float mraw = tmem_rowmax128(t_s, diag, r);
         const float mt = mraw * p.scale_log2;
         int want = diag || p.never_skip;
         if (!want && row_valid) want = (mt - m_ref - __log2f(l)) >= thr;
