@@ -326,8 +326,8 @@ inline mala_status decode_bf16(const void* q, const void* Kc, const void* Vc, vo
   sp.scale_log2 = scale_log2;
   const int grid_a = (int)((sp.total_tiles + sp.tiles_per_cta - 1) / sp.tiles_per_cta);
   MALA_CUDA_TRY(cudaFuncSetAttribute(dec::stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)dec::STATS_SMEM));
-  dec::stats_kernel<<<grid_a, dec::NT, dec::STATS_SMEM, s>>>(mk, sp);
+                                     (int)dec::STATS_RING_SMEM));
+  dec::stats_kernel<<<grid_a, dec::STATS_NT, dec::STATS_RING_SMEM, s>>>(mk, sp);
 
   dec::ScanParams cp;
   cp.stats = w.stats;

@@ -31,11 +31,9 @@ using namespace sm100;
 constexpr int T = 128;
 constexpr int D = 128;
 constexpr int NT = 128;  // 4 warps x 32 keys
-constexpr int NST = 6;   // TMA ring depth of the stats pass
 constexpr int GMAX = 8;  // heads per KV group (the mma N dimension)
 constexpr uint32_t TILE_BYTES = T * D * 2;
 constexpr uint32_t HALF_BYTES = T * 64 * 2;
-constexpr uint32_t STATS_SMEM = NST * TILE_BYTES + 1024 + 1024;
 constexpr uint32_t PV_SMEM = 2 * TILE_BYTES + 1024 + GMAX * T * 4 + 4096 * 4 + 256;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& a0, uint32_t& a1, uint32_t& a2,
@@ -104,15 +102,24 @@ struct StatsParams {
   float scale_log2;
 };
 
-__global__ void __launch_bounds__(NT) stats_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                   const StatsParams p) {
+constexpr int STATS_CONSUMERS = 8;                    // warps, one whole tile each
+constexpr int STATS_NT = 32 * (STATS_CONSUMERS + 1);  // + one TMA producer warp
+constexpr int STATS_NST = 6;                          // TMA ring depth
+constexpr uint32_t STATS_RING_SMEM = STATS_NST * TILE_BYTES + 1024 + 256;
+
+// Phase A: one CTA per SM streams a contiguous run of tiles. Warp 8 keeps a
+// 6-stage TMA ring full; consumer warp w handles tiles w, w+8, ... of the run
+// entirely by itself (8 m16 blocks x 8 k-steps of mma.sync against the
+// group's query heads), so no CTA-wide barrier sits on the stream.
+__global__ void __launch_bounds__(STATS_NT) stats_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                         const StatsParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t ring = smem_u32(base);
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + NST * TILE_BYTES);
-  float* red = reinterpret_cast<float*>(full + NST);  // [4 warps][8 heads] x 2
-  volatile int* abort = reinterpret_cast<volatile int*>(red + 64);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + STATS_NST * TILE_BYTES);
+  uint64_t* empty = full + STATS_NST;
+  volatile int* abort = reinterpret_cast<volatile int*>(empty + STATS_NST);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   const long long begin = (long long)blockIdx.x * p.tiles_per_cta;
@@ -122,45 +129,70 @@ __global__ void __launch_bounds__(NT) stats_kernel(const __grid_constant__ CUten
   const int count = (int)(end - begin);
 
   if (tid == 0) {
-    for (int s = 0; s < NST; ++s) mbar_init(smem_u32(&full[s]), 1);
+    for (int s = 0; s < STATS_NST; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
     *abort = 0;
     fence_mbar_init();
   }
   __syncthreads();
-  auto issue = [&](int k) {
-    const long long flat = begin + k;
-    const int grp = (int)(flat / p.nt), t = (int)(flat % p.nt);
-    const int s = k % NST;
-    const uint32_t bar = smem_u32(&full[s]);
-    mbar_expect_tx(bar, TILE_BYTES);
-    tma_load_3d(ring + s * TILE_BYTES, &tmK, 0, t * T, grp, bar);
-    tma_load_3d(ring + s * TILE_BYTES + HALF_BYTES, &tmK, 64, t * T, grp, bar);
-  };
-  if (tid == 0)
-    for (int k = 0; k < NST && k < count; ++k) issue(k);
+
+  if (warp == STATS_CONSUMERS) {
+    if (lane == 0) {
+      for (int k = 0; k < count; ++k) {
+        const int s = k % STATS_NST;
+        if (k >= STATS_NST)
+          mbar_wait(smem_u32(&empty[s]), ((k / STATS_NST) - 1) & 1, abort, 0x300);
+        const long long flat = begin + k;
+        const int grp = (int)(flat / p.nt), t = (int)(flat % p.nt);
+        const uint32_t bar = smem_u32(&full[s]);
+        mbar_expect_tx(bar, TILE_BYTES);
+        tma_load_3d(ring + s * TILE_BYTES, &tmK, 0, t * T, grp, bar);
+        tma_load_3d(ring + s * TILE_BYTES + HALF_BYTES, &tmK, 64, t * T, grp, bar);
+      }
+    }
+    return;
+  }
 
   uint32_t bq[8][2];
   int cur_grp = -1;
   const int n0 = (lane & 3) * 2;
-  for (int k = 0; k < count; ++k) {
+  for (int k = warp; k < count; k += STATS_CONSUMERS) {
     const long long flat = begin + k;
     const int grp = (int)(flat / p.nt), t = (int)(flat % p.nt);
     if (grp != cur_grp) {
       load_q_frags(p.q, grp, p.G, bq);
       cur_grp = grp;
     }
-    const int s = k % NST;
-    const bool ok = mbar_wait(smem_u32(&full[s]), (k / NST) & 1, abort, 0x301);
-    if (__syncthreads_or(!ok)) break;
-    float acc[2][4];
-    warp_scores(ring + s * TILE_BYTES, bq, acc);
-    // mask keys beyond the cache (ragged last tile), scale to log2 units
+    const int s = k % STATS_NST;
+    mbar_wait(smem_u32(&full[s]), (k / STATS_NST) & 1, abort, 0x301);
+    const uint32_t tile = ring + s * TILE_BYTES;
+    // S[key][head] for all 128 keys: 8 m16 blocks, two blocks per chain
+    float acc[8][4];
+#pragma unroll
+    for (int mb = 0; mb < 8; ++mb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mb][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+      for (int mb = 0; mb < 8; ++mb) {
+        const int r = mb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int c = ks * 16 + (lane >> 4) * 8;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(tile + sw128_chunk_off(r, c, T), a0, a1, a2, a3);
+        mma16816(acc[mb], a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&empty[s]));  // scores are in registers
     float mx0 = kNegInf, mx1 = kNegInf;
 #pragma unroll
-    for (int mb = 0; mb < 2; ++mb)
+    for (int mb = 0; mb < 8; ++mb)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int key = t * T + warp * 32 + mb * 16 + (lane >> 2) + (e >> 1) * 8;
+        const int key = t * T + mb * 16 + (lane >> 2) + (e >> 1) * 8;
         const float v = key < p.Lc ? acc[mb][e] * p.scale_log2 : kNegInf;
         acc[mb][e] = v;
         if (e & 1) mx1 = fmaxf(mx1, v); else mx0 = fmaxf(mx0, v);
@@ -170,20 +202,12 @@ __global__ void __launch_bounds__(NT) stats_kernel(const __grid_constant__ CUten
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
-    if (lane < 4) {
-      red[warp * 8 + n0] = mx0;
-      red[warp * 8 + n0 + 1] = mx1;
-    }
-    __syncthreads();
-    const float mt0 = fmaxf(fmaxf(red[n0], red[8 + n0]), fmaxf(red[16 + n0], red[24 + n0]));
-    const float mt1 =
-        fmaxf(fmaxf(red[n0 + 1], red[9 + n0]), fmaxf(red[17 + n0], red[25 + n0]));
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int mb = 0; mb < 2; ++mb)
+    for (int mb = 0; mb < 8; ++mb)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        if (e & 1) s1 += exp2f(acc[mb][e] - mt1); else s0 += exp2f(acc[mb][e] - mt0);
+        if (e & 1) s1 += exp2f(acc[mb][e] - mx1); else s0 += exp2f(acc[mb][e] - mx0);
       }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
@@ -191,17 +215,9 @@ __global__ void __launch_bounds__(NT) stats_kernel(const __grid_constant__ CUten
       s1 += __shfl_xor_sync(0xffffffffu, s1, o);
     }
     if (lane < 4) {
-      red[32 + warp * 8 + n0] = s0;
-      red[32 + warp * 8 + n0 + 1] = s1;
+      if (n0 < p.G) p.stats[((size_t)grp * p.G + n0) * p.nt + t] = make_float2(mx0, s0);
+      if (n0 + 1 < p.G) p.stats[((size_t)grp * p.G + n0 + 1) * p.nt + t] = make_float2(mx1, s1);
     }
-    __syncthreads();
-    if (tid < p.G) {
-      const float mt = fmaxf(fmaxf(red[tid], red[8 + tid]), fmaxf(red[16 + tid], red[24 + tid]));
-      const float l = red[32 + tid] + red[40 + tid] + red[48 + tid] + red[56 + tid];
-      p.stats[((size_t)grp * p.G + tid) * p.nt + t] = make_float2(mt, l);
-    }
-    __syncthreads();  // stage s and `red` free again
-    if (tid == 0 && k + NST < count) issue(k + NST);
   }
 }
 
