@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(NT, 1)
         for (int X = 0; X < 2; ++X) {
           if (!MALA_PART(X, t)) continue;
           if (t > 0 && MALA_PART(X, t - 1)) {  // S_X of the previous tile consumed
-            mbar_wait(smem_u32(&bars.s_free[X]), free_ph[X], abort, 0x214);
+            mbar_wait_spin(smem_u32(&bars.s_free[X]), free_ph[X], abort, 0x214);
             free_ph[X] ^= 1;
             tc_fence_after();
           }

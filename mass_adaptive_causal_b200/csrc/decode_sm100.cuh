@@ -102,15 +102,17 @@ struct StatsParams {
   float scale_log2;
 };
 
-constexpr int STATS_CONSUMERS = 8;                    // warps, one whole tile each
-constexpr int STATS_NT = 32 * (STATS_CONSUMERS + 1);  // + one TMA producer warp
+// One consumer warp per ring stage: warp w reads stage w only (tiles w,
+// w + 6, ...), so it never waits on a stage more than one phase ahead.
 constexpr int STATS_NST = 6;                          // TMA ring depth
+constexpr int STATS_CONSUMERS = STATS_NST;            // warps, one whole tile each
+constexpr int STATS_NT = 32 * (STATS_CONSUMERS + 1);  // + one TMA producer warp
 constexpr uint32_t STATS_RING_SMEM = STATS_NST * TILE_BYTES + 1024 + 256;
 
-// Phase A: one CTA per SM streams a contiguous run of tiles. Warp 8 keeps a
-// 6-stage TMA ring full; consumer warp w handles tiles w, w+8, ... of the run
-// entirely by itself (8 m16 blocks x 8 k-steps of mma.sync against the
-// group's query heads), so no CTA-wide barrier sits on the stream.
+// Phase A: one CTA per SM streams a contiguous run of tiles. The last warp
+// keeps a 6-stage TMA ring full; consumer warp w handles tiles w, w+6, ... of
+// the run entirely by itself (8 m16 blocks x 8 k-steps of mma.sync against
+// the group's query heads), so no CTA-wide barrier sits on the stream.
 __global__ void __launch_bounds__(STATS_NT) stats_kernel(const __grid_constant__ CUtensorMap tmK,
                                                          const StatsParams p) {
   extern __shared__ unsigned char smem_raw[];

@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
         for (int X = 0; X < 2; ++X) {
           if (MALA_PART(X, t)) {
-            mbar_wait(smem_u32(&bars.decision[X]), dec_ph[X], abort, 0x114);
+            mbar_wait_spin(smem_u32(&bars.decision[X]), dec_ph[X], abort, 0x114);
             dec_ph[X] ^= 1;
             if (*reinterpret_cast<volatile int*>(&bars.keepflag[X])) {
               mbar_wait(smem_u32(&bars.v_full[X]), v_ph[X], abort, 0x115);
@@ -261,6 +261,9 @@ __global__ void __launch_bounds__(NT, 1)
       const uint32_t t_o = tmem + lane_base + 256 + X * 128;
       const uint32_t vdst = sbase + OFF_V + X * TILE_BYTES;
       float m_ref = kNegInf, l = 0.f;
+      // keep iff mraw * scale_log2 - m_ref - log2 l >= thr; cached as a raw
+      // score bound, refreshed whenever (m_ref, l) change
+      float bound_raw = kNegInf;
       int n_kept = 0;
       uint32_t s_ph = 0;
       const int nw = (p.nb + 31) >> 5;
@@ -280,7 +283,7 @@ __global__ void __launch_bounds__(NT, 1)
         const float mraw = tmem_rowmax128(t_s, diag, r);
         const float mt = mraw * p.scale_log2;
         int want = diag || p.never_skip;
-        if (!want && row_valid) want = (mt - m_ref - __log2f(l)) >= thr;
+        if (!want && row_valid) want = mraw >= bound_raw;
         tc_fence_before();
         const int keep = wg_vote_or(want, bar_id);
         kb.set(j, keep != 0);
@@ -345,6 +348,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
         l += lsum;
         ++n_kept;
+        bound_raw = (thr + m_ref + __log2f(l)) / p.scale_log2;
         tc_fence_before();
         wg_sync(bar_id);
         if (r == 0) {

@@ -28,27 +28,28 @@ def rel_l2(got, ref):
     return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))
 
 
-def compare_fwd_keep(gpu_keep, ref_keep, ref_margin, forced_diag=True):
-    """Forward keep sets, one slice: (nb, nb) arrays. Returns (n_mismatch,
-    n_near, bad_blocks) where bad_blocks are query blocks with an allowed
-    flip. Raises AssertionError on a disallowed mismatch."""
-    nb = ref_keep.shape[0]
+def compare_fwd_keep(gpu_keep, ref_keep, ref_margin, row_offset=0):
+    """Forward keep sets of one slice: rows are query blocks row_offset,
+    row_offset + 1, ...; columns are key blocks. Returns (n_near, bad_rows)
+    where bad_rows are local row indices with an allowed flip. Raises
+    AssertionError on a disallowed mismatch."""
     n_near = 0
     bad_blocks = []
-    for i in range(nb):
+    for li in range(ref_keep.shape[0]):
+        i = li + row_offset
         flipped = False
         for j in range(i, -1, -1):
-            g, r = int(gpu_keep[i, j]), int(ref_keep[i, j])
+            g, r = int(gpu_keep[li, j]), int(ref_keep[li, j])
             if g == r:
                 continue
             if flipped:
                 continue  # downstream of an allowed flip in this block
-            mu = ref_margin[i, j]
+            mu = ref_margin[li, j]
             assert abs(mu) <= NEAR, f"keep mismatch at ({i},{j}) margin {mu}"
             n_near += 1
             flipped = True
         if flipped:
-            bad_blocks.append(i)
+            bad_blocks.append(li)
     return n_near, bad_blocks
 
 

@@ -44,7 +44,7 @@ def check_fwd_slice(Qd, Kd, Vd, O_gpu, LSE_gpu, bits_gpu, tile, tau, tol, qblock
     ref = oracle.fwd(Qd, Kd, Vd, tile=tile, tau=tau, want_margin=True, qblocks=qblocks)
     lo, hi = (0, nb) if qblocks is None else qblocks
     gk = mala.unpack_bits(bits_gpu, nb)
-    n_near, bad = compare_fwd_keep(gk[lo:hi], ref["keep"][lo:hi], ref["margin"][lo:hi])
+    n_near, bad = compare_fwd_keep(gk[lo:hi], ref["keep"][lo:hi], ref["margin"][lo:hi], lo)
     bad = [b + lo for b in bad]
     rows = row_mask(L, tile, bad)
     sel = np.zeros(L, bool)
@@ -226,6 +226,20 @@ def check_decode(q, Kc, Vc, o, kept, bits, tau, groups):
             assert kept[b, g].item() == int(ref["keep"][g].sum())
             sl = slice(g * G, (g + 1) * G)
             assert rel_l2(as_f64(o[b, sl]), ref["o"][sl]) <= TOL["bf16"]["decode"]
+
+
+def test_decode_long_cache_wraps_the_ring():
+    """4 groups x 1024 tiles: every CTA of the streaming pass cycles its TMA
+    ring several times."""
+    cfg = synth.DecodeConfig("wrap", 4, 2, 8, 2, 131072, 128, 128, 0.98, 1024, 4)
+    x = synth.decode_inputs(cfg)
+    q = dev_tensor(x["q"], torch.bfloat16)
+    Kc = dev_tensor(x["K"], torch.bfloat16)
+    Vc = dev_tensor(x["V"], torch.bfloat16)
+    for _ in range(2):
+        o, kept, bits = mala.mala_decode(q, Kc, Vc, tau=1.0, trace=True)
+    mala.mala_check()
+    check_decode(q, Kc, Vc, o, kept, bits, 1.0, set(range(cfg.B * cfg.Hkv)))
 
 
 @pytest.mark.parametrize("Lc", [1, 127, 128, 1000, 5000])
