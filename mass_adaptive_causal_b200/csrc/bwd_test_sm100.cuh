@@ -135,6 +135,11 @@ __global__ void __launch_bounds__(NT, 1)
     if (lane == 0) {
       mbar_wait(smem_u32(&bars.q_full), 0, abort, 0x212);
       uint32_t free_ph[2] = {0, 0};
+      const uint64_t dq0 = sdesc_sw128(sbase + OFF_Q, 16, 1024);
+      const uint64_t dq1 = sdesc_sw128(sbase + OFF_Q + TILE_BYTES, 16, 1024);
+      uint64_t dks[NSTAGE];
+#pragma unroll
+      for (int st = 0; st < NSTAGE; ++st) dks[st] = sdesc_sw128(sbase + OFF_K + st * TILE_BYTES, 16, 1024);
       for (int t = 0; t < ntiles; ++t) {
         const int s = t % NSTAGE;
         mbar_wait(smem_u32(&bars.k_full[s]), (t / NSTAGE) & 1, abort, 0x213);
@@ -147,14 +152,12 @@ __global__ void __launch_bounds__(NT, 1)
             free_ph[X] ^= 1;
             tc_fence_after();
           }
-          const uint32_t qa = sbase + OFF_Q + X * TILE_BYTES;
-          const uint32_t ka = sbase + OFF_K + s * TILE_BYTES;
+          const uint64_t dq = X ? dq1 : dq0;
+          const uint64_t dk = s == 0 ? dks[0] : (s == 1 ? dks[1] : dks[2]);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            mma_bf16(tmem + X * 128, sdesc_sw128(qa + off, 16, 1024),
-                     sdesc_sw128(ka + off, 16, 1024), IDESC_QK, kk > 0);
-          }
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16(tmem + X * 128, sdesc_kstep(dq, kk, HALF_BYTES), sdesc_kstep(dk, kk, HALF_BYTES),
+                     IDESC_QK, kk > 0);
           mma_commit(smem_u32(&bars.s_full[X]));
         }
         mma_commit(smem_u32(&bars.k_empty[s]));

@@ -88,6 +88,7 @@ struct Bars {
   int abort;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
+static_assert(NSTAGE == 3, "descriptor selection below assumes three K stages");
 
 // OR-vote over one 128-thread warpgroup on named barrier `id`.
 __device__ __forceinline__ int wg_vote_or(int pred, int id) {
@@ -107,15 +108,13 @@ __device__ __forceinline__ void wg_sync(int id) {
 }
 
 // S_X = Q_X K_t^T (8 MMAs of K = 16), completion signalled on s_full[X].
-__device__ __forceinline__ void issue_qk(Bars& bars, uint32_t sbase, uint32_t tmem, int X, int t) {
-  const uint32_t qa = sbase + OFF_Q + X * TILE_BYTES;
-  const uint32_t ka = sbase + OFF_K + (t % NSTAGE) * TILE_BYTES;
+// dq / dk: base descriptors of Q_X and of the K stage holding tile t.
+__device__ __forceinline__ void issue_qk(Bars& bars, uint32_t tmem, int X, uint64_t dq,
+                                         uint64_t dk) {
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-    mma_bf16(tmem + X * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
+  for (int kk = 0; kk < D / 16; ++kk)
+    mma_bf16(tmem + X * 128, sdesc_kstep(dq, kk, HALF_BYTES), sdesc_kstep(dk, kk, HALF_BYTES),
              IDESC_QK, kk > 0);
-  }
   mma_commit(smem_u32(&bars.s_full[X]));
 }
 
@@ -203,10 +202,22 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_wait(smem_u32(&bars.q_full), 0, abort, 0x112);
       uint32_t dec_ph[2] = {0, 0}, v_ph[2] = {0, 0};
       int pv_count[2] = {0, 0};
+      // base descriptors, computed once
+      const uint64_t dq0 = sdesc_sw128(sbase + OFF_Q, 16, 1024);
+      const uint64_t dq1 = sdesc_sw128(sbase + OFF_Q + TILE_BYTES, 16, 1024);
+      uint64_t dks[NSTAGE];
+#pragma unroll
+      for (int st = 0; st < NSTAGE; ++st) dks[st] = sdesc_sw128(sbase + OFF_K + st * TILE_BYTES, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sbase + OFF_V, HALF_BYTES, 1024);
+      const uint64_t dv1 = sdesc_sw128(sbase + OFF_V + TILE_BYTES, HALF_BYTES, 1024);
+      auto kdesc = [&](int t) -> uint64_t {
+        const int st = t % NSTAGE;
+        return st == 0 ? dks[0] : (st == 1 ? dks[1] : dks[2]);
+      };
       wait_k_full(bars, 0, abort);
 #pragma unroll
       for (int X = 0; X < 2; ++X)
-        if (MALA_PART(X, 0)) issue_qk(bars, sbase, tmem, X, 0);
+        if (MALA_PART(X, 0)) issue_qk(bars, tmem, X, X ? dq1 : dq0, kdesc(0));
       mma_commit(smem_u32(&bars.k_empty[0]));
       for (int t = 0; t < ntiles; ++t) {
         bool k_next_ready = false;
@@ -219,15 +230,14 @@ __global__ void __launch_bounds__(NT, 1)
               mbar_wait(smem_u32(&bars.v_full[X]), v_ph[X], abort, 0x115);
               v_ph[X] ^= 1;
               tc_fence_after();
-              const uint32_t va = sbase + OFF_V + X * TILE_BYTES;
+              const uint64_t dv = X ? dv1 : dv0;
 #pragma unroll
               for (int half = 0; half < 2; ++half) {
 #pragma unroll
                 for (int kk = 0; kk < T / 16; ++kk) {
                   const uint32_t a_t = tmem + X * 128 + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half;
-                  mma_bf16_ts(tmem + 256 + X * 128, a_t,
-                              sdesc_sw128(va + kk * 2048, HALF_BYTES, 1024), IDESC_PV,
-                              (pv_count[X] > 0 || half > 0 || kk > 0) ? 1u : 0u);
+                  mma_bf16_ts(tmem + 256 + X * 128, a_t, dv + (uint64_t)((kk * 2048) >> 4),
+                              IDESC_PV, (pv_count[X] > 0 || half > 0 || kk > 0) ? 1u : 0u);
                 }
               }
               mma_commit(smem_u32(&bars.pv_done[X]));
@@ -239,7 +249,7 @@ __global__ void __launch_bounds__(NT, 1)
               wait_k_full(bars, t + 1, abort);
               k_next_ready = true;
             }
-            issue_qk(bars, sbase, tmem, X, t + 1);
+            issue_qk(bars, tmem, X, X ? dq1 : dq0, kdesc(t + 1));
           }
         }
         if (t + 1 < ntiles) mma_commit(smem_u32(&bars.k_empty[(t + 1) % NSTAGE]));

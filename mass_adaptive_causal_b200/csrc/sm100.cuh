@@ -143,6 +143,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// Descriptor for the k-step `kk` (16 elements) of a K-major 128-byte-swizzled
+// operand whose base descriptor is `d0`: the start address advances 32 bytes
+// inside a 64-column block and 16 KB (`blk_bytes`) between blocks. All
+// offsets are compile-time after unrolling, so an MMA issue costs one add.
+__device__ __forceinline__ uint64_t sdesc_kstep(uint64_t d0, int kk, uint32_t blk_bytes) {
+  return d0 + (uint64_t)((((kk >> 2) * blk_bytes) + (kk & 3) * 32) >> 4);
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B and an
 // f32 accumulator. a_mn / b_mn select MN-major operands.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
