@@ -267,6 +267,39 @@ __device__ __forceinline__ float tmem_rowmax128(uint32_t taddr, bool diag, int r
   return m;
 }
 
+// Row max over 64 TMEM columns of this thread's lane (columns col0 .. col0+63
+// of the tile). With `diag`, tile columns c > r are excluded.
+__device__ __forceinline__ float tmem_rowmax64(uint32_t taddr, bool diag, int r, int col0) {
+  float s[64];
+  tmem_ld64(taddr, s);
+  float m = -__builtin_huge_valf();
+  if (!diag) {
+#pragma unroll
+    for (int e = 0; e < 63; e += 2) m = fmax3f(m, s[e], s[e + 1]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 64; ++e) m = fmaxf(m, (col0 + e > r) ? -__builtin_huge_valf() : s[e]);
+  }
+  return m;
+}
+
+// OR-vote / barrier over `count` threads on named barrier `id` (1..15).
+__device__ __forceinline__ int bar_vote_or(int pred, int id, int count) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "barrier.cta.red.or.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(out)
+      : "r"(pred), "r"(id), "r"(count)
+      : "memory");
+  return (int)out;
+}
+__device__ __forceinline__ void bar_sync_n(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Byte offset of the 16-byte chunk holding element (row, col) of a bf16
 // operand tile stored in 64-column swizzled blocks of `rows` rows.
 __device__ __forceinline__ uint32_t sw128_chunk_off(int row, int col, int rows) {
