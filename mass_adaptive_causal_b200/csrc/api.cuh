@@ -113,6 +113,7 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
   p.LSE = LSE;
   p.L = L;
   p.nb = (L + fwd100::T - 1) / fwd100::T;
+  p.npairs = (p.nb + 1) / 2;
   p.scale_log2 = scale * kLog2e;
   p.never_skip = tau == 0.f;
   p.log2_tau = tau > 0.f ? log2f(tau) : 0.f;
@@ -121,7 +122,7 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
   MALA_CUDA_TRY(cudaFuncSetAttribute(fwd100::fwd_bf16_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)fwd100::SMEM_BYTES));
-  fwd100::fwd_bf16_kernel<<<dim3(p.nb, Z), fwd100::NT, fwd100::SMEM_BYTES, s>>>(mq, mk, mv, p);
+  fwd100::fwd_bf16_kernel<<<dim3(p.npairs, Z), fwd100::NT, fwd100::SMEM_BYTES, s>>>(mq, mk, mv, p);
   return launch_status();
 }
 
@@ -227,13 +228,14 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
     tp.LSE = LSE;
     tp.L = L;
     tp.nb = nb;
+    tp.npairs = (nb + 1) / 2;
     tp.scale_log2 = scale * kLog2e;
     tp.log2_tau = log2f(tau);
     tp.bits = tile_bits;
     MALA_CUDA_TRY(cudaFuncSetAttribute(bwdtest::test_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bwdtest::SMEM_BYTES));
-    bwdtest::test_kernel<<<dim3(nb, Z), bwdtest::NT, bwdtest::SMEM_BYTES, s>>>(mq, mk, tp);
+    bwdtest::test_kernel<<<dim3(tp.npairs, Z), bwdtest::NT, bwdtest::SMEM_BYTES, s>>>(mq, mk, tp);
   } else if (bits) {
     const size_t nwords = (size_t)Z * nb * ((nb + 31) / 32);
     aux::lower_bits_kernel<<<blocks_for(nwords, 256, 4 * sm_count()), 256, 0, s>>>(bits, nb,
