@@ -50,7 +50,8 @@ typedef enum {
   MALA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned, tau < 0 */
   MALA_ERR_UNSUPPORTED = 2, /* (dtype, d, tile) combination not built */
   MALA_ERR_CUDA = 3,        /* CUDA runtime error at launch or check */
-  MALA_ERR_TIMEOUT = 4      /* a device-side wait ran out (see mala_check) */
+  MALA_ERR_TIMEOUT = 4,     /* a device-side wait ran out (see mala_check) */
+  MALA_ERR_TOO_LARGE = 5    /* shape needs more than the built-in scratch */
 } mala_status;
 
 typedef enum { MALA_F32 = 0, MALA_BF16 = 1 } mala_dtype;
@@ -158,6 +159,47 @@ mala_status mala_decode(const void* q, const void* Kcache, const void* Vcache,
                         float tau, float scale, void* workspace,
                         size_t workspace_bytes, int32_t* kept_tiles,
                         uint32_t* keep_bits, void* stream);
+
+/* Size of the device scratch array that mala_decode_noalloc uses in place
+ * of a caller's workspace (8 MiB; B = 16, Hq = 32, Hkv = 8, Lc = 131072 needs
+ * about 4.8 MiB). */
+#define MALA_DECODE_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * mala_decode without a workspace argument, for callers that cannot allocate
+ * device memory. The paper has no counterpart: this is an interface choice.
+ *
+ * Who needs it: code whose host program hands it only the buffers it reads
+ * and writes and keeps every other byte of device memory for itself (a plugin
+ * or custom operator inside an inference server with its own memory pool, a
+ * runtime that reserves the GPU's memory at start-up). There a cudaMalloc
+ * either fails or forces the pool to give memory back, and a serving loop
+ * cannot afford that in the middle of a step.
+ *
+ * Scratch: a file-scope __device__ array of MALA_DECODE_NOALLOC_SCRATCH_BYTES
+ * bytes inside this library. Every GPU that loads the library holds it until
+ * the process exits. The first call on a device, with that device current,
+ * looks up the array's device address (cudaGetSymbolAddress) and caches it;
+ * make that first call before any stream capture begins. The call itself
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ * routine.
+ *
+ * All calls on a device share the one array and it keeps the last call's
+ * contents; the kernels clear the part that must start at zero (the float32
+ * output accumulator) in every call. Calls that overlap on the GPU (two
+ * streams, or two host threads, at once) race on the array: serialise them.
+ *
+ * Arguments, layouts, outputs and the rule are those of mala_decode.
+ * Errors: as mala_decode, and MALA_ERR_TOO_LARGE, before any launch, when
+ * mala_decode_workspace_bytes(B, Hq, Hkv, Lc, d) exceeds
+ * MALA_DECODE_NOALLOC_SCRATCH_BYTES. MALA_ERR_CUDA if the array's address
+ * cannot be found on the current device.
+ */
+mala_status mala_decode_noalloc(const void* q, const void* Kcache,
+                                const void* Vcache, void* o, int B, int Hq,
+                                int Hkv, int Lc, int d, float tau, float scale,
+                                int32_t* kept_tiles, uint32_t* keep_bits,
+                                void* stream);
 
 /*
  * Synchronizes `stream`, then reads and clears this GPU's device status word.

@@ -18,7 +18,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["mala_fwd", "mala_bwd", "mala_decode", "mala_check", "MalaError", "lib",
+__all__ = ["mala_fwd", "mala_bwd", "mala_decode", "mala_decode_noalloc", "mala_check", "MalaError", "lib",
            "LIB_PATH", "MALA_F32", "MALA_BF16", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(_HERE, "libmala.so")
 
 MALA_F32, MALA_BF16 = 0, 1
 STATUS = {0: "MALA_OK", 1: "MALA_ERR_INVALID_ARG", 2: "MALA_ERR_UNSUPPORTED",
-          3: "MALA_ERR_CUDA", 4: "MALA_ERR_TIMEOUT"}
+          3: "MALA_ERR_CUDA", 4: "MALA_ERR_TIMEOUT", 5: "MALA_ERR_TOO_LARGE"}
 
 
 class MalaError(RuntimeError):
@@ -62,6 +62,9 @@ def lib() -> ctypes.CDLL:
         L.mala_decode.argtypes = [_vp, _vp, _vp, _vp, ci, ci, ci, ci, ci, cf, cf, _vp, cs, _i32p,
                                   _u32p, _vp]
         L.mala_decode.restype = ci
+        L.mala_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, ci, ci, ci, ci, ci, cf, cf, _i32p,
+                                          _u32p, _vp]
+        L.mala_decode_noalloc.restype = ci
         L.mala_check.argtypes = [_vp]
         L.mala_check.restype = ci
         L.mala_status_string.argtypes = [ci]
@@ -216,6 +219,37 @@ def mala_decode(q, k_cache, v_cache, tau: float = 1.0, scale: float = 0.0, trace
                              float(tau), float(scale), _ptr(ws), ws.numel(), _ptr(kept),
                              _ptr(bits), _stream(stream))
     _raise(code, "mala_decode")
+    return (o, kept, bits) if trace else o
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20  # MALA_DECODE_NOALLOC_SCRATCH_BYTES in include/mala.h
+
+
+def mala_decode_noalloc(q, k_cache, v_cache, tau: float = 1.0, scale: float = 0.0,
+                        trace: bool = False, out=None, stream=None):
+    """mala_decode without a workspace: the library's own static device array
+    (NOALLOC_SCRATCH_BYTES, shared by every call on the device) serves as
+    scratch, for callers that cannot allocate device memory. Calls that
+    overlap on the GPU race on that array. Raises MalaError
+    (MALA_ERR_TOO_LARGE) when the shape needs more scratch than the array
+    holds. The output (and trace) tensors are the caller's: pass ``out`` to
+    avoid allocating here too."""
+    torch = _torch()
+    for t in (q, k_cache, v_cache):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("decode tensors must be contiguous bf16 CUDA tensors")
+    B, Hq, d = q.shape
+    _, Hkv, Lc, _ = k_cache.shape
+    o = torch.empty_like(q) if out is None else out
+    kept = bits = None
+    if trace:
+        nt = n_blocks(Lc, 128)
+        kept = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+        bits = torch.empty((B, Hkv, (nt + 31) // 32), dtype=torch.int32, device=q.device)
+    code = lib().mala_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), B, Hq, Hkv,
+                                     Lc, d, float(tau), float(scale), _ptr(kept), _ptr(bits),
+                                     _stream(stream))
+    _raise(code, "mala_decode_noalloc")
     return (o, kept, bits) if trace else o
 
 

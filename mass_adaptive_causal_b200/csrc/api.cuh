@@ -386,6 +386,7 @@ const char* mala_status_string(mala_status s) {
     case MALA_ERR_UNSUPPORTED: return "MALA_ERR_UNSUPPORTED";
     case MALA_ERR_CUDA: return "MALA_ERR_CUDA";
     case MALA_ERR_TIMEOUT: return "MALA_ERR_TIMEOUT";
+    case MALA_ERR_TOO_LARGE: return "MALA_ERR_TOO_LARGE";
   }
   return "MALA_ERR_UNKNOWN";
 }

@@ -2,3 +2,63 @@
 // device status word (common.cuh) exists once per GPU and every kernel can
 // set it without relocatable device code.
 #include "api.cuh"
+
+// -------------------------------------------------------------------------
+// mala_decode_noalloc: the decode step with its workspace in a static device
+// array, for callers that cannot allocate device memory (their host program
+// owns all of it). The array is part of this library's module, so every GPU
+// that loads the library holds MALA_DECODE_NOALLOC_SCRATCH_BYTES until exit.
+// -------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_decode_scratch[MALA_DECODE_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+unsigned char* g_scratch_ptr[kMaxDevices];  // device address per device, once found
+
+// In host code `g_decode_scratch` only names the array; its address on the
+// current device comes from the runtime, once per device, and is cached.
+mala_status scratch_on_current_device(unsigned char** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MALA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    unsigned char* ptr = nullptr;
+    if (cudaGetSymbolAddress((void**)&ptr, g_decode_scratch) != cudaSuccess || !ptr)
+      return MALA_ERR_CUDA;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return MALA_OK;
+}
+
+}  // namespace
+
+extern "C" mala_status mala_decode_noalloc(const void* q, const void* Kcache, const void* Vcache,
+                                           void* o, int B, int Hq, int Hkv, int Lc, int d,
+                                           float tau, float scale, int32_t* kept_tiles,
+                                           uint32_t* keep_bits, void* stream) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lc < 1 || d < 1) return MALA_ERR_INVALID_ARG;
+  if (!tau_ok(tau)) return MALA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return MALA_ERR_INVALID_ARG;
+  if (d != 128 || Hq / Hkv > mala::dec::GMAX) return MALA_ERR_UNSUPPORTED;
+  if ((long long)B * Hkv > 4095) return MALA_ERR_UNSUPPORTED;
+  if (!q || !Kcache || !Vcache || !o) return MALA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, Kcache, Vcache, o};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MALA_ERR_INVALID_ARG;
+  if (mala_decode_workspace_bytes(B, Hq, Hkv, Lc, d) > MALA_DECODE_NOALLOC_SCRATCH_BYTES)
+    return MALA_ERR_TOO_LARGE;
+  unsigned char* scratch = nullptr;
+  const mala_status st = scratch_on_current_device(&scratch);
+  if (st != MALA_OK) return st;
+  // Every region is written before it is read within the call; the scan
+  // kernel zeroes the float32 output accumulator, the one region that must
+  // start at zero.
+  DecWorkspace w = dec_ws_carve(scratch, B, Hq, Hkv, Lc, d);
+  return decode_bf16(q, Kcache, Vcache, o, B, Hq, Hkv, Lc, resolve_scale(scale, d), tau, w,
+                     kept_tiles, keep_bits, as_stream(stream));
+}

@@ -90,3 +90,18 @@ def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(mala, "_lib", None)
     with pytest.raises(RuntimeError):
         mala.lib()
+
+
+def test_decode_noalloc_argument_checks(lib):
+    """Shape checks, including the scratch limit, come before any CUDA call."""
+    p = [ctypes.c_void_p(16)] * 4
+    f = lib.mala_decode_noalloc
+    assert f(*p, 1, 8, 2, 1000, 128, -1.0, 0.0, None, None, None) == 1
+    assert f(*p, 1, 8, 3, 1000, 128, 1.0, 0.0, None, None, None) == 1
+    assert f(*p, 1, 8, 2, 1000, 64, 1.0, 0.0, None, None, None) == 2
+    assert f(*p, 1, 32, 2, 1000, 128, 1.0, 0.0, None, None, None) == 2
+    assert f(None, *p[1:], 1, 8, 2, 1000, 128, 1.0, 0.0, None, None, None) == 1
+    B, Hq, Hkv, Lc, d = 64, 64, 8, 32768, 128
+    assert mala.decode_workspace_bytes(B, Hq, Hkv, Lc, d) > mala.NOALLOC_SCRATCH_BYTES
+    assert f(*p, B, Hq, Hkv, Lc, d, 1.0, 0.0, None, None, None) == 5
+    assert lib.mala_status_string(5).decode() == "MALA_ERR_TOO_LARGE"
