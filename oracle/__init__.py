@@ -185,6 +185,35 @@ def omitted_mass(Q, K, keep, LSE_dense, tile, scale=None):
     return mass
 
 
+def tile_row_max(Q, K, tile, qblocks=None):
+    """Raw (unscaled) score maximum of every query row over every legal key
+    tile: for query block i, key block j <= i and row r of block i,
+        out[i][j, r] = max over key c of block j with c <= i*tile + r of Q[i*tile + r] . K[c].
+    This is the quantity the backward's offline test compares with the final
+    log-normalizer (MassAlloc Attention; jaehun.me review, "Backward: offline
+    sparse probabilities": a tile stays iff some row's largest score clears
+    LSE + ln tau - ln(position)). Rows past L are -inf.
+
+    Returns {i: array (i + 1, tile)} for the query blocks in ``qblocks``
+    (a (lo, hi) range; default all)."""
+    Q, K = _f64(Q), _f64(K)
+    L, d = Q.shape
+    nb = n_blocks(L, tile)
+    lo, hi = (0, nb) if qblocks is None else qblocks
+    out = {}
+    for i in range(lo, hi):
+        r0, r1 = i * tile, min(L, (i + 1) * tile)
+        S = Q[r0:r1] @ K[:r1].T                       # (rows, keys <= last row)
+        rows = np.arange(r0, r1)[:, None]
+        S[np.arange(r1)[None, :] > rows] = -np.inf    # causal mask
+        m = np.full((i + 1, tile), -np.inf)
+        for j in range(i + 1):
+            c0, c1 = j * tile, min(r1, (j + 1) * tile)
+            m[j, :r1 - r0] = S[:, c0:c1].max(axis=1)
+        out[i] = m
+    return out
+
+
 def retained_slots(keep, L, tile):
     """Mean over query rows of the number of legal keys inside kept tiles
     (the pages' "post-score key slots per query")."""

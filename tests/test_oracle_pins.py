@@ -360,3 +360,48 @@ def test_decode_group_rows():
         assert omitted <= 0.5 + 1e-12
         w = np.exp(s[kept_cols] - s[kept_cols].max())
         assert np.allclose(grp["o"][h], (w / w.sum()) @ Vc[g][kept_cols], rtol=0, atol=1e-12)
+
+
+def test_tile_row_max_bruteforce():
+    """Pure-Python enumeration of every (row, legal key) score on a tiny
+    ragged case (L = 7, tile 3: blocks of 3, 3, 1 rows)."""
+    rng = np.random.default_rng(41)
+    L, d, T = 7, 2, 3
+    Q, K = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    got = oracle.tile_row_max(Q, K, T)
+    assert sorted(got) == [0, 1, 2]
+    for i in range(3):
+        for j in range(i + 1):
+            for r in range(T):
+                row = i * T + r
+                if row >= L:
+                    assert got[i][j, r] == -np.inf
+                    continue
+                best = -math.inf
+                for c in range(j * T, min(L, (j + 1) * T)):
+                    if c <= row:
+                        best = max(best, sum(Q[row, e] * K[c, e] for e in range(d)))
+                assert got[i][j, r] == pytest.approx(best, abs=1e-12)
+
+
+@pytest.mark.parametrize("tau", [1.0, 0.25])
+def test_tile_row_max_decides_the_backward_keep_set(tau):
+    """The backward's keep set follows from the tile row maxima and the final
+    LSE alone: tile (i, j) stays iff some valid row has
+    scale * max >= LSE + ln tau - ln(row + 1)."""
+    L, d, T = 300, 8, 8
+    Q, K, V, dO = rand_inputs(L, d, 43, scale_qk=3.0)
+    scale = 1.0 / math.sqrt(d)
+    f = oracle.fwd(Q, K, V, tile=T, tau=tau)
+    g = oracle.bwd(Q, K, V, f["O"], dO, f["LSE"], tile=T, tau=tau, want_margin=True)
+    rm = oracle.tile_row_max(Q, K, T)
+    nb = oracle.n_blocks(L, T)
+    skipped = 0
+    for i in range(nb):
+        for j in range(i + 1):
+            rows = np.arange(i * T, min(L, (i + 1) * T))
+            margin = scale * rm[i][j, :len(rows)] - (f["LSE"][rows] + math.log(tau) - np.log(rows + 1))
+            assert int(margin.max() >= 0) == g["keep"][i, j], (i, j)
+            assert margin.max() == pytest.approx(g["margin"][i, j], abs=1e-9)
+            skipped += int(g["keep"][i, j] == 0)
+    assert skipped > 0
