@@ -188,6 +188,11 @@ def legal_pairs(L: int) -> int:
     return L * (L + 1) // 2
 
 
+def legal_tiles(L: int, tile: int) -> int:
+    nb = (L + tile - 1) // tile
+    return nb * (nb + 1) // 2
+
+
 def retained_pairs(kept_bits, L: int, tile: int) -> int:
     """Sum over query rows of the legal keys inside kept tiles, from the
     [.., nb, nw] keep bitmask (row = query block, bit = key block)."""
@@ -251,18 +256,22 @@ def run_mala(args, rank, world, local_rank):
     LSE = torch.empty((P.B, P.H, P.L), dtype=torch.float32, device=dev)
     dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
     o = torch.empty_like(q)
+    RM = torch.empty(mala.tile_rowmax_bytes(P.B, P.H, P.L, P.tile) // 4, dtype=torch.float32,
+                     device=dev)
     ws_b = torch.empty(mala.bwd_workspace_bytes(P.B, P.H, P.L, P.d), dtype=torch.uint8, device=dev)
     ws_d = torch.empty(mala.decode_workspace_bytes(Dc.B, Dc.Hq, Dc.Hkv, Dc.Lc, Dc.d),
                        dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(tau, ev=None):
+    def step(tau, ev=None, rowmax=True):
+        rm = RM if rowmax else None
         if ev is not None:
             ev[0].record(stream)
-        mala.mala_fwd(Q, K, V, tau=tau, out=O, lse=LSE, o32=O32)
+        mala.mala_fwd(Q, K, V, tau=tau, out=O, lse=LSE, o32=O32, rowmax=rm)
         if ev is not None:
             ev[1].record(stream)
-        mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, workspace=ws_b, grads=(dQ, dK, dV), o32=O32)
+        mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, workspace=ws_b, grads=(dQ, dK, dV), o32=O32,
+                      rowmax=rm)
         if ev is not None:
             ev[2].record(stream)
         mala.mala_decode(q, Kc, Vc, tau=tau, workspace=ws_d, out=o)
@@ -282,9 +291,9 @@ def run_mala(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    def timed(tau, steps, warmup):
+    def timed(tau, steps, warmup, rowmax=True):
         for _ in range(warmup):
-            step(tau)
+            step(tau, rowmax=rowmax)
         mala.mala_check()
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
         barrier()
@@ -293,7 +302,7 @@ def run_mala(args, rank, world, local_rank):
         end = torch.cuda.Event(enable_timing=True)
         start.record(stream)
         for k in range(steps):
-            step(tau, evs[k])
+            step(tau, evs[k], rowmax=rowmax)
         end.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -309,8 +318,10 @@ def run_mala(args, rank, world, local_rank):
 
     # trace pass (untimed): retained work and kept decode tiles at tau=1 and 0
     def trace(tau):
-        _, _, kept_f, bits_f = mala.mala_fwd(Q, K, V, tau=tau, trace=True, out=O, lse=LSE, o32=O32)[:4]
-        _, _, _, kept_b, bits_b = mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, trace=True, o32=O32)
+        _, _, kept_f, bits_f = mala.mala_fwd(Q, K, V, tau=tau, trace=True, out=O, lse=LSE, o32=O32,
+                                             rowmax=RM)[:4]
+        _, _, _, kept_b, bits_b = mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, trace=True, o32=O32,
+                                                rowmax=RM)
         _, kept_d, _ = mala.mala_decode(q, Kc, Vc, tau=tau, trace=True)
         mala.mala_check()
         nt = (Dc.Lc + 127) // 128
@@ -324,6 +335,10 @@ def run_mala(args, rank, world, local_rank):
     t1 = timed(1.0, args.steps, args.warmup)
     clocks = clock.stop()
     work1 = trace(1.0)
+    # the backward that recomputes every tile's scores for its test (no row maxima)
+    recompute = timed(1.0, max(1, min(args.steps, 3)), 1, rowmax=False)
+    work1["bwd_recompute_ms"] = recompute["bwd_ms"]
+    work1["fwd_no_rowmax_ms"] = recompute["fwd_ms"]
     dense = timed(0.0, max(1, min(args.steps, 3)), 1) if not args.no_dense else None
     e2e = None if args.no_e2e else run_e2e(args, x, dev, world, max_over_ranks)
     return t1, work1, dense, clocks, e2e
@@ -360,8 +375,10 @@ def run_e2e(args, x, dev, world, max_over_ranks):
         q_.copy_(hq, non_blocking=True)
         Kc_.copy_(hKc, non_blocking=True)
         Vc_.copy_(hVc, non_blocking=True)
-        O, LSE, O32 = mala.mala_fwd(dQ_["Q"], dQ_["K"], dQ_["V"], tau=1.0, o32=True)
-        dQ, dK, dV = mala.mala_bwd(dQ_["Q"], dQ_["K"], dQ_["V"], O, dQ_["dO"], LSE, tau=1.0, o32=O32)
+        O, LSE, O32, RM = mala.mala_fwd(dQ_["Q"], dQ_["K"], dQ_["V"], tau=1.0, o32=True,
+                                        rowmax=True)
+        dQ, dK, dV = mala.mala_bwd(dQ_["Q"], dQ_["K"], dQ_["V"], O, dQ_["dO"], LSE, tau=1.0, o32=O32,
+                                   rowmax=RM)
         o = mala.mala_decode(q_, Kc_, Vc_, tau=1.0)
         for n, t in (("O", O), ("dQ", dQ), ("dK", dK), ("dV", dV)):
             outs_h[n].copy_(t, non_blocking=True)
@@ -452,10 +469,12 @@ def profile_case(args):
     if args.profile in ("fwd", "bwd"):
         x = synth.prefill_inputs(PREFILL, L=args.L)
         t = {n: torch.tensor(x[n]).to(torch.bfloat16).cuda() for n in ("Q", "K", "V", "dO")}
-        O, LSE, O32 = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, o32=True)
-        run = (lambda: mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, out=O, lse=LSE, o32=O32)) \
+        O, LSE, O32, RM = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, o32=True, rowmax=True)
+        run = (lambda: mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, out=O, lse=LSE, o32=O32,
+                                     rowmax=RM)) \
             if args.profile == "fwd" else \
-            (lambda: mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=1.0, o32=O32))
+            (lambda: mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=1.0, o32=O32,
+                                   rowmax=RM))
     else:
         cfg = synth.DecodeConfig("profile", 4, 4, DECODE.Hq, DECODE.Hkv, DECODE.Lc, DECODE.d,
                                  128, DECODE.rho, DECODE.n_pairs, DECODE.n_query_targets)
@@ -536,7 +555,10 @@ def main():
     d = P.d
     P_legal = P.B * P.H * legal_pairs(P.L)
     fwd_flop = 2 * d * P_legal + 2 * d * work["fwd_ret"]
-    bwd_flop = 2 * d * P_legal + 8 * d * work["bwd_ret"]
+    # with the forward's tile row maxima the backward's test reads 512 bytes per
+    # legal tile and recomputes no score; kept tiles then cost S, dP, dV, dK, dQ
+    bwd_flop = 10 * d * work["bwd_ret"]
+    rm_bytes = 4 * 128 * P.B * P.H * legal_tiles(P.L, P.tile)
     fwd_tf = fwd_flop / (t1["fwd_ms"] * 1e-3) / 1e12
     bwd_tf = bwd_flop / (t1["bwd_ms"] * 1e-3) / 1e12
     kc_bytes = Dc.B * Dc.Hkv * Dc.Lc * Dc.d * 2
@@ -566,6 +588,10 @@ def main():
         "config": {"workload": WORKLOAD, "tau": 1.0, "l2": "inputs larger than L2 (no flush)",
                    "parallelism": f"replicas x{world} (independent heads/sequences per rank)"},
         "fwd_ms": t1["fwd_ms"], "bwd_ms": t1["bwd_ms"], "decode_us": t1["decode_us"],
+        "bwd_recompute_ms": work["bwd_recompute_ms"], "fwd_no_rowmax_ms": work["fwd_no_rowmax_ms"],
+        "bwd_recompute_tflops_eff": (2 * d * P_legal + 8 * d * work["bwd_ret"]) /
+        (work["bwd_recompute_ms"] * 1e-3) / 1e12,
+        "rowmax_bytes": rm_bytes,
         "fwd_tflops_eff": fwd_tf, "bwd_tflops_eff": bwd_tf,
         "fwd_frac_bf16": fwd_tf / peaks["bf16_tflops"], "bwd_frac_bf16": bwd_tf / peaks["bf16_tflops"],
         "decode_gbs": dec_gbs, "decode_frac_hbm": dec_gbs / peaks["hbm_gbs"],
@@ -575,7 +601,7 @@ def main():
         "decode_kept_tile_frac": work["decode_kept_tiles"] / work["decode_tiles"],
         "roofline": roof,
         "clocks": clocks,
-        "gpu_launches": args.steps * (1 + 4 + 4),
+        "gpu_launches": args.steps * (1 + 5 + 4),  # fwd 1; bwd row-dot, zero, test, work, convert; decode 4
     }
     if dense is not None:
         line["dense_tau0"] = {"fwd_ms": dense["fwd_ms"], "bwd_ms": dense["bwd_ms"],

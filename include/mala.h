@@ -80,16 +80,29 @@ typedef enum { MALA_F32 = 0, MALA_BF16 = 1 } mala_dtype;
  *         D = <dO, O> feed dQ through a sum over keys whose rows cancel, so
  *         D computed from a bf16-rounded O costs dQ percents of accuracy when
  *         keys share a large common component.
+ *         tile_rowmax (may be NULL; MALA_BF16 only): float32, for every
+ *         legal tile (query block i, key block j <= i) and every row r of
+ *         block i, the largest raw score q_r . k_c (unscaled) over the
+ *         tile's keys c <= row; laid out [B][H][i(i+1)/2 + j][tile]
+ *         (mala_tile_rowmax_bytes). Values of rows past L are unspecified.
+ *         Pass it to mala_bwd: the backward's skip test then reads these
+ *         maxima instead of recomputing every tile's scores.
  * Trace   kept_tiles: [B][H][nb] kept key tiles per query block;
  *         keep_bits: [B][H][nb][ceil(nb/32)], row = query block, bit = key
  *         block. nb = ceil(L / tile).
  * Supported: (dt, d, tile) in {(MALA_BF16, 128, 128), (MALA_F32, 32|64|128, 64)};
- *            any L >= 0 (a ragged last block is masked), B, H >= 1.
+ *            any L >= 0 (a ragged last block is masked), B, H >= 1;
+ *            with tile_rowmax, L <= 4194304 (else MALA_ERR_UNSUPPORTED).
  */
 mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O,
-                     float* LSE, float* O_f32, int B, int H, int L, int d, mala_dtype dt,
-                     float tau, int tile, float scale, int32_t* kept_tiles,
-                     uint32_t* keep_bits, void* stream);
+                     float* LSE, float* O_f32, float* tile_rowmax, int B, int H,
+                     int L, int d, mala_dtype dt, float tau, int tile, float scale,
+                     int32_t* kept_tiles, uint32_t* keep_bits, void* stream);
+
+/* Bytes of the forward's optional tile_rowmax output:
+ * B * H * nb(nb+1)/2 * tile * 4 for nb = ceil(L / tile) (2 GiB for B = 1,
+ * H = 8, L = 131072, tile = 128). 0 for invalid sizes. */
+size_t mala_tile_rowmax_bytes(int B, int H, int L, int tile);
 
 /* Bytes of device workspace mala_bwd needs: the row terms D (float32
  * [B][H][L]), the float32 dQ accumulator [B][H][L][d] and the per-tile keep
@@ -101,10 +114,12 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
  * Backward pass.
  *
  * Uses the forward's final LSE instead of replaying its partial normalizers.
- * Every legal tile (i, j) has its scores recomputed; the tile is skipped iff
- * every valid row r satisfies  max_c S_rc - LSE_r  <  ln tau - ln (r + 1).
- * There is no forced keep and no stored mask; in exact arithmetic the kept
- * set is inside the forward's. Kept tiles do the standard work with
+ * Tile (i, j) is skipped iff every valid row r satisfies
+ *     max_c S_rc - LSE_r  <  ln tau - ln (r + 1).
+ * The row maxima come from tile_rowmax when given (the forward recorded them
+ * from the same scores), else every legal tile's scores are recomputed;
+ * both give the same decisions. There is no forced keep and no stored mask;
+ * in exact arithmetic the kept set is inside the forward's. Kept tiles do the standard work with
  * P = exp(S - LSE), D_r = <dO_r, O_r>: dV_j += P^T dO_i, dP = dO_i V_j^T,
  * dS = P o (dP - D), dQ_i += scale dS K_j, dK_j += scale dS^T Q_i.
  * Sources: agihunt.info summary, backward paragraph; jaehun.me review,
@@ -112,7 +127,9 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
  *
  * Inputs  Q, K, V, O, dO: [B][H][L][d] of dtype dt; LSE from mala_fwd;
  *         O_f32 (may be NULL): the float32 output of mala_fwd, used for the
- *         row terms D instead of O when given.
+ *         row terms D instead of O when given;
+ *         tile_rowmax (may be NULL; MALA_BF16 only): the forward's tile row
+ *         maxima for the same Q, K (read only when tau > 0).
  * Outputs dQ, dK, dV: [B][H][L][d] of dtype dt (fully overwritten).
  * workspace: device buffer of at least mala_bwd_workspace_bytes(B,H,L,d)
  *         bytes, 256-byte aligned, contents ignored on entry.
@@ -123,7 +140,7 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
  */
 mala_status mala_bwd(const void* Q, const void* K, const void* V,
                      const void* O, const float* O_f32, const void* dO,
-                     const float* LSE, void* dQ,
+                     const float* LSE, const float* tile_rowmax, void* dQ,
                      void* dK, void* dV, void* workspace,
                      size_t workspace_bytes, int B, int H, int L, int d,
                      mala_dtype dt, float tau, int tile, float scale,

@@ -174,11 +174,8 @@ __global__ void __launch_bounds__(NT, 1)
     if (X == 0 || hasB) {
       const int bar_id = 1 + X;
       const int row = iX * T + r;
-      // threshold in log2 units on the raw score: s * scale_log2 >= c2
-      float c2 = __int_as_float(0x7f800000);  // invalid rows never keep
-      if (row < p.L)
-        c2 = p.LSE[(size_t)z * p.L + row] * kLog2e + p.log2_tau - __log2f((float)(row + 1));
-      const float craw = c2 / p.scale_log2;
+      const float craw =
+          bwd_keep_bound_raw(p.LSE, (size_t)z * p.L, row, p.L, p.log2_tau, p.scale_log2);
       const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16) + X * 256;
       const int nw = (p.nb + 31) >> 5;
       KeepBits kb;
@@ -220,6 +217,51 @@ __global__ void __launch_bounds__(NT, 1)
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+}
+
+// The same test from the tile row maxima the forward recorded
+// (rowmax[z][i(i+1)/2 + j][r], raw scores): no score is recomputed, so the
+// pass only streams 512 bytes per legal tile. CTA = query block i (largest
+// first); each warp takes key blocks j = warp, warp + 8, ...; lane l holds
+// the bounds of rows 4l .. 4l+3 and reads their four maxima as one float4.
+constexpr int RM_NT = 256;
+constexpr int RM_UNROLL = 4;
+
+__global__ void __launch_bounds__(RM_NT)
+    rowmax_test_kernel(const float* __restrict__ rowmax, const Params p) {
+  __shared__ uint32_t words[1024];  // keep bits of this query block (nb <= 32768)
+  const int i = p.nb - 1 - (int)blockIdx.x;
+  const int z = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nw = (p.nb + 31) >> 5;
+  for (int w = tid; w < nw; w += RM_NT) words[w] = 0u;
+  float c[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    c[e] = bwd_keep_bound_raw(p.LSE, (size_t)z * p.L, i * T + 4 * lane + e, p.L, p.log2_tau,
+                              p.scale_log2);
+  __syncthreads();
+  const size_t ntri = (size_t)p.nb * (p.nb + 1) / 2;
+  const float4* src = reinterpret_cast<const float4*>(
+      rowmax + ((size_t)z * ntri + (size_t)i * (i + 1) / 2) * T) + lane;
+  constexpr int NWARP = RM_NT / 32;
+  for (int j0 = warp; j0 <= i; j0 += NWARP * RM_UNROLL) {
+    float4 m[RM_UNROLL];
+#pragma unroll
+    for (int u = 0; u < RM_UNROLL; ++u) {
+      const int j = j0 + u * NWARP;
+      m[u] = j <= i ? __ldcs(src + (size_t)j * (T / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < RM_UNROLL; ++u) {
+      const int j = j0 + u * NWARP;
+      const bool want = m[u].x >= c[0] || m[u].y >= c[1] || m[u].z >= c[2] || m[u].w >= c[3];
+      if (__any_sync(0xffffffffu, want) && lane == 0 && j <= i) atomicOr(&words[j >> 5], 1u << (j & 31));
+    }
+  }
+  __syncthreads();
+  uint32_t* out = p.bits + ((size_t)z * p.nb + i) * nw;
+  for (int w = tid; w < nw; w += RM_NT) out[w] = words[w];
 }
 
 }  // namespace bwdtest

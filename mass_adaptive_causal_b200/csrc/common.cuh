@@ -45,6 +45,17 @@ __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); 
 // Keep-bit bookkeeping shared by the prefill kernels: row `rowblk` of the
 // [nb][nw] bit matrix of slice z. Thread 0 of a CTA accumulates 32 decisions
 // at a time and stores whole words, so no atomics are needed.
+// The backward's offline test for one query row, as a bound on the raw
+// (unscaled) score: the row keeps a tile iff its largest raw score in that
+// tile is >= this value. LSE is the forward's final natural log-normalizer;
+// rows past L never keep (+inf).
+__device__ __forceinline__ float bwd_keep_bound_raw(const float* LSE, size_t row_off, int row,
+                                                    int L, float log2_tau, float scale_log2) {
+  if (row >= L) return __int_as_float(0x7f800000);
+  const float c2 = LSE[row_off + row] * kLog2e + log2_tau - __log2f((float)(row + 1));
+  return c2 / scale_log2;
+}
+
 struct KeepBits {
   uint32_t* row;  // nullptr when not requested
   uint32_t word;

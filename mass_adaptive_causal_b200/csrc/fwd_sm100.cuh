@@ -73,6 +73,10 @@ struct Params {
   int never_skip;
   int32_t* kept_tiles;
   uint32_t* keep_bits;
+  // optional: raw score maximum of every row over every legal tile,
+  // [Z][i(i+1)/2 + j][T] (query block i, key block j <= i), for the
+  // backward's test
+  float* rowmax;
 };
 
 struct Bars {
@@ -281,6 +285,9 @@ __global__ void __launch_bounds__(NT, 1)
       kb.init(r == 0 ? p.keep_bits : nullptr, ((size_t)z * p.nb + iX) * nw);
       if (r == 0 && p.keep_bits)
         for (int w = iX / 32 + 1; w < nw; ++w) p.keep_bits[((size_t)z * p.nb + iX) * nw + w] = 0u;
+      float* rm = p.rowmax ? p.rowmax + ((size_t)z * ((size_t)p.nb * (p.nb + 1) / 2) +
+                                         (size_t)iX * (iX + 1) / 2) * T + r
+                           : nullptr;
 
       for (int t = 0; t < ntiles; ++t) {
         if (!MALA_PART(X, t)) continue;
@@ -291,6 +298,7 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_after();
         // ---- row max of the tile (raw scores: the positive scale commutes)
         const float mraw = tmem_rowmax128(t_s, diag, r);
+        if (rm) rm[(size_t)j * T] = mraw;
         const float mt = mraw * p.scale_log2;
         int want = diag || p.never_skip;
         if (!want && row_valid) want = mraw >= bound_raw;

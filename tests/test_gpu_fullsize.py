@@ -48,12 +48,18 @@ def prefill_run(inputs):
     P = bench.PREFILL
     shape = (P.B, P.H, P.L, P.d)
     t = {n: u16_to_dev(inputs["p" + n], shape) for n in ("Q", "K", "V", "dO")}
-    O, LSE, kept, bits, O32 = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, trace=True, o32=True)
+    O, LSE, kept, bits, O32, RM = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, trace=True,
+                                                o32=True, rowmax=True)
     dQ, dK, dV, kept_b, bits_b = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=1.0,
-                                               trace=True, o32=O32)
+                                               trace=True, o32=O32, rowmax=RM)
+    del RM
+    # the same test recomputing every tile's scores
+    *_, kept_s, bits_s = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=1.0,
+                                       trace=True, o32=O32)
     mala.mala_check()
+    same_test = torch.equal(bits_s, bits_b) and torch.equal(kept_s, kept_b)
     out = {"O": O, "LSE": LSE, "kept": kept, "bits": bits, "dQ": dQ, "dK": dK, "dV": dV,
-           "kept_b": kept_b, "bits_b": bits_b}
+           "kept_b": kept_b, "bits_b": bits_b, "same_test": same_test}
     del t
     return out
 
@@ -94,6 +100,7 @@ def test_long_128k_keep_properties(prefill_run):
         assert np.array_equal(prefill_run["kept"][0, h].cpu().numpy(), f.sum(axis=1))
         assert np.array_equal(prefill_run["kept_b"][0, h].cpu().numpy(), b.sum(axis=0))
         assert b.sum() <= f.sum()
+    assert prefill_run["same_test"]  # row-maxima test == recomputing test, bit for bit
 
 
 def test_long_128k_backward_sampled_blocks(inputs, prefill_run):

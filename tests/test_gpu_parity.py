@@ -109,14 +109,15 @@ def test_f32_ragged_shapes(L, d, B, H):
 # ----------------------------------------------------------------------------
 # bf16 tcgen05 path (128 x 128 tiles, d = 128)
 # ----------------------------------------------------------------------------
-def run_bf16_prefill(t, tau, use_o32=True):
-    """The training chain: forward (with its float32 output when use_o32),
-    then backward."""
+def run_bf16_prefill(t, tau, use_o32=True, use_rowmax=False):
+    """The training chain: forward (with its float32 output when use_o32, its
+    tile row maxima when use_rowmax), then backward."""
     O, LSE, kept, bits, *rest = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True,
-                                              o32=use_o32)
-    o32 = rest[0] if use_o32 else None
+                                              o32=use_o32, rowmax=use_rowmax)
+    o32 = rest.pop(0) if use_o32 else None
+    rm = rest.pop(0) if use_rowmax else None
     dQ, dK, dV, kept_b, bits_b = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
-                                               trace=True, o32=o32)
+                                               trace=True, o32=o32, rowmax=rm)
     mala.mala_check()
     if use_o32:  # the float32 output is the bf16 output before rounding
         assert torch.equal(o32.to(torch.bfloat16), O)
@@ -155,13 +156,45 @@ def check_bf16_slice(t, outs, b, h, tau, grads=True, o_rounded=False):
 
 @pytest.mark.parametrize("L", [128, 1000, 1536])
 @pytest.mark.parametrize("tau", [1.0, 0.0])
-def test_bf16_small_fwd_bwd(L, tau):
+@pytest.mark.parametrize("use_rowmax", [False, True])
+def test_bf16_small_fwd_bwd(L, tau, use_rowmax):
     cfg = synth.CONFIGS["matched_8k"]
     t = prefill_case(cfg, L=L, heads=[0, 1])
     t = {n: v[:, :2].contiguous() for n, v in t.items()}
-    outs = run_bf16_prefill(t, tau)
+    outs = run_bf16_prefill(t, tau, use_rowmax=use_rowmax)
     for h in range(2):
         check_bf16_slice(t, outs, 0, h, tau)
+
+
+@pytest.mark.parametrize("L,tau", [(1000, 1.0), (1536, 0.25), (2048, 1.0)])
+def test_bf16_tile_rowmax(L, tau):
+    """The forward's recorded tile row maxima against the oracle's (valid
+    rows; float32 sums of 128 exact bf16 products, bounded by 128 ulp of
+    |q| max|k|), and the backward's test from them against the test that
+    recomputes every score: the same bits, the same counts."""
+    cfg = synth.CONFIGS["matched_8k"]
+    t = prefill_case(cfg, L=L, heads=[0, 1])
+    t = {n: v[:, :2].contiguous() for n, v in t.items()}
+    O, LSE, O32, RM = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, o32=True, rowmax=True)
+    *_, kept_r, bits_r = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
+                                       trace=True, o32=O32, rowmax=RM)
+    *_, kept_s, bits_s = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
+                                       trace=True, o32=O32)
+    mala.mala_check()
+    assert torch.equal(bits_r, bits_s)
+    assert torch.equal(kept_r, kept_s)
+    nb = oracle.n_blocks(L, 128)
+    ntri = nb * (nb + 1) // 2
+    rm = RM.view(2, ntri, 128).double().cpu().numpy()
+    for h in range(2):
+        Qd, Kd = rounded(t["Q"][0, h]), rounded(t["K"][0, h])
+        ref = oracle.tile_row_max(Qd, Kd, 128)
+        kmax = np.linalg.norm(Kd, axis=1).max()
+        for i in range(nb):
+            rows = min(L - i * 128, 128)
+            bound = 128 * 2.0 ** -24 * np.linalg.norm(Qd[i * 128:i * 128 + rows], axis=1) * kmax
+            got = rm[h, i * (i + 1) // 2:i * (i + 1) // 2 + i + 1, :rows]
+            assert np.all(np.abs(got - ref[i][:, :rows]) <= bound[None, :] + 1e-30), i
 
 
 @pytest.mark.parametrize("L", [1000])
@@ -190,7 +223,7 @@ def test_bf16_matched_work_config_full():
     """B=1 H=8 L=8192 d=128 bf16 tile 128 tau=1: every head, every output."""
     cfg = synth.CONFIGS["matched_8k"]
     t = prefill_case(cfg)
-    outs = run_bf16_prefill(t, 1.0)
+    outs = run_bf16_prefill(t, 1.0, use_rowmax=True)
     for h in range(cfg.H):
         check_bf16_slice(t, outs, 0, h, 1.0)
 
