@@ -14,13 +14,17 @@
 // share every K tile: K_{2c+1} (B's diagonal, B only), then K_{2c} ... K_0
 // for both. Sharing halves the L2 -> SM traffic per tensor-core FLOP.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3  softmax/test warpgroup of A (thread r owns query row r = TMEM lane r)
 //   warps 4-7  softmax/test warpgroup of B
 //   warp  8    TMA producer: Q_A, Q_B, then the K ring (3 stages)
-//   warp  9    MMA issuer (one thread): QK^T and PV, ping-ponging A and B so
-//              the tensor pipe computes one block's scores while the other
-//              block's warpgroup runs its test
+//   warp  9    MMA issuer of A (one thread): QK^T and PV of block A
+//   warp  10   MMA issuer of B
+// The two blocks ping-pong on the tensor pipe: one block's scores are
+// computed while the other block's warpgroup runs its test. An issuing
+// thread's own shared-memory reads (its mbarrier polls) wait for the MMAs it
+// has queued, so each block gets its own issuer: while A's issuer waits for
+// A's decision, B's MMAs stay queued and the pipe does not drain.
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 // A kept tile's P = exp2(s2 - m) is written back over its own S columns as
 // bf16 pairs: each 32-column chunk holds 16 columns of P_hi and 16 of P_lo
@@ -45,9 +49,10 @@ using namespace sm100;
 
 constexpr int T = 128;
 constexpr int D = 128;
-constexpr int NT = 320;
+constexpr int NT = 352;  // 11 warps: 3 share a sub-partition, so at most 168 registers
 constexpr int WARP_PRODUCER = 8;
-constexpr int WARP_MMA = 9;
+constexpr int WARP_MMA_A = 9;   // issues block A's MMAs; allocates TMEM
+constexpr int WARP_MMA_B = 10;  // issues block B's MMAs
 constexpr int NSTAGE = 3;
 constexpr uint32_t TILE_BYTES = T * D * 2;   // 32 KB
 constexpr uint32_t HALF_BYTES = T * 64 * 2;  // one 64-column swizzled block
@@ -153,7 +158,7 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(smem_u32(&bars.q_full), 1);
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(smem_u32(&bars.k_full[s]), 1);
-      mbar_init(smem_u32(&bars.k_empty[s]), 1);
+      mbar_init(smem_u32(&bars.k_empty[s]), 2);  // one commit per issuer
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(smem_u32(&bars.s_full[x]), 1);
@@ -164,7 +169,7 @@ __global__ void __launch_bounds__(NT, 1)
     bars.abort = 0;
     fence_mbar_init();
   }
-  if (warp == WARP_MMA) {
+  if (warp == WARP_MMA_A) {
     tmem_alloc(smem_u32(&bars.tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
@@ -200,63 +205,61 @@ __global__ void __launch_bounds__(NT, 1)
       }
     }
     __syncwarp();
-  } else if (warp == WARP_MMA) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == WARP_MMA_A || warp == WARP_MMA_B) {
+    // ----------------------------------------------- MMA issuers (one per block)
+    // Each block has its own issuing thread, so that one issuer waiting for
+    // its block's decision never holds back the other block's MMAs: the
+    // tensor pipe keeps the other block's work queued meanwhile.
+    const int X = warp - WARP_MMA_A;
     if (lane == 0) {
       mbar_wait(smem_u32(&bars.q_full), 0, abort, 0x112);
-      uint32_t dec_ph[2] = {0, 0}, v_ph[2] = {0, 0};
-      int pv_count[2] = {0, 0};
+      uint32_t dec_ph = 0, v_ph = 0;
+      int pv_count = 0;
       // base descriptors, computed once
-      const uint64_t dq0 = sdesc_sw128(sbase + OFF_Q, 16, 1024);
-      const uint64_t dq1 = sdesc_sw128(sbase + OFF_Q + TILE_BYTES, 16, 1024);
+      const uint64_t dq = sdesc_sw128(sbase + OFF_Q + X * TILE_BYTES, 16, 1024);
       uint64_t dks[NSTAGE];
 #pragma unroll
       for (int st = 0; st < NSTAGE; ++st) dks[st] = sdesc_sw128(sbase + OFF_K + st * TILE_BYTES, 16, 1024);
-      const uint64_t dv0 = sdesc_sw128(sbase + OFF_V, HALF_BYTES, 1024);
-      const uint64_t dv1 = sdesc_sw128(sbase + OFF_V + TILE_BYTES, HALF_BYTES, 1024);
+      const uint64_t dv = sdesc_sw128(sbase + OFF_V + X * TILE_BYTES, HALF_BYTES, 1024);
       auto kdesc = [&](int t) -> uint64_t {
         const int st = t % NSTAGE;
         return st == 0 ? dks[0] : (st == 1 ? dks[1] : dks[2]);
       };
-      wait_k_full(bars, 0, abort);
-#pragma unroll
-      for (int X = 0; X < 2; ++X)
-        if (MALA_PART(X, 0)) issue_qk(bars, tmem, X, X ? dq1 : dq0, kdesc(0));
+      // Both issuers commit k_empty once per tile (count 2), whether or not
+      // their block takes part in it.
+      if (MALA_PART(X, 0)) {
+        wait_k_full(bars, 0, abort);
+        issue_qk(bars, tmem, X, dq, kdesc(0));
+      }
       mma_commit(smem_u32(&bars.k_empty[0]));
       for (int t = 0; t < ntiles; ++t) {
-        bool k_next_ready = false;
+        if (MALA_PART(X, t)) {
+          mbar_wait_spin(smem_u32(&bars.decision[X]), dec_ph, abort, 0x114);
+          dec_ph ^= 1;
+          if (*reinterpret_cast<volatile int*>(&bars.keepflag[X])) {
+            mbar_wait(smem_u32(&bars.v_full[X]), v_ph, abort, 0x115);
+            v_ph ^= 1;
+            tc_fence_after();
 #pragma unroll
-        for (int X = 0; X < 2; ++X) {
-          if (MALA_PART(X, t)) {
-            mbar_wait_spin(smem_u32(&bars.decision[X]), dec_ph[X], abort, 0x114);
-            dec_ph[X] ^= 1;
-            if (*reinterpret_cast<volatile int*>(&bars.keepflag[X])) {
-              mbar_wait(smem_u32(&bars.v_full[X]), v_ph[X], abort, 0x115);
-              v_ph[X] ^= 1;
-              tc_fence_after();
-              const uint64_t dv = X ? dv1 : dv0;
+            for (int half = 0; half < 2; ++half) {
 #pragma unroll
-              for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                for (int kk = 0; kk < T / 16; ++kk) {
-                  const uint32_t a_t = tmem + X * 128 + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half;
-                  mma_bf16_ts(tmem + 256 + X * 128, a_t, dv + (uint64_t)((kk * 2048) >> 4),
-                              IDESC_PV, (pv_count[X] > 0 || half > 0 || kk > 0) ? 1u : 0u);
-                }
+              for (int kk = 0; kk < T / 16; ++kk) {
+                const uint32_t a_t = tmem + X * 128 + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half;
+                mma_bf16_ts(tmem + 256 + X * 128, a_t, dv + (uint64_t)((kk * 2048) >> 4),
+                            IDESC_PV, (pv_count > 0 || half > 0 || kk > 0) ? 1u : 0u);
               }
-              mma_commit(smem_u32(&bars.pv_done[X]));
-              ++pv_count[X];
             }
-          }
-          if (t + 1 < ntiles && MALA_PART(X, t + 1)) {
-            if (!k_next_ready) {
-              wait_k_full(bars, t + 1, abort);
-              k_next_ready = true;
-            }
-            issue_qk(bars, tmem, X, X ? dq1 : dq0, kdesc(t + 1));
+            mma_commit(smem_u32(&bars.pv_done[X]));
+            ++pv_count;
           }
         }
-        if (t + 1 < ntiles) mma_commit(smem_u32(&bars.k_empty[(t + 1) % NSTAGE]));
+        if (t + 1 < ntiles) {
+          if (MALA_PART(X, t + 1)) {
+            wait_k_full(bars, t + 1, abort);
+            issue_qk(bars, tmem, X, dq, kdesc(t + 1));
+          }
+          mma_commit(smem_u32(&bars.k_empty[(t + 1) % NSTAGE]));
+        }
       }
     }
     __syncwarp();
@@ -298,7 +301,6 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_after();
         // ---- row max of the tile (raw scores: the positive scale commutes)
         const float mraw = tmem_rowmax128(t_s, diag, r);
-        if (rm) rm[(size_t)j * T] = mraw;
         const float mt = mraw * p.scale_log2;
         int want = diag || p.never_skip;
         if (!want && row_valid) want = mraw >= bound_raw;
@@ -310,8 +312,12 @@ __global__ void __launch_bounds__(NT, 1)
             bars.keepflag[X] = 0;
             mbar_arrive(smem_u32(&bars.decision[X]));
           }
+          // global stores after the decision, so the arrive (a release) and
+          // the vote's barrier never wait for them
+          if (rm) rm[(size_t)j * T] = mraw;
           continue;
         }
+        if (rm) rm[(size_t)j * T] = mraw;
         // ---- kept tile ----------------------------------------------------
         if (n_kept > 0) {  // the previous PV of this block reads V_X and O_X
           mbar_wait(smem_u32(&bars.pv_done[X]), (n_kept - 1) & 1, abort, 0x117);
@@ -410,7 +416,7 @@ __global__ void __launch_bounds__(NT, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == WARP_MMA) {
+  if (warp == WARP_MMA_A) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
