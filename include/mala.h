@@ -80,13 +80,19 @@ typedef enum { MALA_F32 = 0, MALA_BF16 = 1 } mala_dtype;
  *         D = <dO, O> feed dQ through a sum over keys whose rows cancel, so
  *         D computed from a bf16-rounded O costs dQ percents of accuracy when
  *         keys share a large common component.
- *         tile_rowmax (may be NULL; MALA_BF16 only): float32, for every
- *         legal tile (query block i, key block j <= i) and every row r of
- *         block i, the largest raw score q_r . k_c (unscaled) over the
- *         tile's keys c <= row; laid out [B][H][i(i+1)/2 + j][tile]
- *         (mala_tile_rowmax_bytes). Values of rows past L are unspecified.
- *         Pass it to mala_bwd: the backward's skip test then reads these
- *         maxima instead of recomputing every tile's scores.
+ *         tile_rowmax (may be NULL; MALA_BF16 only; mala_tile_rowmax_bytes
+ *         bytes): what the backward's skip test needs from this pass. Part
+ *         1, float32 [B][H][i(i+1)/2 + j][tile]: for legal tile (query block
+ *         i, key block j <= i) and row r of block i, the largest raw score
+ *         q_r . k_c (unscaled) over the tile's keys c <= row. Part 2 (from
+ *         the next 256-byte boundary), uint32 [B][H][nb][ceil(nb/32)]: bit j
+ *         of row i set iff tile (i, j)'s maxima were stored. They are stored
+ *         for every kept tile and for skipped tiles with some row within a
+ *         relative 1e-3 of the forward's bound; every other tile fails the
+ *         backward's test (the final normalizer only raises the bound), so
+ *         its maxima are not needed. Rows past L are unspecified. Pass the
+ *         buffer to mala_bwd: its skip test then reads the stored maxima
+ *         instead of recomputing every tile's scores.
  * Trace   kept_tiles: [B][H][nb] kept key tiles per query block;
  *         keep_bits: [B][H][nb][ceil(nb/32)], row = query block, bit = key
  *         block. nb = ceil(L / tile).
@@ -99,9 +105,11 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O,
                      int L, int d, mala_dtype dt, float tau, int tile, float scale,
                      int32_t* kept_tiles, uint32_t* keep_bits, void* stream);
 
-/* Bytes of the forward's optional tile_rowmax output:
- * B * H * nb(nb+1)/2 * tile * 4 for nb = ceil(L / tile) (2 GiB for B = 1,
- * H = 8, L = 131072, tile = 128). 0 for invalid sizes. */
+/* Bytes of the forward's optional tile_rowmax output: B * H * nb(nb+1)/2 *
+ * tile * 4 (maxima) plus B * H * nb * ceil(nb/32) * 4 (flags), each rounded
+ * up to 256, for nb = ceil(L / tile): 2 GiB for B = 1, H = 8, L = 131072,
+ * tile = 128, of which the forward writes only the flagged tiles (a few
+ * percent when most tiles are skipped). 0 for invalid sizes. */
 size_t mala_tile_rowmax_bytes(int B, int H, int L, int tile);
 
 /* Bytes of device workspace mala_bwd needs: the row terms D (float32

@@ -28,6 +28,22 @@ namespace host {
 // shared memory: nb <= 32768 blocks of 128 rows.
 constexpr int kMaxRowmaxL = 32768 * 128;
 
+// The forward's tile row maxima buffer: the maxima [Z][nb(nb+1)/2][tile]
+// float32, then one flag bit per tile [Z][nb][ceil(nb/32)] saying which
+// tiles' maxima were stored, each part rounded up to 256 bytes.
+inline size_t rowmax_maxima_bytes(size_t Z, size_t L, size_t tile) {
+  const size_t nb = (L + tile - 1) / tile;
+  return (Z * (nb * (nb + 1) / 2) * tile * sizeof(float) + 255) & ~size_t(255);
+}
+inline size_t rowmax_flag_bytes(size_t Z, size_t L, size_t tile) {
+  const size_t nb = (L + tile - 1) / tile;
+  return (Z * nb * ((nb + 31) / 32) * sizeof(uint32_t) + 255) & ~size_t(255);
+}
+inline uint32_t* rowmax_flags(const float* rowmax, size_t Z, size_t L, size_t tile) {
+  return reinterpret_cast<uint32_t*>(
+      const_cast<char*>(reinterpret_cast<const char*>(rowmax)) + rowmax_maxima_bytes(Z, L, tile));
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline bool tau_ok(float tau) { return isfinite(tau) && tau >= 0.f; }
@@ -124,6 +140,7 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
   p.kept_tiles = kept;
   p.keep_bits = bits;
   p.rowmax = rowmax;
+  p.rm_bits = rowmax ? rowmax_flags(rowmax, Z, L, fwd100::T) : nullptr;
   MALA_CUDA_TRY(cudaFuncSetAttribute(fwd100::fwd_bf16_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)fwd100::SMEM_BYTES));
@@ -238,7 +255,8 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
     tp.log2_tau = log2f(tau);
     tp.bits = tile_bits;
     if (rowmax) {  // from the forward's recorded tile row maxima
-      bwdtest::rowmax_test_kernel<<<dim3(nb, Z), bwdtest::RM_NT, 0, s>>>(rowmax, tp);
+      bwdtest::rowmax_test_kernel<<<dim3(nb, Z), bwdtest::RM_NT, 0, s>>>(
+          rowmax, rowmax_flags(rowmax, Z, L, bwd100::T), tp);
     } else {       // recompute every tile's scores
       MALA_CUDA_TRY(cudaFuncSetAttribute(bwdtest::test_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -420,8 +438,7 @@ static mala_status check_prefill_shape(int B, int H, int L, int d, mala_dtype dt
 
 size_t mala_tile_rowmax_bytes(int B, int H, int L, int tile) {
   if (B < 1 || H < 1 || L < 0 || tile < 1) return 0;
-  const size_t nb = ((size_t)L + tile - 1) / tile;
-  return (size_t)B * H * (nb * (nb + 1) / 2) * tile * sizeof(float);
+  return rowmax_maxima_bytes((size_t)B * H, L, tile) + rowmax_flag_bytes((size_t)B * H, L, tile);
 }
 
 mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE,

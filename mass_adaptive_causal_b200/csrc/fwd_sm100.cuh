@@ -78,11 +78,22 @@ struct Params {
   int never_skip;
   int32_t* kept_tiles;
   uint32_t* keep_bits;
-  // optional: raw score maximum of every row over every legal tile,
-  // [Z][i(i+1)/2 + j][T] (query block i, key block j <= i), for the
-  // backward's test
+  // optional, for the backward's test: raw score maxima of every row,
+  // [Z][i(i+1)/2 + j][T] (query block i, key block j <= i), written only for
+  // the tiles whose maxima can decide that test (see kNearSkip) and flagged
+  // in rm_bits [Z][nb][ceil(nb/32)] (bit j of row i: tile (i, j) stored)
   float* rowmax;
+  uint32_t* rm_bits;
 };
+
+// The backward keeps tile (i, j) iff some row's maximum reaches the bound set
+// by the final log-normalizer, which is never below the partial one the
+// forward tests against (the normalizer only grows as tiles are added). A
+// tile the forward skips with every row's maximum below its bound by more
+// than this relative margin therefore fails the backward's test too, whatever
+// the rounding of either bound; its maxima are not stored. Kept tiles and
+// tiles skipped by less are stored.
+constexpr float kNearSkip = 1e-3f;
 
 struct Bars {
   uint64_t q_full;
@@ -291,6 +302,10 @@ __global__ void __launch_bounds__(NT, 1)
       float* rm = p.rowmax ? p.rowmax + ((size_t)z * ((size_t)p.nb * (p.nb + 1) / 2) +
                                          (size_t)iX * (iX + 1) / 2) * T + r
                            : nullptr;
+      KeepBits kbs;  // which tiles' maxima are stored
+      kbs.init(r == 0 ? p.rm_bits : nullptr, ((size_t)z * p.nb + iX) * nw);
+      if (r == 0 && p.rm_bits)
+        for (int w = iX / 32 + 1; w < nw; ++w) p.rm_bits[((size_t)z * p.nb + iX) * nw + w] = 0u;
 
       for (int t = 0; t < ntiles; ++t) {
         if (!MALA_PART(X, t)) continue;
@@ -312,12 +327,21 @@ __global__ void __launch_bounds__(NT, 1)
             bars.keepflag[X] = 0;
             mbar_arrive(smem_u32(&bars.decision[X]));
           }
-          // global stores after the decision, so the arrive (a release) and
-          // the vote's barrier never wait for them
-          if (rm) rm[(size_t)j * T] = mraw;
+          // after the decision (off the issuer's path): is any row close
+          // enough to its bound that the backward's test could keep the tile?
+          if (rm) {
+            const bool near =
+                row_valid && mraw >= bound_raw - kNearSkip * (1.f + fabsf(bound_raw));
+            const int store = wg_vote_or(near, bar_id);
+            if (store) rm[(size_t)j * T] = mraw;
+            kbs.set(j, store != 0);
+          }
           continue;
         }
-        if (rm) rm[(size_t)j * T] = mraw;
+        if (rm) {
+          rm[(size_t)j * T] = mraw;
+          kbs.set(j, true);
+        }
         // ---- kept tile ----------------------------------------------------
         if (n_kept > 0) {  // the previous PV of this block reads V_X and O_X
           mbar_wait(smem_u32(&bars.pv_done[X]), (n_kept - 1) & 1, abort, 0x117);
@@ -381,6 +405,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
       kb.flush();
+      kbs.flush();
       // ---- epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2 -------------------
       mbar_wait(smem_u32(&bars.pv_done[X]), (n_kept - 1) & 1, abort, 0x118);
       tc_fence_after();

@@ -166,16 +166,31 @@ def test_bf16_small_fwd_bwd(L, tau, use_rowmax):
         check_bf16_slice(t, outs, 0, h, tau)
 
 
+def rowmax_parts(RM, Z, L, T=128):
+    """Split the forward's row-maxima buffer into maxima [Z, ntri, T] and the
+    per-tile stored flags [Z, nb, nb] (host numpy)."""
+    nb = oracle.n_blocks(L, T)
+    ntri = nb * (nb + 1) // 2
+    r256 = lambda x: (x + 255) // 256 * 256
+    nmax = r256(Z * ntri * T * 4) // 4
+    nw = (nb + 31) // 32
+    maxima = RM[:Z * ntri * T].view(Z, ntri, T).double().cpu().numpy()
+    flags = RM[nmax:nmax + Z * nb * nw].view(torch.int32).view(Z, nb, nw)
+    return maxima, mala.unpack_bits(flags, nb)
+
+
 @pytest.mark.parametrize("L,tau", [(1000, 1.0), (1536, 0.25), (2048, 1.0)])
 def test_bf16_tile_rowmax(L, tau):
     """The forward's recorded tile row maxima against the oracle's (valid
-    rows; float32 sums of 128 exact bf16 products, bounded by 128 ulp of
-    |q| max|k|), and the backward's test from them against the test that
-    recomputes every score: the same bits, the same counts."""
+    rows of every stored tile; float32 sums of 128 exact bf16 products,
+    bounded by 128 ulp of |q| max|k|); every tile the forward kept is stored;
+    and the backward's test from them equals the test that recomputes every
+    score: the same bits, the same counts."""
     cfg = synth.CONFIGS["matched_8k"]
     t = prefill_case(cfg, L=L, heads=[0, 1])
     t = {n: v[:, :2].contiguous() for n, v in t.items()}
-    O, LSE, O32, RM = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, o32=True, rowmax=True)
+    O, LSE, kept, fbits, O32, RM = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True,
+                                                 o32=True, rowmax=True)
     *_, kept_r, bits_r = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
                                        trace=True, o32=O32, rowmax=RM)
     *_, kept_s, bits_s = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
@@ -184,8 +199,11 @@ def test_bf16_tile_rowmax(L, tau):
     assert torch.equal(bits_r, bits_s)
     assert torch.equal(kept_r, kept_s)
     nb = oracle.n_blocks(L, 128)
-    ntri = nb * (nb + 1) // 2
-    rm = RM.view(2, ntri, 128).double().cpu().numpy()
+    maxima, stored = rowmax_parts(RM, 2, L)
+    fkeep = mala.unpack_bits(fbits, nb)[0]
+    assert np.all(stored[fkeep == 1] == 1)
+    assert not np.any(np.triu(stored[0], 1)) and not np.any(np.triu(stored[1], 1))
+    n_checked = 0
     for h in range(2):
         Qd, Kd = rounded(t["Q"][0, h]), rounded(t["K"][0, h])
         ref = oracle.tile_row_max(Qd, Kd, 128)
@@ -193,8 +211,11 @@ def test_bf16_tile_rowmax(L, tau):
         for i in range(nb):
             rows = min(L - i * 128, 128)
             bound = 128 * 2.0 ** -24 * np.linalg.norm(Qd[i * 128:i * 128 + rows], axis=1) * kmax
-            got = rm[h, i * (i + 1) // 2:i * (i + 1) // 2 + i + 1, :rows]
-            assert np.all(np.abs(got - ref[i][:, :rows]) <= bound[None, :] + 1e-30), i
+            for j in np.nonzero(stored[h, i, :i + 1])[0]:
+                got = maxima[h, i * (i + 1) // 2 + j, :rows]
+                assert np.all(np.abs(got - ref[i][j, :rows]) <= bound + 1e-30), (i, j)
+                n_checked += 1
+    assert n_checked > 0
 
 
 @pytest.mark.parametrize("L", [1000])
