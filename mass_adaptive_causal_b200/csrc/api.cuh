@@ -11,6 +11,7 @@
 #include "bwd_sm100.cuh"
 #include "bwd_test_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "fwd2_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "mala.h"
 #include "simt_f32.cuh"
@@ -72,13 +73,14 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // bf16 tensor [Z][rows][128] seen as 3-D (x = d, y = row, z = slice), box
-// 64 x 128 x 1 with 128-byte swizzle; rows past `rows` read as zero.
-inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t Z) {
+// 64 x box_rows x 1 with 128-byte swizzle; rows past `rows` read as zero.
+inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t Z,
+                     uint32_t box_rows = 128) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {128, rows, Z};
   cuuint64_t strides[2] = {128 * 2, rows * 128 * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   memset(m, 0, sizeof(*m));
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
@@ -124,15 +126,17 @@ inline mala_status fwd_f32(const float* Q, const float* K, const float* V, float
 inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O, float* LSE,
                             float* O32, float* rowmax, int Z, int L, float scale, float tau,
                             int32_t* kept, uint32_t* bits, cudaStream_t s) {
+  // Q and V in 128-row boxes; K in 64-row boxes (each CTA of a pair loads
+  // half of every key tile)
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, L, Z) || !make_map(&mk, K, L, Z) || !make_map(&mv, V, L, Z))
+  if (!make_map(&mq, Q, L, Z) || !make_map(&mk, K, L, Z, 64) || !make_map(&mv, V, L, Z))
     return MALA_ERR_CUDA;
-  fwd100::Params p;
+  fwd2::Params p;
   p.O = reinterpret_cast<__nv_bfloat16*>(O);
   p.O32 = O32;
   p.LSE = LSE;
   p.L = L;
-  p.nb = (L + fwd100::T - 1) / fwd100::T;
+  p.nb = (L + fwd2::T - 1) / fwd2::T;
   p.npairs = (p.nb + 1) / 2;
   p.scale_log2 = scale * kLog2e;
   p.never_skip = tau == 0.f;
@@ -140,11 +144,23 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
   p.kept_tiles = kept;
   p.keep_bits = bits;
   p.rowmax = rowmax;
-  p.rm_bits = rowmax ? rowmax_flags(rowmax, Z, L, fwd100::T) : nullptr;
-  MALA_CUDA_TRY(cudaFuncSetAttribute(fwd100::fwd_bf16_kernel,
+  p.rm_bits = rowmax ? rowmax_flags(rowmax, Z, L, fwd2::T) : nullptr;
+  MALA_CUDA_TRY(cudaFuncSetAttribute(fwd2::fwd_pair_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)fwd100::SMEM_BYTES));
-  fwd100::fwd_bf16_kernel<<<dim3(p.npairs, Z), fwd100::NT, fwd100::SMEM_BYTES, s>>>(mq, mk, mv, p);
+                                     (int)fwd2::SMEM_BYTES));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * p.npairs, Z, 1);
+  cfg.blockDim = dim3(fwd2::NT, 1, 1);
+  cfg.dynamicSmemBytes = fwd2::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  MALA_CUDA_TRY(cudaLaunchKernelEx(&cfg, fwd2::fwd_pair_kernel, mq, mk, mv, p));
   return launch_status();
 }
 
