@@ -570,9 +570,9 @@ def main():
     dominant = "fwd" if t1["fwd_ms"] >= t1["bwd_ms"] else "bwd"
     traffic = load_profile_traffic()
     if dominant == "fwd":
-        roof = {"bound": "tensor", "kernel": "mala::fwd100::fwd_bf16_kernel", "achieved": fwd_tf,
+        roof = {"bound": "tensor", "kernel": "mala::fwd2::fwd_pair_kernel", "achieved": fwd_tf,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": fwd_tf / peaks["bf16_tflops"],
-                "traffic": traffic.get("fwd_bf16_kernel")}
+                "traffic": traffic.get("fwd_pair_kernel")}
     else:
         roof = {"bound": "tensor", "kernel": "mala::bwd100::bwd_bf16_kernel", "achieved": bwd_tf,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": bwd_tf / peaks["bf16_tflops"],
