@@ -495,6 +495,69 @@ def profile_case(args):
                       "ms_per_launch": s.elapsed_time(e) / args.launches}), flush=True)
 
 
+def tau_study(args):
+    """Slots per query, omitted mass and output error against dense attention
+    over a sweep of tau, on the long_128k prefill and the decode_128k step
+    (group rows and per-head rows). The omitted mass of row r is
+    1 - exp(LSE_tau - LSE_dense): LSE_tau normalizes over the kept keys only.
+    Everything runs on the GPU kernels; one JSON line."""
+    import torch
+    import mass_adaptive_causal_b200 as mala
+    torch.cuda.set_device(0)
+    P, Dc = PREFILL, DECODE
+    x = generate_inputs(args.workers or min(16, os.cpu_count() or 1))
+
+    def to_dev(u16, shape):
+        return torch.from_numpy(u16.view(np.int16)).view(torch.bfloat16).reshape(shape).cuda()
+
+    pshape = (P.B, P.H, P.L, P.d)
+    Q, K, V = (to_dev(x["p" + n], pshape) for n in ("Q", "K", "V"))
+    O0, L0 = mala.mala_fwd(Q, K, V, tau=0.0)
+
+    def timed(fn, reps=3):
+        fn()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(reps):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        return s.elapsed_time(e) / reps
+
+    rows = []
+    for tau in (0.0625, 0.25, 1.0, 4.0, 16.0):
+        O, LSE, kept, bits = mala.mala_fwd(Q, K, V, tau=tau, trace=True)
+        mala.mala_check()
+        om = (1.0 - torch.exp(LSE.double() - L0.double())).clamp_min(0.0)
+        rel = float(torch.linalg.norm((O.float() - O0.float()).flatten()) /
+                    torch.linalg.norm(O0.float().flatten()))
+        rows.append({"tau": tau, "fwd_ms": timed(lambda: mala.mala_fwd(Q, K, V, tau=tau)),
+                     "slots_per_query": retained_pairs(bits, P.L, P.tile) / (P.B * P.H * P.L),
+                     "omitted_mass_mean": float(om.mean()), "omitted_mass_max": float(om.max()),
+                     "bound_tau_over_1_plus_tau": tau / (1 + tau), "out_rel_l2_vs_dense": rel})
+    del Q, K, V, O0, L0
+    q = to_dev(x["dq"], (Dc.B, Dc.Hq, Dc.d))
+    Kc = to_dev(x["dK"], (Dc.B, Dc.Hkv, Dc.Lc, Dc.d))
+    Vc = to_dev(x["dV"], (Dc.B, Dc.Hkv, Dc.Lc, Dc.d))
+    o0 = mala.mala_decode(q, Kc, Vc, tau=0.0)
+    nt = (Dc.Lc + 127) // 128
+    drows = []
+    for per_head in (False, True):
+        for tau in (0.25, 1.0, 4.0):
+            o, kept, _ = mala.mala_decode(q, Kc, Vc, tau=tau, trace=True, per_head=per_head)
+            mala.mala_check()
+            units = Dc.Hq if per_head else Dc.Hkv
+            rel = float(torch.linalg.norm((o.float() - o0.float()).flatten()) /
+                        torch.linalg.norm(o0.float().flatten()))
+            drows.append({"rows": "per_head" if per_head else "group", "tau": tau,
+                          "decode_us": 1000 * timed(lambda: mala.mala_decode(
+                              q, Kc, Vc, tau=tau, per_head=per_head)),
+                          "kept_tile_frac": float(kept.sum()) / (Dc.B * units * nt),
+                          "out_rel_l2_vs_dense": rel})
+    print(json.dumps({"study": "tau_sweep", "prefill": {"workload": "long_128k", "rows": rows},
+                      "decode": {"workload": "decode_128k", "rows": drows}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -509,9 +572,13 @@ def main():
                     help="run only a small case of one call (for ncu captures)")
     ap.add_argument("--L", type=int, default=32768, help="sequence length of --profile")
     ap.add_argument("--launches", type=int, default=2, help="timed launches of --profile")
+    ap.add_argument("--study", choices=["tau"], default=None,
+                    help="tau sweep: slots, omitted mass and error against dense, one JSON line")
     args = ap.parse_args()
     if args.profile:
         return profile_case(args)
+    if args.study == "tau":
+        return tau_study(args)
     args.warmup = max(3, args.warmup)
 
     rank = int(os.environ.get("RANK", "0"))

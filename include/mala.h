@@ -165,23 +165,26 @@ size_t mala_decode_workspace_bytes(int B, int Hq, int Hkv, int Lc, int d);
  *
  * The cache holds Lc keys per (b, kv head) including the current token, so
  * Lq = Lc. Key tiles of 128 positions are aligned from position 0 and
- * visited newest first; the newest tile is always kept. The rows of a tile
- * are the G = Hq / Hkv query heads that share the KV head, and the tile is
- * skipped iff every one of them is below the threshold (tile granularity is
- * conservative). Kept tiles update the per-head online softmax; the output is
- * softmax over the kept tiles.
+ * visited newest first; the newest tile is always kept. With per_head = 0
+ * the rows of a tile are the G = Hq / Hkv query heads that share the KV
+ * head, and the tile is skipped iff every one of them is below the threshold
+ * (tile granularity is conservative). With per_head = 1 every query head
+ * applies the test alone, with its own running statistics (finer skipping;
+ * a tile's K and V are still read once for all heads that kept it). Kept
+ * tiles update the per-head online softmax; the output is softmax over the
+ * kept tiles.
  *
  * Inputs  q: [B][Hq][d] bf16; Kcache, Vcache: [B][Hkv][Lc][d] bf16.
  * Output  o: [B][Hq][d] bf16.
  * workspace: at least mala_decode_workspace_bytes(B,Hq,Hkv,Lc,d) bytes.
  * Trace   kept_tiles: [B][Hkv]; keep_bits: [B][Hkv][ceil(nt/32)], nt =
- *         ceil(Lc / 128).
+ *         ceil(Lc / 128); with per_head = 1, [B][Hq] and [B][Hq][ceil(nt/32)].
  * Supported: d = 128, Hq % Hkv == 0, 1 <= Hq / Hkv <= 8, B * Hkv <= 4095,
  *            Lc >= 1.
  */
 mala_status mala_decode(const void* q, const void* Kcache, const void* Vcache,
                         void* o, int B, int Hq, int Hkv, int Lc, int d,
-                        float tau, float scale, void* workspace,
+                        float tau, float scale, int per_head, void* workspace,
                         size_t workspace_bytes, int32_t* kept_tiles,
                         uint32_t* keep_bits, void* stream);
 

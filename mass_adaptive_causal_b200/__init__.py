@@ -61,8 +61,8 @@ def lib() -> ctypes.CDLL:
         L.mala_bwd.restype = ci
         L.mala_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
         L.mala_decode_workspace_bytes.restype = cs
-        L.mala_decode.argtypes = [_vp, _vp, _vp, _vp, ci, ci, ci, ci, ci, cf, cf, _vp, cs, _i32p,
-                                  _u32p, _vp]
+        L.mala_decode.argtypes = [_vp, _vp, _vp, _vp, ci, ci, ci, ci, ci, cf, cf, ci, _vp, cs,
+                                  _i32p, _u32p, _vp]
         L.mala_decode.restype = ci
         L.mala_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, ci, ci, ci, ci, ci, cf, cf, _i32p,
                                           _u32p, _vp]
@@ -217,10 +217,11 @@ def decode_workspace_bytes(B, Hq, Hkv, Lc, d) -> int:
 
 
 def mala_decode(q, k_cache, v_cache, tau: float = 1.0, scale: float = 0.0, trace: bool = False,
-                workspace=None, out=None, stream=None):
+                workspace=None, out=None, stream=None, per_head: bool = False):
     """One decode step. q: [B, Hq, d] bf16; caches: [B, Hkv, Lc, d] bf16.
     Returns o [B, Hq, d] or, with ``trace=True``, (o, kept_tiles [B, Hkv],
-    keep_bits [B, Hkv, nw])."""
+    keep_bits [B, Hkv, nw]); with ``per_head=True`` every query head applies
+    the test alone and the trace is per query head ([B, Hq], [B, Hq, nw])."""
     torch = _torch()
     for t in (q, k_cache, v_cache):
         if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
@@ -234,11 +235,12 @@ def mala_decode(q, k_cache, v_cache, tau: float = 1.0, scale: float = 0.0, trace
     kept = bits = None
     if trace:
         nt = n_blocks(Lc, 128)
-        kept = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
-        bits = torch.empty((B, Hkv, (nt + 31) // 32), dtype=torch.int32, device=q.device)
+        rows = Hq if per_head else Hkv
+        kept = torch.empty((B, rows), dtype=torch.int32, device=q.device)
+        bits = torch.empty((B, rows, (nt + 31) // 32), dtype=torch.int32, device=q.device)
     code = lib().mala_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), B, Hq, Hkv, Lc, d,
-                             float(tau), float(scale), _ptr(ws), ws.numel(), _ptr(kept),
-                             _ptr(bits), _stream(stream))
+                             float(tau), float(scale), int(bool(per_head)), _ptr(ws), ws.numel(),
+                             _ptr(kept), _ptr(bits), _stream(stream))
     _raise(code, "mala_decode")
     return (o, kept, bits) if trace else o
 

@@ -318,13 +318,14 @@ struct DecWorkspace {
   float* mfin;
   float* lfin;
   float* oacc;
+  uint8_t* head_mask;
 };
 inline size_t dec_ws_bytes(size_t B, size_t Hq, size_t Hkv, size_t Lc, size_t d) {
   const size_t groups = B * Hkv;
   const size_t nt = (Lc + 127) / 128;
   return round256(B * Hq * nt * sizeof(float2)) + round256(groups * nt * sizeof(int)) +
          round256(groups * sizeof(int)) + 2 * round256(B * Hq * sizeof(float)) +
-         round256(B * Hq * d * sizeof(float));
+         round256(B * Hq * d * sizeof(float)) + round256(groups * nt);
 }
 inline DecWorkspace dec_ws_carve(void* ws, size_t B, size_t Hq, size_t Hkv, size_t Lc, size_t d) {
   const size_t groups = B * Hkv;
@@ -342,12 +343,15 @@ inline DecWorkspace dec_ws_carve(void* ws, size_t B, size_t Hq, size_t Hkv, size
   w.lfin = reinterpret_cast<float*>(p);
   p += round256(B * Hq * sizeof(float));
   w.oacc = reinterpret_cast<float*>(p);
+  p += round256(B * Hq * d * sizeof(float));
+  w.head_mask = reinterpret_cast<uint8_t*>(p);
   return w;
 }
 
 inline mala_status decode_bf16(const void* q, const void* Kc, const void* Vc, void* o, int B,
-                               int Hq, int Hkv, int Lc, float scale, float tau, DecWorkspace w,
-                               int32_t* kept_tiles, uint32_t* bits, cudaStream_t s) {
+                               int Hq, int Hkv, int Lc, float scale, float tau, int per_head,
+                               DecWorkspace w, int32_t* kept_tiles, uint32_t* bits,
+                               cudaStream_t s) {
   const int G = Hq / Hkv;
   const int groups = B * Hkv;
   const int nt = (Lc + dec::T - 1) / dec::T;
@@ -386,6 +390,8 @@ inline mala_status decode_bf16(const void* q, const void* Kc, const void* Vc, vo
   cp.thr = tau > 0.f ? log2f(tau) - log2f((float)Lc) : 0.f;
   cp.kept_tiles = kept_tiles;
   cp.keep_bits = bits;
+  cp.per_head = per_head;
+  cp.head_mask = w.head_mask;
   const size_t scan_smem = (size_t)G * nt * sizeof(float2);
   const int stage = scan_smem <= 200 * 1024;
   MALA_CUDA_TRY(cudaFuncSetAttribute(dec::scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -403,6 +409,7 @@ inline mala_status decode_bf16(const void* q, const void* Kc, const void* Vc, vo
   pp.nt = nt;
   pp.n_groups = groups;
   pp.scale_log2 = scale_log2;
+  pp.head_mask = per_head ? w.head_mask : nullptr;
   MALA_CUDA_TRY(cudaFuncSetAttribute(dec::pv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)dec::PV_SMEM));
   dec::pv_kernel<<<2 * nsm, dec::NT, dec::PV_SMEM, s>>>(mk, mv, pp);
@@ -532,10 +539,11 @@ size_t mala_decode_workspace_bytes(int B, int Hq, int Hkv, int Lc, int d) {
 }
 
 mala_status mala_decode(const void* q, const void* Kcache, const void* Vcache, void* o, int B,
-                        int Hq, int Hkv, int Lc, int d, float tau, float scale, void* workspace,
-                        size_t workspace_bytes, int32_t* kept_tiles, uint32_t* keep_bits,
-                        void* stream) {
+                        int Hq, int Hkv, int Lc, int d, float tau, float scale, int per_head,
+                        void* workspace, size_t workspace_bytes, int32_t* kept_tiles,
+                        uint32_t* keep_bits, void* stream) {
   if (B < 1 || Hq < 1 || Hkv < 1 || Lc < 1 || d < 1) return MALA_ERR_INVALID_ARG;
+  if (per_head != 0 && per_head != 1) return MALA_ERR_INVALID_ARG;
   if (!tau_ok(tau)) return MALA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return MALA_ERR_INVALID_ARG;
   if (d != 128 || Hq / Hkv > mala::dec::GMAX) return MALA_ERR_UNSUPPORTED;
@@ -547,8 +555,8 @@ mala_status mala_decode(const void* q, const void* Kcache, const void* Vcache, v
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MALA_ERR_INVALID_ARG;
   if (workspace_bytes < mala_decode_workspace_bytes(B, Hq, Hkv, Lc, d)) return MALA_ERR_INVALID_ARG;
   DecWorkspace w = dec_ws_carve(workspace, B, Hq, Hkv, Lc, d);
-  return decode_bf16(q, Kcache, Vcache, o, B, Hq, Hkv, Lc, resolve_scale(scale, d), tau, w,
-                     kept_tiles, keep_bits, as_stream(stream));
+  return decode_bf16(q, Kcache, Vcache, o, B, Hq, Hkv, Lc, resolve_scale(scale, d), tau, per_head,
+                     w, kept_tiles, keep_bits, as_stream(stream));
 }
 
 mala_status mala_check(void* stream) {

@@ -233,9 +233,84 @@ struct ScanParams {
   int G, nt, n_groups;
   float thr;       // log2(tau) - log2(Lc)
   int never_skip;
-  int32_t* kept_tiles;
-  uint32_t* keep_bits;  // [n_groups][nw]
+  int32_t* kept_tiles;   // [n_groups] (per_head: [n_groups][G])
+  uint32_t* keep_bits;   // [n_groups][nw] (per_head: [n_groups][G][nw])
+  // per_head: every query head decides alone (its own ratio test); the list
+  // holds the tiles any head kept, head_mask[list entry] which heads did
+  int per_head;
+  uint8_t* head_mask;    // [n_groups][nt]
 };
+
+// Per-head rows: head h keeps tile t iff  m_t,h - m_h - log2 l_h >= thr  with
+// its own running (m_h, l_h); the newest tile is every head's first. Warp 0
+// looks 32 tiles ahead: lane k tests tile next - k for every head; the first
+// tile some head wants is taken by exactly the heads that want it (no head's
+// state changed on the tiles before it, so their tests there stand).
+__device__ __forceinline__ void scan_per_head(const ScanParams& p, const float2* st, int grp) {
+  const int lane = threadIdx.x & 31;
+  const int G = p.G, nt = p.nt, nw = (nt + 31) >> 5;
+  float m[GMAX], l[GMAX];
+  int cnt[GMAX];
+  int count = 0;
+  int* kept = p.kept + (size_t)grp * nt;
+  uint8_t* mask = p.head_mask + (size_t)grp * nt;
+  uint32_t* bits = p.keep_bits ? p.keep_bits + (size_t)grp * G * nw : nullptr;
+  auto take = [&](int t, uint32_t hm) {
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+      if (h < G && ((hm >> h) & 1u)) {
+        const float2 s = st[h * nt + t];
+        if (cnt[h] == 0) {
+          m[h] = s.x;
+          l[h] = s.y;
+        } else {
+          const float mn = fmaxf(m[h], s.x);
+          l[h] = l[h] * exp2f(m[h] - mn) + s.y * exp2f(s.x - mn);
+          m[h] = mn;
+        }
+        ++cnt[h];
+        if (bits && lane == 0) bits[(size_t)h * nw + (t >> 5)] |= 1u << (t & 31);
+      }
+    }
+    if (lane == 0) {
+      kept[count] = t;
+      mask[count] = (uint8_t)hm;
+    }
+    ++count;
+  };
+#pragma unroll
+  for (int h = 0; h < GMAX; ++h) cnt[h] = 0;
+  take(nt - 1, (1u << G) - 1u);
+  int next = nt - 2;
+  while (next >= 0) {
+    const int tt = next - lane;
+    uint32_t want = 0;
+    if (tt >= 0) {
+#pragma unroll
+      for (int h = 0; h < GMAX; ++h)
+        if (h < G && (p.never_skip || (st[h * nt + tt].x - m[h] - __log2f(l[h])) >= p.thr))
+          want |= 1u << h;
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, want != 0u);
+    if (bal == 0u) {
+      next -= 32;
+      continue;
+    }
+    const int src = __ffs(bal) - 1;
+    const uint32_t hm = __shfl_sync(0xffffffffu, want, src);
+    take(next - src, hm);
+    __syncwarp();
+    next = next - src - 1;
+  }
+  if (lane == 0) p.counts[grp] = count;
+#pragma unroll
+  for (int h = 0; h < GMAX; ++h)
+    if (h < G && lane == h) {
+      p.mfin[(size_t)grp * G + h] = m[h];
+      p.lfin[(size_t)grp * G + h] = l[h];
+      if (p.kept_tiles) p.kept_tiles[(size_t)grp * G + h] = cnt[h];
+    }
+}
 
 // One CTA (128 threads) per group: stage the group's stats in shared memory
 // (when they fit; otherwise they are read from global memory), then warp 0
@@ -254,10 +329,15 @@ __global__ void __launch_bounds__(NT) scan_kernel(const ScanParams p, int stage_
   float* oz = p.oacc + (size_t)grp * G * D;
   for (int e = tid; e < G * D; e += NT) oz[e] = 0.f;
   const int nw = (nt + 31) >> 5;
+  const int nbits = p.per_head ? G * nw : nw;
   if (p.keep_bits)
-    for (int e = tid; e < nw; e += NT) p.keep_bits[(size_t)grp * nw + e] = 0u;
+    for (int e = tid; e < nbits; e += NT) p.keep_bits[(size_t)grp * nbits + e] = 0u;
   __syncthreads();
   if (tid >= 32) return;
+  if (p.per_head) {
+    scan_per_head(p, st, grp);
+    return;
+  }
 
   float m[GMAX], l[GMAX];
   int count = 0;
@@ -328,6 +408,7 @@ struct PVParams {
   float* oacc;
   int G, Lc, nt, n_groups;
   float scale_log2;
+  const uint8_t* head_mask;  // per-head rows: heads that kept each list entry (else null)
 };
 
 // Persistent CTAs over the flattened list of kept tiles of all groups.
@@ -372,6 +453,7 @@ __global__ void __launch_bounds__(NT) pv_kernel(const __grid_constant__ CUtensor
     }
     const int grp = lo;
     const int t = p.kept[(size_t)grp * p.nt + (item - prefix[grp])];
+    const uint32_t hm = p.head_mask ? p.head_mask[(size_t)grp * p.nt + (item - prefix[grp])] : 0xffu;
     if (tid == 0) {
       const uint32_t b = smem_u32(bar);
       mbar_expect_tx(b, 2 * TILE_BYTES);
@@ -398,7 +480,7 @@ __global__ void __launch_bounds__(NT) pv_kernel(const __grid_constant__ CUtensor
         const int kl = warp * 32 + mb * 16 + (lane >> 2) + (e >> 1) * 8;
         const int n = n0 + (e & 1);
         if (n < G) {
-          const bool valid = t * T + kl < p.Lc;
+          const bool valid = t * T + kl < p.Lc && ((hm >> n) & 1u);
           ps[n * T + kl] =
               valid ? exp2f(acc[mb][e] * p.scale_log2 - ((e & 1) ? mf1 : mf0)) : 0.f;
         }

@@ -59,6 +59,6 @@ extern "C" mala_status mala_decode_noalloc(const void* q, const void* Kcache, co
   // kernel zeroes the float32 output accumulator, the one region that must
   // start at zero.
   DecWorkspace w = dec_ws_carve(scratch, B, Hq, Hkv, Lc, d);
-  return decode_bf16(q, Kcache, Vcache, o, B, Hq, Hkv, Lc, resolve_scale(scale, d), tau, w,
+  return decode_bf16(q, Kcache, Vcache, o, B, Hq, Hkv, Lc, resolve_scale(scale, d), tau, 0, w,
                      kept_tiles, keep_bits, as_stream(stream));
 }

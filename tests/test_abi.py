@@ -78,13 +78,15 @@ def test_bwd_and_decode_argument_checks(lib):
     assert lib.mala_bwd(*args, need, 1, 2, 0, 128, 1, 1.0, 128, 0.0, None, None, None) == 0
     ws = lib.mala_decode_workspace_bytes(2, 8, 2, 1000, 128)
     assert ws > 0
-    dec = lambda Hq, Hkv, d, tau, nbytes: lib.mala_decode(v, v, v, v, 2, Hq, Hkv, 1000, d, tau,
-                                                          0.0, v, nbytes, None, None, None)
+    dec = lambda Hq, Hkv, d, tau, nbytes, ph=0: lib.mala_decode(v, v, v, v, 2, Hq, Hkv, 1000, d,
+                                                                tau, 0.0, ph, v, nbytes, None,
+                                                                None, None)
     assert dec(8, 3, 128, 1.0, ws) == 1    # Hq % Hkv
     assert dec(8, 2, 64, 1.0, ws) == 2     # d
     assert dec(32, 2, 128, 1.0, 1 << 30) == 2  # group of 16 heads > 8
     assert dec(8, 2, 128, -1.0, ws) == 1
     assert dec(8, 2, 128, 1.0, ws - 1) == 1
+    assert dec(8, 2, 128, 1.0, ws, ph=2) == 1   # per_head is 0 or 1
 
 
 def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):

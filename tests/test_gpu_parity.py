@@ -326,3 +326,30 @@ def test_empty_and_status():
     O, LSE = mala.mala_fwd(z, z, z)
     assert O.numel() == 0
     mala.mala_check()
+
+
+@pytest.mark.parametrize("Lc,tau", [(5000, 1.0), (20000, 1.0), (3000, 4.0), (1000, 0.0)])
+def test_decode_per_head_rows(Lc, tau):
+    """Per-head rows: every query head applies the test alone (oracle flag
+    per_head): keep sets per head, kept counts and outputs."""
+    cfg = synth.DecodeConfig("per_head", 7, 2, 8, 2, Lc, 128, 128, 0.98, max(1, Lc // 256), 4)
+    x = synth.decode_inputs(cfg)
+    q = dev_tensor(x["q"], torch.bfloat16)
+    Kc = dev_tensor(x["K"], torch.bfloat16)
+    Vc = dev_tensor(x["V"], torch.bfloat16)
+    o, kept, bits = mala.mala_decode(q, Kc, Vc, tau=tau, trace=True, per_head=True)
+    mala.mala_check()
+    nt = oracle.n_blocks(Lc, 128)
+    B, Hq = q.shape[0], q.shape[1]
+    gk = mala.unpack_bits(bits, nt)  # [B, Hq, nt]
+    fewer = 0
+    for b in range(B):
+        ref = oracle.decode(rounded(q[b]), rounded(Kc[b]), rounded(Vc[b]), tau=tau, per_head=True,
+                            want_margin=True)
+        for h in range(Hq):
+            if compare_decode_keep(gk[b, h], ref["keep"][h], ref["margin"][h]):
+                continue
+            assert kept[b, h].item() == int(ref["keep"][h].sum())
+            assert rel_l2(as_f64(o[b, h]), ref["o"][h]) <= TOL["bf16"]["decode"]
+            fewer += int(ref["keep"][h].sum())
+    assert fewer > 0

@@ -405,3 +405,19 @@ def test_tile_row_max_decides_the_backward_keep_set(tau):
             assert margin.max() == pytest.approx(g["margin"][i, j], abs=1e-9)
             skipped += int(g["keep"][i, j] == 0)
     assert skipped > 0
+
+
+@pytest.mark.parametrize("tau", [0.5, 1.0, 4.0])
+def test_omitted_mass_from_two_log_normalizers(tau):
+    """The mass a query row loses to skipped tiles equals 1 - exp(LSE_tau -
+    LSE_dense): LSE_tau normalizes over the kept keys only (the forward's
+    output), LSE_dense over all legal keys (tau = 0). Checked against the
+    per-tile enumeration of omitted_mass."""
+    L, d, T = 300, 8, 8
+    Q, K, V, _ = rand_inputs(L, d, 51, scale_qk=3.0)
+    f = oracle.fwd(Q, K, V, tile=T, tau=tau)
+    dense = oracle.fwd(Q, K, V, tile=T, tau=0.0)
+    mass = oracle.omitted_mass(Q, K, f["keep"], dense["LSE"], tile=T)
+    np.testing.assert_allclose(mass, 1.0 - np.exp(f["LSE"] - dense["LSE"]), atol=1e-12)
+    assert mass.max() > 0
+    assert mass.max() <= tau / (1 + tau) + 1e-12
