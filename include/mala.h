@@ -71,7 +71,10 @@ typedef enum { MALA_F32 = 0, MALA_BF16 = 1 } mala_dtype;
  * Sources: agihunt.info summary, forward paragraph; jaehun.me review,
  * "Forward: online sparse softmax".
  *
- * Inputs  Q, K, V: [B][H][L][d] of dtype dt.
+ * Inputs  Q: [B][H][L][d], K, V: [B][Hkv][L][d] of dtype dt. Grouped
+ *         query heads: query head h reads key/value head h / (H / Hkv);
+ *         Hkv = H is ordinary multi-head attention. Every query head applies
+ *         the rule to its own rows.
  * Outputs O: [B][H][L][d] of dtype dt, softmax over the retained tiles;
  *         LSE: [B][H][L] float32, natural-log normalizer m + ln l over the
  *         retained keys (with O, the only state backward needs);
@@ -97,13 +100,15 @@ typedef enum { MALA_F32 = 0, MALA_BF16 = 1 } mala_dtype;
  *         keep_bits: [B][H][nb][ceil(nb/32)], row = query block, bit = key
  *         block. nb = ceil(L / tile).
  * Supported: (dt, d, tile) in {(MALA_BF16, 128, 128), (MALA_F32, 32|64|128, 64)};
- *            any L >= 0 (a ragged last block is masked), B, H >= 1;
- *            with tile_rowmax, L <= 4194304 (else MALA_ERR_UNSUPPORTED).
+ *            any L >= 0 (a ragged last block is masked), B, H >= 1, H % Hkv
+ *            == 0 (Hkv < H: MALA_BF16 only); with tile_rowmax, L <= 4194304
+ *            (else MALA_ERR_UNSUPPORTED).
  */
 mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O,
                      float* LSE, float* O_f32, float* tile_rowmax, int B, int H,
-                     int L, int d, mala_dtype dt, float tau, int tile, float scale,
-                     int32_t* kept_tiles, uint32_t* keep_bits, void* stream);
+                     int Hkv, int L, int d, mala_dtype dt, float tau, int tile,
+                     float scale, int32_t* kept_tiles, uint32_t* keep_bits,
+                     void* stream);
 
 /* Bytes of the forward's optional tile_rowmax output: B * H * nb(nb+1)/2 *
  * tile * 4 (maxima) plus B * H * nb * ceil(nb/32) * 4 (flags), each rounded
@@ -133,12 +138,14 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
  * Sources: agihunt.info summary, backward paragraph; jaehun.me review,
  * "Backward: offline sparse probabilities".
  *
- * Inputs  Q, K, V, O, dO: [B][H][L][d] of dtype dt; LSE from mala_fwd;
+ * Inputs  Q, O, dO: [B][H][L][d], K, V: [B][Hkv][L][d] of dtype dt (grouped
+ *         heads as in mala_fwd); LSE from mala_fwd;
  *         O_f32 (may be NULL): the float32 output of mala_fwd, used for the
  *         row terms D instead of O when given;
  *         tile_rowmax (may be NULL; MALA_BF16 only): the forward's tile row
  *         maxima for the same Q, K (read only when tau > 0).
- * Outputs dQ, dK, dV: [B][H][L][d] of dtype dt (fully overwritten).
+ * Outputs dQ: [B][H][L][d]; dK, dV: [B][Hkv][L][d], summed over the query
+ *         heads of each group; dtype dt (fully overwritten).
  * workspace: device buffer of at least mala_bwd_workspace_bytes(B,H,L,d)
  *         bytes, 256-byte aligned, contents ignored on entry.
  * Trace   kept_tiles: [B][H][nb] kept query blocks per key block;
@@ -150,7 +157,7 @@ mala_status mala_bwd(const void* Q, const void* K, const void* V,
                      const void* O, const float* O_f32, const void* dO,
                      const float* LSE, const float* tile_rowmax, void* dQ,
                      void* dK, void* dV, void* workspace,
-                     size_t workspace_bytes, int B, int H, int L, int d,
+                     size_t workspace_bytes, int B, int H, int Hkv, int L, int d,
                      mala_dtype dt, float tau, int tile, float scale,
                      int32_t* kept_tiles, uint32_t* keep_bits, void* stream);
 

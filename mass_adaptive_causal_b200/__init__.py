@@ -49,14 +49,14 @@ def lib() -> ctypes.CDLL:
                 " (or __graft_entry__.build())")
         L = ctypes.CDLL(LIB_PATH)
         ci, cf, cs = ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-        L.mala_fwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _fp, _fp, ci, ci, ci, ci, ci, cf, ci, cf,
+        L.mala_fwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _fp, _fp, ci, ci, ci, ci, ci, ci, cf, ci, cf,
                                _i32p, _u32p, _vp]
         L.mala_tile_rowmax_bytes.argtypes = [ci, ci, ci, ci]
         L.mala_tile_rowmax_bytes.restype = cs
         L.mala_fwd.restype = ci
         L.mala_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
         L.mala_bwd_workspace_bytes.restype = cs
-        L.mala_bwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _fp, _fp, _vp, _vp, _vp, _vp, cs, ci,
+        L.mala_bwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _fp, _fp, _vp, _vp, _vp, _vp, cs, ci, ci,
                                ci, ci, ci, ci, cf, ci, cf, _i32p, _u32p, _vp]
         L.mala_bwd.restype = ci
         L.mala_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
@@ -101,16 +101,22 @@ def _dtype_code(t):
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def _check_prefill(*ts):
+def _check_prefill(q, k, v, *rest):
+    """q (and o, do in rest): [B, H, L, d]; k, v: [B, Hkv, L, d] with H % Hkv == 0
+    (grouped query heads; Hkv = H is multi-head attention)."""
     torch = _torch()
-    ref = ts[0]
-    for t in ts:
+    for t in (q, k, v) + rest:
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError("tensors must be contiguous CUDA tensors")
-        if t.shape != ref.shape or t.dtype != ref.dtype:
-            raise ValueError("Q, K, V (, O, dO) must share shape and dtype")
-    if ref.dim() != 4:
-        raise ValueError("expected [B, H, L, d]")
+        if t.dtype != q.dtype or t.dim() != 4:
+            raise ValueError("expected [B, H, L, d] tensors of one dtype")
+    if k.shape != v.shape or k.shape[0] != q.shape[0] or k.shape[2:] != q.shape[2:]:
+        raise ValueError("K and V must be [B, Hkv, L, d] matching Q's B, L, d")
+    if q.shape[1] % k.shape[1] != 0:
+        raise ValueError("the query heads must be a multiple of the key/value heads")
+    for t in rest:
+        if t.shape != q.shape:
+            raise ValueError("O and dO must have Q's shape")
     return torch
 
 
@@ -165,7 +171,7 @@ def mala_fwd(q, k, v, tau: float = 1.0, tile: int | None = None, scale: float = 
         kept = torch.empty((B, H, nb), dtype=torch.int32, device=q.device)
         bits = torch.empty((B, H, nb, (nb + 31) // 32), dtype=torch.int32, device=q.device)
     code = lib().mala_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), _ptr(o32_t),
-                          _ptr(rm_t), B, H, L, d, _dtype_code(q), float(tau), int(tile),
+                          _ptr(rm_t), B, H, k.shape[1], L, d, _dtype_code(q), float(tau), int(tile),
                           float(scale), _ptr(kept), _ptr(bits), _stream(stream))
     _raise(code, "mala_fwd")
     res = (o, lse_t, kept, bits) if trace else (o, lse_t)
@@ -205,7 +211,7 @@ def mala_bwd(q, k, v, o, do, lse, tau: float = 1.0, tile: int | None = None,
         raise ValueError("rowmax is smaller than tile_rowmax_bytes")
     code = lib().mala_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(o32), _ptr(do), _ptr(lse),
                           _ptr(rowmax), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), B, H,
-                          L, d, _dtype_code(q),
+                          k.shape[1], L, d, _dtype_code(q),
                           float(tau), int(tile), float(scale), _ptr(kept), _ptr(bits),
                           _stream(stream))
     _raise(code, "mala_bwd")

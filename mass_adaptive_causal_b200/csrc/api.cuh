@@ -124,12 +124,13 @@ inline mala_status fwd_f32(const float* Q, const float* K, const float* V, float
 }
 
 inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O, float* LSE,
-                            float* O32, float* rowmax, int Z, int L, float scale, float tau,
-                            int32_t* kept, uint32_t* bits, cudaStream_t s) {
+                            float* O32, float* rowmax, int B, int Hq, int Hkv, int L, float scale,
+                            float tau, int32_t* kept, uint32_t* bits, cudaStream_t s) {
+  const int Z = B * Hq, Zkv = B * Hkv;
   // Q and V in 128-row boxes; K in 64-row boxes (each CTA of a pair loads
   // half of every key tile)
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, L, Z) || !make_map(&mk, K, L, Z, 64) || !make_map(&mv, V, L, Z))
+  if (!make_map(&mq, Q, L, Z) || !make_map(&mk, K, L, Zkv, 64) || !make_map(&mv, V, L, Zkv))
     return MALA_ERR_CUDA;
   fwd2::Params p;
   p.O = reinterpret_cast<__nv_bfloat16*>(O);
@@ -145,6 +146,8 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
   p.keep_bits = bits;
   p.rowmax = rowmax;
   p.rm_bits = rowmax ? rowmax_flags(rowmax, Z, L, fwd2::T) : nullptr;
+  p.Hq = Hq;
+  p.G = Hq / Hkv;
   MALA_CUDA_TRY(cudaFuncSetAttribute(fwd2::fwd_pair_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)fwd2::SMEM_BYTES));
@@ -251,10 +254,12 @@ inline mala_status bwd_f32(const float* Q, const float* K, const float* V, const
 
 inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const void* dO,
                             const float* LSE, const float* rowmax, BwdWorkspace w, void* dQ,
-                            void* dK, void* dV, int Z, int L, float scale, float tau,
+                            void* dK, void* dV, int B, int Hq, int Hkv, int L, float scale,
+                            float tau,
                             int32_t* kept, uint32_t* bits, cudaStream_t s) {
   CUtensorMap mq, mk, mv, mdo;
-  if (!make_map(&mq, Q, L, Z) || !make_map(&mk, K, L, Z) || !make_map(&mv, V, L, Z) ||
+  const int Z = B * Hq, Zkv = B * Hkv;
+  if (!make_map(&mq, Q, L, Z) || !make_map(&mk, K, L, Zkv) || !make_map(&mv, V, L, Zkv) ||
       !make_map(&mdo, dO, L, Z))
     return MALA_ERR_CUDA;
   const int nb = (L + bwd100::T - 1) / bwd100::T;
@@ -267,6 +272,8 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
     tp.L = L;
     tp.nb = nb;
     tp.npairs = (nb + 1) / 2;
+    tp.Hq = Hq;
+    tp.G = Hq / Hkv;
     tp.scale_log2 = scale * kLog2e;
     tp.log2_tau = log2f(tau);
     tp.bits = tile_bits;
@@ -299,11 +306,15 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
   p.never_skip = never;
   p.kept_tiles = kept;
   p.bits = tile_bits;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
   MALA_CUDA_TRY(cudaFuncSetAttribute(bwd100::bwd_bf16_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)bwd100::SMEM_BYTES));
-  bwd100::bwd_bf16_kernel<<<dim3(p.nb, Z), bwd100::NT, bwd100::SMEM_BYTES, s>>>(mq, mk, mv, mdo,
-                                                                               p);
+  // one CTA per (key block, key/value head): dK_j, dV_j sum over its query heads
+  bwd100::bwd_bf16_kernel<<<dim3(p.nb, Zkv), bwd100::NT, bwd100::SMEM_BYTES, s>>>(mq, mk, mv,
+                                                                                 mdo, p);
   const size_t n4 = (size_t)Z * L * 128 / 4;
   aux::convert_bf16_v4_kernel<<<blocks_for(n4, 256, 4 * sm_count()), 256, 0, s>>>(
       reinterpret_cast<const float4*>(w.dQacc), reinterpret_cast<uint2*>(dQ), n4);
@@ -444,9 +455,11 @@ const char* mala_status_string(mala_status s) {
 
 int mala_version(void) { return 100; }
 
-static mala_status check_prefill_shape(int B, int H, int L, int d, mala_dtype dt, float tau,
-                                       int tile) {
-  if (B < 1 || H < 1 || L < 0 || d < 1) return MALA_ERR_INVALID_ARG;
+static mala_status check_prefill_shape(int B, int H, int Hkv, int L, int d, mala_dtype dt,
+                                       float tau, int tile) {
+  if (B < 1 || H < 1 || Hkv < 1 || L < 0 || d < 1) return MALA_ERR_INVALID_ARG;
+  if (H % Hkv != 0) return MALA_ERR_INVALID_ARG;
+  if (dt == MALA_F32 && Hkv != H) return MALA_ERR_UNSUPPORTED;  // grouped heads: bf16 only
   if ((long long)B * H > 65535) return MALA_ERR_INVALID_ARG;
   if (!tau_ok(tau)) return MALA_ERR_INVALID_ARG;
   if (dt == MALA_BF16) {
@@ -465,10 +478,10 @@ size_t mala_tile_rowmax_bytes(int B, int H, int L, int tile) {
 }
 
 mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE,
-                     float* O_f32, float* tile_rowmax, int B, int H, int L, int d, mala_dtype dt,
-                     float tau, int tile, float scale, int32_t* kept_tiles, uint32_t* keep_bits,
-                     void* stream) {
-  mala_status st = check_prefill_shape(B, H, L, d, dt, tau, tile);
+                     float* O_f32, float* tile_rowmax, int B, int H, int Hkv, int L, int d,
+                     mala_dtype dt, float tau, int tile, float scale, int32_t* kept_tiles,
+                     uint32_t* keep_bits, void* stream) {
+  mala_status st = check_prefill_shape(B, H, Hkv, L, d, dt, tau, tile);
   if (st != MALA_OK) return st;
   if (tile_rowmax && dt != MALA_BF16) return MALA_ERR_UNSUPPORTED;
   if (tile_rowmax && L > kMaxRowmaxL) return MALA_ERR_UNSUPPORTED;
@@ -489,7 +502,8 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
                                     cudaMemcpyDeviceToDevice, s));
     return st;
   }
-  return fwd_bf16(Q, K, V, O, LSE, O_f32, tile_rowmax, Z, L, sc, tau, kept_tiles, keep_bits, s);
+  return fwd_bf16(Q, K, V, O, LSE, O_f32, tile_rowmax, B, H, Hkv, L, sc, tau, kept_tiles,
+                  keep_bits, s);
 }
 
 size_t mala_bwd_workspace_bytes(int B, int H, int L, int d) {
@@ -500,10 +514,10 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d) {
 mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
                      const float* O_f32, const void* dO, const float* LSE,
                      const float* tile_rowmax, void* dQ, void* dK, void* dV, void* workspace,
-                     size_t workspace_bytes, int B, int H, int L, int d, mala_dtype dt, float tau,
-                     int tile, float scale, int32_t* kept_tiles, uint32_t* keep_bits,
+                     size_t workspace_bytes, int B, int H, int Hkv, int L, int d, mala_dtype dt,
+                     float tau, int tile, float scale, int32_t* kept_tiles, uint32_t* keep_bits,
                      void* stream) {
-  mala_status st = check_prefill_shape(B, H, L, d, dt, tau, tile);
+  mala_status st = check_prefill_shape(B, H, Hkv, L, d, dt, tau, tile);
   if (st != MALA_OK) return st;
   if (tile_rowmax && dt != MALA_BF16) return MALA_ERR_UNSUPPORTED;
   if (tile_rowmax && L > kMaxRowmaxL) return MALA_ERR_UNSUPPORTED;
@@ -529,8 +543,8 @@ mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
                    reinterpret_cast<const float*>(V), reinterpret_cast<const float*>(dO), LSE, w,
                    reinterpret_cast<float*>(dQ), reinterpret_cast<float*>(dK),
                    reinterpret_cast<float*>(dV), Z, L, d, sc, tau, kept_tiles, keep_bits, s);
-  return bwd_bf16(Q, K, V, dO, LSE, tile_rowmax, w, dQ, dK, dV, Z, L, sc, tau, kept_tiles,
-                  keep_bits, s);
+  return bwd_bf16(Q, K, V, dO, LSE, tile_rowmax, w, dQ, dK, dV, B, H, Hkv, L, sc, tau,
+                  kept_tiles, keep_bits, s);
 }
 
 size_t mala_decode_workspace_bytes(int B, int Hq, int Hkv, int Lc, int d) {

@@ -59,8 +59,9 @@ struct Params {
   float scale;       // softmax scale (dS is scaled before the bf16 cast)
   float scale_log2;  // scale * log2(e)
   int never_skip;    // tau == 0: every legal tile is kept (no bits read)
-  int32_t* kept_tiles;
-  const uint32_t* bits;  // [Z][nb][nw] from the test pass
+  int32_t* kept_tiles;   // [B * Hq][nb]
+  const uint32_t* bits;  // [B * Hq][nb][nw] from the test pass
+  int Hq, Hkv, G;        // query heads, key/value heads, G = Hq / Hkv
 };
 
 // Row of a TMEM accumulator (this thread's lane) -> bf16 global row. Every
@@ -108,8 +109,10 @@ __global__ void __launch_bounds__(NT, 1)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
-  const int j = blockIdx.x;  // key block 0 has the most query blocks: first
-  const int z = blockIdx.y;
+  const int j = blockIdx.x;   // key block 0 has the most query blocks: first
+  const int zkv = blockIdx.y;  // (b, key/value head): K_j, V_j, dK_j, dV_j
+  // dK_j and dV_j sum over the G query heads that share this key/value head
+  const int zq0 = (zkv / p.Hkv) * p.Hq + (zkv % p.Hkv) * p.G;
   const uint32_t bar_kv = smem_u32(&bars[0]);
   const uint32_t bar_q = smem_u32(&bars[1]);
   const uint32_t bar_mma = smem_u32(&bars[3]);
@@ -138,10 +141,10 @@ __global__ void __launch_bounds__(NT, 1)
 
   if (tid == 0) {
     mbar_expect_tx(bar_kv, 2 * TILE_BYTES);
-    tma_load_3d(ka, &tmK, 0, j * T, z, bar_kv);
-    tma_load_3d(ka + HALF_BYTES, &tmK, 64, j * T, z, bar_kv);
-    tma_load_3d(va, &tmV, 0, j * T, z, bar_kv);
-    tma_load_3d(va + HALF_BYTES, &tmV, 64, j * T, z, bar_kv);
+    tma_load_3d(ka, &tmK, 0, j * T, zkv, bar_kv);
+    tma_load_3d(ka + HALF_BYTES, &tmK, 64, j * T, zkv, bar_kv);
+    tma_load_3d(va, &tmV, 0, j * T, zkv, bar_kv);
+    tma_load_3d(va + HALF_BYTES, &tmV, 64, j * T, zkv, bar_kv);
   }
   uint32_t ph_q = 0, ph_mma = 0;
   int kept_count = 0;
@@ -149,6 +152,9 @@ __global__ void __launch_bounds__(NT, 1)
   const int nw = (p.nb + 31) >> 5;
   const int lane = tid & 31;
 
+  for (int hg = 0; hg < p.G && ok; ++hg) {
+  const int z = zq0 + hg;  // query head: Q_i, dO_i, LSE, D, dQ, the keep bits
+  const int kept_before = kept_count;
   for (int i0 = j; i0 < p.nb && ok; i0 += LIST_CHUNK) {
     // ---- list the kept query blocks i in [i0, i0 + LIST_CHUNK), ascending
     int n_list = 0;
@@ -328,13 +334,15 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     }
   }
+  if (tid == 0 && p.kept_tiles) p.kept_tiles[(size_t)z * p.nb + j] = kept_count - kept_before;
+  }
 
   // ---- epilogue: dK_j, dV_j (bf16); zero if no tile was kept ----------------
   // (TMEM loads are warp-collective: all lanes load, valid key rows store)
   const int key = j * T + tid;
   if (ok) {
-    __nv_bfloat16* dk = p.dK + ((size_t)z * p.L + (key < p.L ? key : 0)) * D;
-    __nv_bfloat16* dv = p.dV + ((size_t)z * p.L + (key < p.L ? key : 0)) * D;
+    __nv_bfloat16* dk = p.dK + ((size_t)zkv * p.L + (key < p.L ? key : 0)) * D;
+    __nv_bfloat16* dv = p.dV + ((size_t)zkv * p.L + (key < p.L ? key : 0)) * D;
     if (kept_count > 0) {
       tc_fence_after();
       store_row_bf16(dk, t_dk, key < p.L);
@@ -348,7 +356,6 @@ __global__ void __launch_bounds__(NT, 1)
       }
     }
   }
-  if (tid == 0 && p.kept_tiles) p.kept_tiles[(size_t)z * p.nb + j] = kept_count;
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

@@ -52,6 +52,7 @@ struct Params {
   float scale_log2;
   float log2_tau;
   uint32_t* bits;  // [Z][nb][nw]: bit j of row i set iff tile (i, j) is kept
+  int Hq, G;       // query heads; G query heads share each key/value head
 };
 
 struct Bars {
@@ -130,8 +131,9 @@ __global__ void __launch_bounds__(NT, 1)
         const uint32_t kb = smem_u32(&bars.k_full[s]);
         const uint32_t dst = sbase + OFF_K + s * TILE_BYTES;
         mbar_expect_tx(kb, TILE_BYTES);
-        tma_load_3d(dst, &tmK, 0, (jtop - t) * T, z, kb);
-        tma_load_3d(dst + HALF_BYTES, &tmK, 64, (jtop - t) * T, z, kb);
+        const int zkv = (z / p.Hq) * (p.Hq / p.G) + (z % p.Hq) / p.G;
+        tma_load_3d(dst, &tmK, 0, (jtop - t) * T, zkv, kb);
+        tma_load_3d(dst + HALF_BYTES, &tmK, 64, (jtop - t) * T, zkv, kb);
       }
     }
     __syncwarp();

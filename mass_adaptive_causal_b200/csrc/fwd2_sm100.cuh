@@ -96,6 +96,7 @@ struct Params {
   // only kept tiles and tiles skipped by less are stored.
   float* rowmax;
   uint32_t* rm_bits;
+  int Hq, G;  // query heads; G query heads share each key/value head
 };
 
 struct Bars {
@@ -150,7 +151,8 @@ __global__ void __launch_bounds__(NT, 1)
   const bool leader = rank == 0;
 
   const int c = p.npairs - 1 - (int)(blockIdx.x >> 1);  // longest pairs first
-  const int z = blockIdx.y;
+  const int z = blockIdx.y;  // (b, query head)
+  const int zkv = (z / p.Hq) * (p.Hq / p.G) + (z % p.Hq) / p.G;  // its key/value head
   const int i0 = 2 * c, i1 = 2 * c + 1;
   const bool hasB = i1 < p.nb;
   const bool mine = leader || hasB;  // this CTA has a query block
@@ -213,8 +215,8 @@ __global__ void __launch_bounds__(NT, 1)
         if (leader) mbar_expect_tx(smem_u32(&bars.k_full[s]), 2 * KH_BYTES);
         const int row = (jtop - t) * T + 64 * (int)rank;
         const uint32_t dst = sbase + OFF_K + s * KH_BYTES;
-        tma_load_3d_pair(dst, &tmK, 0, row, z, lead(&bars.k_full[s]));
-        tma_load_3d_pair(dst + KH_BLK, &tmK, 64, row, z, lead(&bars.k_full[s]));
+        tma_load_3d_pair(dst, &tmK, 0, row, zkv, lead(&bars.k_full[s]));
+        tma_load_3d_pair(dst + KH_BLK, &tmK, 64, row, zkv, lead(&bars.k_full[s]));
       }
     }
     __syncwarp();
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (n >= NSV && !mbar_wait(smem_u32(&bars.v_empty[vs]), ((n / NSV) - 1) & 1, abort, 0x213))
           break;
         if (leader) mbar_expect_tx(smem_u32(&bars.v_full[vs]), 2 * VH_BYTES);
-        tma_load_3d_pair(sbase + OFF_V + vs * VH_BYTES, &tmV, 64 * (int)rank, j * T, z,
+        tma_load_3d_pair(sbase + OFF_V + vs * VH_BYTES, &tmV, 64 * (int)rank, j * T, zkv,
                          lead(&bars.v_full[vs]));
       }
     }

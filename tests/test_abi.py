@@ -40,9 +40,11 @@ def test_status_strings(lib):
     assert lib.mala_version() >= 100
 
 
-def _fwd(lib, ptrs=(16, 16, 16, 16, 16, 0, 0), B=1, H=1, L=256, d=128, dt=1, tau=1.0, tile=128):
+def _fwd(lib, ptrs=(16, 16, 16, 16, 16, 0, 0), B=1, H=1, L=256, d=128, dt=1, tau=1.0, tile=128,
+         Hkv=None):
     p = [ctypes.c_void_p(x) if x else None for x in ptrs]
-    return lib.mala_fwd(*p, B, H, L, d, dt, tau, tile, 0.0, None, None, None)
+    return lib.mala_fwd(*p, B, H, H if Hkv is None else Hkv, L, d, dt, tau, tile, 0.0, None, None,
+                        None)
 
 
 def test_fwd_argument_checks(lib):
@@ -64,6 +66,10 @@ def test_fwd_argument_checks(lib):
     assert _fwd(lib, ptrs=(16, 16, 16, 16, 16, 0, 16), L=(1 << 22) + 1) == 2  # L limit
     assert _fwd(lib, L=0) == 0                   # empty input: nothing to do
     assert _fwd(lib, B=300, H=300) == 1          # grid limit
+    assert _fwd(lib, H=4, Hkv=3) == 1            # query heads not a multiple of kv heads
+    assert _fwd(lib, H=4, Hkv=0) == 1
+    assert _fwd(lib, H=4, Hkv=2, dt=0, d=64, tile=64) == 2  # grouped heads: bf16 only
+    assert _fwd(lib, H=4, Hkv=2, L=0) == 0
 
 
 def test_bwd_and_decode_argument_checks(lib):
@@ -73,9 +79,10 @@ def test_bwd_and_decode_argument_checks(lib):
     nb64 = (1000 + 63) // 64
     assert need == r256(2 * 1000 * 4) + r256(2 * 1000 * 128 * 4) + r256(2 * nb64 * ((nb64 + 31) // 32) * 4)
     args = [v] * 7 + [None] + [v] * 4
-    assert lib.mala_bwd(*args, need - 1, 1, 2, 1000, 128, 1, 1.0, 128, 0.0, None, None, None) == 1
-    assert lib.mala_bwd(*args, need, 1, 2, 1000, 128, 1, -0.5, 128, 0.0, None, None, None) == 1
-    assert lib.mala_bwd(*args, need, 1, 2, 0, 128, 1, 1.0, 128, 0.0, None, None, None) == 0
+    assert lib.mala_bwd(*args, need - 1, 1, 2, 2, 1000, 128, 1, 1.0, 128, 0.0, None, None, None) == 1
+    assert lib.mala_bwd(*args, need, 1, 2, 2, 1000, 128, 1, -0.5, 128, 0.0, None, None, None) == 1
+    assert lib.mala_bwd(*args, need, 1, 2, 2, 0, 128, 1, 1.0, 128, 0.0, None, None, None) == 0
+    assert lib.mala_bwd(*args, need, 1, 2, 3, 1000, 128, 1, 1.0, 128, 0.0, None, None, None) == 1
     ws = lib.mala_decode_workspace_bytes(2, 8, 2, 1000, 128)
     assert ws > 0
     dec = lambda Hq, Hkv, d, tau, nbytes, ph=0: lib.mala_decode(v, v, v, v, 2, Hq, Hkv, 1000, d,

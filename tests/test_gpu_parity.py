@@ -353,3 +353,56 @@ def test_decode_per_head_rows(Lc, tau):
             assert rel_l2(as_f64(o[b, h]), ref["o"][h]) <= TOL["bf16"]["decode"]
             fewer += int(ref["keep"][h].sum())
     assert fewer > 0
+
+
+def gqa_case(L):
+    """Two key/value heads of the matched_8k recipe, four query heads: query
+    heads 0, 1 read kv head 0, heads 2, 3 read kv head 1 (each a copy of that
+    head's own queries, the second one perturbed)."""
+    cfg = synth.CONFIGS["matched_8k"]
+    x = synth.prefill_inputs(cfg, L=L, heads=[0, 1])
+    rng = np.random.default_rng(L + 17)
+    Q = np.concatenate([x["Q"][:, :1], x["Q"][:, :1] + 0.3 * rng.standard_normal(x["Q"][:, :1].shape),
+                        x["Q"][:, 1:2], 0.9 * x["Q"][:, 1:2]], axis=1)
+    dO = rng.standard_normal(Q.shape)
+    t = {"Q": dev_tensor(Q, torch.bfloat16), "dO": dev_tensor(dO, torch.bfloat16),
+         "K": dev_tensor(x["K"][:, :2], torch.bfloat16), "V": dev_tensor(x["V"][:, :2], torch.bfloat16)}
+    return t
+
+
+@pytest.mark.parametrize("L,tau,use_rowmax", [(1000, 1.0, True), (1536, 0.25, False), (640, 0.0, False)])
+def test_bf16_grouped_query_heads(L, tau, use_rowmax):
+    """Grouped query heads (Hq = 4, Hkv = 2): per query head the rule on the
+    shared K, V; dK, dV of a kv head are the sums over its query heads."""
+    t = gqa_case(L)
+    O, LSE, kept, bits, *rest = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True,
+                                              o32=True, rowmax=use_rowmax)
+    O32 = rest[0]
+    rm = rest[1] if use_rowmax else None
+    dQ, dK, dV, kept_b, bits_b = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
+                                               trace=True, o32=O32, rowmax=rm)
+    mala.mala_check()
+    nb = oracle.n_blocks(L, 128)
+    Kd, Vd = [rounded(t["K"][0, g]) for g in range(2)], [rounded(t["V"][0, g]) for g in range(2)]
+    refK, refV = [np.zeros_like(Kd[0]), np.zeros_like(Kd[0])], [np.zeros_like(Vd[0]), np.zeros_like(Vd[0])]
+    clean = True
+    for h in range(4):
+        g = h // 2
+        Qd, dOd = rounded(t["Q"][0, h]), rounded(t["dO"][0, h])
+        _, n_near, ref = check_fwd_slice(Qd, Kd[g], Vd[g], as_f64(O[0, h]), as_f64(LSE[0, h]),
+                                         bits[0, h], 128, tau, TOL["bf16"])
+        gk = mala.unpack_bits(bits[0, h], nb)
+        _, bad = compare_fwd_keep(gk, ref["keep"], ref["margin"])
+        gr = oracle.bwd(Qd, Kd[g], Vd[g], ref["O"], dOd, ref["LSE"], tile=128, tau=tau,
+                        want_margin=True)
+        compare_bwd_keep(mala.unpack_bits(bits_b[0, h], nb), gr["keep"], gr["margin"],
+                         skip_blocks=bad)
+        clean = clean and not bad
+        if not bad:
+            assert rel_l2(as_f64(dQ[0, h]), gr["dQ"]) <= TOL["bf16"]["grad"]
+        refK[g] += gr["dK"]
+        refV[g] += gr["dV"]
+    if clean:
+        for g in range(2):
+            assert rel_l2(as_f64(dK[0, g]), refK[g]) <= TOL["bf16"]["grad"]
+            assert rel_l2(as_f64(dV[0, g]), refV[g]) <= TOL["bf16"]["grad"]

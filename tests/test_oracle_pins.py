@@ -421,3 +421,36 @@ def test_omitted_mass_from_two_log_normalizers(tau):
     np.testing.assert_allclose(mass, 1.0 - np.exp(f["LSE"] - dense["LSE"]), atol=1e-12)
     assert mass.max() > 0
     assert mass.max() <= tau / (1 + tau) + 1e-12
+
+
+def test_grouped_heads_backward_sums_over_the_group():
+    """Grouped query heads (several query heads read one key/value head): the
+    forward is the per-head rule on the shared K, V, and dK, dV of the shared
+    head are the sums of the per-head gradients. At tau = 0 this is checked
+    against torch autograd through K, V repeated for every query head (the
+    repeat's backward does the summing)."""
+    rng = np.random.default_rng(61)
+    G, L, d, T = 3, 40, 8, 8
+    K, V = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    Qs = [rng.standard_normal((L, d)) * 1.3 for _ in range(G)]
+    dOs = [rng.standard_normal((L, d)) for _ in range(G)]
+    dK, dV = np.zeros((L, d)), np.zeros((L, d))
+    outs = []
+    for Q, dO in zip(Qs, dOs):
+        f = oracle.fwd(Q, K, V, tile=T, tau=0.0)
+        g = oracle.bwd(Q, K, V, f["O"], dO, f["LSE"], tile=T, tau=0.0)
+        dK += g["dK"]
+        dV += g["dV"]
+        outs.append((f["O"], g["dQ"]))
+    q = torch.tensor(np.stack(Qs), requires_grad=True)
+    k = torch.tensor(K, requires_grad=True)
+    v = torch.tensor(V, requires_grad=True)
+    o = torch.nn.functional.scaled_dot_product_attention(
+        q[None], k[None, None].expand(1, G, L, d), v[None, None].expand(1, G, L, d),
+        is_causal=True)[0]
+    o.backward(torch.tensor(np.stack(dOs)))
+    for h, (O, dQ) in enumerate(outs):
+        np.testing.assert_allclose(O, o[h].detach().numpy(), atol=1e-10)
+        np.testing.assert_allclose(dQ, q.grad[h].numpy(), atol=1e-9)
+    np.testing.assert_allclose(dK, k.grad.numpy(), atol=1e-9)
+    np.testing.assert_allclose(dV, v.grad.numpy(), atol=1e-9)
