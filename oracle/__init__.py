@@ -58,6 +58,8 @@ def _load():
             lib.mala_oracle_decode.argtypes = [_dp, _dp, _dp, c_int, c_int, c_int, c_int, c_int,
                                                c_double, c_double, c_int, _dp, _u8p, _dp]
             lib.mala_oracle_dense_fwd.argtypes = [_dp, _dp, _dp, c_int, c_int, c_double, _dp, _dp]
+            lib.mala_oracle_fwd_chunk.argtypes = [_dp, _dp, _dp, c_int, c_int, c_int, c_int,
+                                                  c_double, c_double, _dp, _dp, _u8p, _dp]
             lib.mala_oracle_dense_bwd.argtypes = [_dp, _dp, _dp, _dp, c_int, c_int, c_double,
                                                   _dp, _dp, _dp]
             lib.mala_oracle_omitted_mass.argtypes = [_dp, _dp, c_int, c_int, c_int, c_double,
@@ -105,6 +107,31 @@ def fwd(Q, K, V, tile, tau=1.0, scale=None, force_first=True, qblocks=None,
                             int(force_first), _p(O), _p(LSE), _p(keep, _u8p),
                             _p(margin), int(lo), int(hi))
     out = {"O": O, "LSE": LSE, "keep": keep}
+    if want_margin:
+        out["margin"] = margin
+    return out
+
+
+def fwd_chunk(Q, K, V, tile, tau=1.0, scale=None, want_margin=False):
+    """MALA forward of a prefill chunk appended to a KV cache: Q (Lq, d) are
+    the last Lq positions of a sequence whose keys/values K, V are (Lk, d).
+    Query row r sits at position Lk - Lq + r. Key tiles are aligned to the
+    chunk's query blocks (tile k starts at position off + tile (k - koff),
+    koff = ceil(off / tile)); keep / margin are (nbq, nbq + koff)."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    Lq, d = Q.shape
+    Lk = K.shape[0]
+    assert Lk >= Lq
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    nbq = n_blocks(Lq, tile)
+    koff = n_blocks(Lk - Lq, tile)
+    O = np.full((Lq, d), np.nan)
+    LSE = np.full(Lq, np.nan)
+    keep = np.zeros((nbq, nbq + koff), np.uint8)
+    margin = np.full((nbq, nbq + koff), np.nan) if want_margin else None
+    _load().mala_oracle_fwd_chunk(_p(Q), _p(K), _p(V), Lq, Lk, d, tile, scale, float(tau),
+                                  _p(O), _p(LSE), _p(keep, _u8p), _p(margin))
+    out = {"O": O, "LSE": LSE, "keep": keep, "koff": koff}
     if want_margin:
         out["margin"] = margin
     return out

@@ -166,6 +166,93 @@ int mala_oracle_fwd(const double *Q, const double *K, const double *V, int L,
   return 0;
 }
 
+/*
+ * Forward of a prefill chunk appended to a KV cache (one (batch, head)
+ * slice): Lq new queries after Lk - Lq cached keys, so query row r sits at
+ * position off + r (off = Lk - Lq) and its legal keys are 0 .. off + r, with
+ * Lq,r = off + r + 1 in the threshold ([R1], [R3]). Query blocks are the
+ * chunk's own 128-row blocks; key tiles are aligned to them: key tile k
+ * covers positions off + T (k - koff) .. + T - 1, koff = ceil(off / T), so
+ * query block i's diagonal tile is k = i + koff and tile 0 may start below
+ * position 0 (those keys do not exist). Traversal k = i + koff down to 0
+ * ([R2]); the diagonal tile is always kept.
+ * Q: [Lq][d]; K, V: [Lk][d]. O: [Lq][d], LSE: [Lq].
+ * keep, margin (may be NULL): [nbq][nbq + koff], entry (i, k).
+ */
+int mala_oracle_fwd_chunk(const double *Q, const double *K, const double *V, int Lq,
+                          int Lk, int d, int T, double scale, double tau, double *O,
+                          double *LSE, uint8_t *keep, double *margin) {
+  if (Lq <= 0) return 0;
+  const int off = Lk - Lq;
+  const int nbq = (Lq + T - 1) / T, koff = (off + T - 1) / T, nkt = nbq + koff;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int i = nbq - 1; i >= 0; --i) {
+    const int r0 = i * T, R = imin(Lq, (i + 1) * T) - r0;
+    double *m = malloc(sizeof(double) * R);
+    double *l = malloc(sizeof(double) * R);
+    double *mt = malloc(sizeof(double) * R);
+    double *acc = calloc((size_t)R * d, sizeof(double));
+    double *s = malloc(sizeof(double) * (size_t)R * T);
+    for (int r = 0; r < R; ++r) { m[r] = NEG_INF; l[r] = 0.0; }
+    for (int k = i + koff; k >= 0; --k) {
+      const int p0 = off + T * (k - koff); /* position of the tile's first key */
+      for (int r = 0; r < R; ++r) {
+        const int pos = off + r0 + r;
+        double mx = NEG_INF;
+        for (int c = 0; c < T; ++c) {
+          const int kp = p0 + c;
+          double v = NEG_INF;
+          if (kp >= 0 && kp <= pos) v = scale * dot(Q + (size_t)(r0 + r) * d, K + (size_t)kp * d, d);
+          s[(size_t)r * T + c] = v;
+          if (v > mx) mx = v;
+        }
+        mt[r] = mx;
+      }
+      int kept;
+      double mu = NEG_INF;
+      if (k == i + koff || tau <= 0.0) {
+        kept = 1;
+        mu = INFINITY;
+      } else {
+        kept = 0;
+        for (int r = 0; r < R; ++r) {
+          const double lhs = mt[r] - m[r] - log(l[r]);
+          const double crit = lhs - log_threshold(tau, (double)(off + r0 + r + 1));
+          if (crit > mu) mu = crit;
+          if (crit >= 0.0) kept = 1;
+        }
+      }
+      if (keep) keep[(size_t)i * nkt + k] = (uint8_t)kept;
+      if (margin) margin[(size_t)i * nkt + k] = mu;
+      if (!kept) continue;
+      for (int r = 0; r < R; ++r) {
+        if (mt[r] == NEG_INF) continue; /* no legal key of this row in the tile */
+        const double mnew = mt[r] > m[r] ? mt[r] : m[r];
+        const double alpha = (m[r] == NEG_INF) ? 0.0 : exp(m[r] - mnew);
+        double *a = acc + (size_t)r * d;
+        for (int e = 0; e < d; ++e) a[e] *= alpha;
+        double lsum = l[r] * alpha;
+        for (int c = 0; c < T; ++c) {
+          const double sv = s[(size_t)r * T + c];
+          if (sv == NEG_INF) continue;
+          const double pr = exp(sv - mnew);
+          lsum += pr;
+          const double *vc = V + (size_t)(p0 + c) * d;
+          for (int e = 0; e < d; ++e) a[e] += pr * vc[e];
+        }
+        l[r] = lsum;
+        m[r] = mnew;
+      }
+    }
+    for (int r = 0; r < R; ++r) {
+      for (int e = 0; e < d; ++e) O[(size_t)(r0 + r) * d + e] = acc[(size_t)r * d + e] / l[r];
+      LSE[r0 + r] = m[r] + log(l[r]);
+    }
+    free(m); free(l); free(mt); free(acc); free(s);
+  }
+  return 0;
+}
+
 /* Backward tile test ([R3]): keep iff some valid row has
  * max_c s_rc - LSE_r >= ln tau - ln Lq. Returns the keep flag; *mu gets the
  * max over rows of that difference. s must hold the tile's scores. */

@@ -454,3 +454,48 @@ def test_grouped_heads_backward_sums_over_the_group():
         np.testing.assert_allclose(dQ, q.grad[h].numpy(), atol=1e-9)
     np.testing.assert_allclose(dK, k.grad.numpy(), atol=1e-9)
     np.testing.assert_allclose(dV, v.grad.numpy(), atol=1e-9)
+
+
+@pytest.mark.parametrize("off", [0, 16, 24, 5])
+def test_chunk_forward_dense_is_bottom_right_causal_softmax(off):
+    """tau = 0: a chunk of Lq queries after `off` cached keys is softmax
+    attention where query r sees keys 0 .. off + r (library: torch SDPA with
+    that mask, float64)."""
+    rng = np.random.default_rng(71 + off)
+    Lq, d, T = 37, 8, 8
+    Lk = Lq + off
+    Q, K, V = (rng.standard_normal((n, d)) for n in (Lq, Lk, Lk))
+    f = oracle.fwd_chunk(Q, K, V, tile=T, tau=0.0)
+    mask = np.arange(Lk)[None, :] <= (off + np.arange(Lq))[:, None]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(Q)[None, None], torch.tensor(K)[None, None], torch.tensor(V)[None, None],
+        attn_mask=torch.tensor(mask)[None, None])[0, 0].numpy()
+    np.testing.assert_allclose(f["O"], ref, atol=1e-12)
+
+
+@pytest.mark.parametrize("tau", [0.5, 1.0, 4.0])
+def test_chunk_forward_equals_full_prefill_rows(tau):
+    """A chunk whose cache length is a multiple of the tile sees exactly the
+    tiles and running state of the full prefill's last blocks, so it
+    reproduces their outputs, log-normalizers and keep sets."""
+    L, d, T = 160, 8, 16
+    Q, K, V, _ = rand_inputs(L, d, 73, scale_qk=2.5)
+    for off in (0, 48, 96):
+        full = oracle.fwd(Q, K, V, tile=T, tau=tau)
+        ch = oracle.fwd_chunk(Q[off:], K, V, tile=T, tau=tau)
+        np.testing.assert_allclose(ch["O"], full["O"][off:], atol=1e-12)
+        np.testing.assert_allclose(ch["LSE"], full["LSE"][off:], atol=1e-12)
+        b0 = off // T
+        assert np.array_equal(ch["keep"], full["keep"][b0:, :])
+
+
+def test_chunk_forward_keeps_the_mass_bound():
+    """Any cache offset: the mass a row loses stays below tau / (1 + tau)."""
+    rng = np.random.default_rng(79)
+    Lq, d, T, off, tau = 70, 8, 8, 29, 1.0
+    Q, K, V = (rng.standard_normal((n, d)) * 2.5 for n in (Lq, Lq + off, Lq + off))
+    f = oracle.fwd_chunk(Q, K, V, tile=T, tau=tau)
+    dense = oracle.fwd_chunk(Q, K, V, tile=T, tau=0.0)
+    lost = 1.0 - np.exp(f["LSE"] - dense["LSE"])
+    assert lost.max() > 0 and lost.max() <= tau / (1 + tau)
+    assert f["keep"].sum() < dense["keep"].sum()
