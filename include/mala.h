@@ -110,6 +110,46 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O,
                      float scale, int32_t* kept_tiles, uint32_t* keep_bits,
                      void* stream);
 
+/*
+ * Prefill of chunks appended to KV caches, several sequences packed
+ * (SURVEY's next row "varlen prefill": prefill uses the same tau;
+ * agihunt.info summary, "one tau for prefill and decode").
+ *
+ * Sequence b's new queries are tokens [cu_seqlens_q[b], cu_seqlens_q[b+1])
+ * of Q; its keys and values, cached ones first, are tokens
+ * [cu_seqlens_k[b], cu_seqlens_k[b+1]) of K and V, with Lk_b >= Lq_b. Query
+ * r of the chunk sits at position off_b + r (off_b = Lk_b - Lq_b), sees keys
+ * 0 .. off_b + r and has Lq = off_b + r + 1 in the threshold. Query blocks
+ * are the chunk's own 128-row blocks; key tiles are aligned to them (tile k
+ * starts at position off_b + 128 (k - koff_b), koff_b = ceil(off_b / 128),
+ * positions below 0 do not exist), so a chunk whose cache is a whole number
+ * of tiles reproduces the full prefill's rows exactly. Each block visits its
+ * diagonal tile (always kept) and then the earlier tiles, with the rule of
+ * mala_fwd.
+ *
+ * Inputs  Q: [total_q][H][d] bf16; K, V: [total_k][Hkv][d] bf16 (query head
+ *         h reads key/value head h / (H / Hkv)); cu_seqlens_q,
+ *         cu_seqlens_k: device int32 [batch + 1], non-decreasing from 0.
+ *         max_seqlen_q >= every Lq_b (blocks past it are not computed),
+ *         max_seqlen_k >= every Lk_b (trace layout). A sequence with
+ *         Lk_b < Lq_b is left untouched.
+ * Outputs O: [total_q][H][d] bf16; LSE: [H][total_q] float32.
+ * Trace   kept_tiles: [batch][H][nbq] with nbq = ceil(max_seqlen_q / 128);
+ *         keep_bits: [batch][H][nbq][mala_varlen_trace_words(...)], bit k of
+ *         a row = key tile k kept.
+ * Supported: d = 128, tile = 128, H % Hkv == 0, batch * H <= 65535.
+ */
+mala_status mala_fwd_varlen(const void* Q, const void* K, const void* V, void* O,
+                            float* LSE, const int32_t* cu_seqlens_q,
+                            const int32_t* cu_seqlens_k, int batch,
+                            int max_seqlen_q, int max_seqlen_k, int total_q,
+                            int total_k, int H, int Hkv, int d, float tau,
+                            int tile, float scale, int32_t* kept_tiles,
+                            uint32_t* keep_bits, void* stream);
+
+/* 32-bit words per query block in mala_fwd_varlen's keep_bits. */
+int mala_varlen_trace_words(int max_seqlen_q, int max_seqlen_k);
+
 /* Bytes of the forward's optional tile_rowmax output: B * H * nb(nb+1)/2 *
  * tile * 4 (maxima) plus B * H * nb * ceil(nb/32) * 4 (flags), each rounded
  * up to 256, for nb = ceil(L / tile): 2 GiB for B = 1, H = 8, L = 131072,

@@ -18,7 +18,8 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["mala_fwd", "mala_bwd", "mala_decode", "mala_decode_noalloc", "mala_check", "MalaError", "lib",
+__all__ = ["mala_fwd", "mala_fwd_varlen", "mala_bwd", "mala_decode", "mala_decode_noalloc", "mala_check",
+           "MalaError", "lib",
            "LIB_PATH", "MALA_F32", "MALA_BF16", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -51,6 +52,11 @@ def lib() -> ctypes.CDLL:
         ci, cf, cs = ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         L.mala_fwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _fp, _fp, ci, ci, ci, ci, ci, ci, cf, ci, cf,
                                _i32p, _u32p, _vp]
+        L.mala_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _vp, ci, ci, ci, ci, ci, ci,
+                                      ci, ci, cf, ci, cf, _i32p, _u32p, _vp]
+        L.mala_fwd_varlen.restype = ci
+        L.mala_varlen_trace_words.argtypes = [ci, ci]
+        L.mala_varlen_trace_words.restype = ci
         L.mala_tile_rowmax_bytes.argtypes = [ci, ci, ci, ci]
         L.mala_tile_rowmax_bytes.restype = cs
         L.mala_fwd.restype = ci
@@ -178,6 +184,40 @@ def mala_fwd(q, k, v, tau: float = 1.0, tile: int | None = None, scale: float = 
     if o32_t is not None:
         res = res + (o32_t,)
     return res + (rm_t,) if rm_t is not None else res
+
+
+def mala_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                    tau: float = 1.0, scale: float = 0.0, trace: bool = False, out=None,
+                    lse=None, stream=None):
+    """Prefill of chunks appended to KV caches, sequences packed.
+    q: [total_q, H, d] bf16; k, v: [total_k, Hkv, d] bf16; cu_seqlens_*:
+    int32 CUDA tensors [batch + 1]. Returns (O [total_q, H, d], LSE [H,
+    total_q]) or, with ``trace=True``, also kept_tiles [batch, H, nbq] and
+    keep_bits [batch, H, nbq, nw] (bit k = key tile k)."""
+    torch = _torch()
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16 or t.dim() != 3:
+            raise ValueError("q, k, v must be contiguous [tokens, heads, d] bf16 CUDA tensors")
+    for t in (cu_seqlens_q, cu_seqlens_k):
+        if not t.is_cuda or t.dtype != torch.int32 or not t.is_contiguous():
+            raise ValueError("cu_seqlens must be contiguous int32 CUDA tensors")
+    total_q, H, d = q.shape
+    total_k, Hkv, _ = k.shape
+    batch = cu_seqlens_q.numel() - 1
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((H, total_q), dtype=torch.float32, device=q.device) if lse is None else lse
+    kept = bits = None
+    if trace:
+        nbq = n_blocks(max_seqlen_q, 128)
+        nw = int(lib().mala_varlen_trace_words(max_seqlen_q, max_seqlen_k))
+        kept = torch.zeros((batch, H, nbq), dtype=torch.int32, device=q.device)
+        bits = torch.zeros((batch, H, nbq, nw), dtype=torch.int32, device=q.device)
+    code = lib().mala_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t),
+                                 _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), batch, int(max_seqlen_q),
+                                 int(max_seqlen_k), total_q, total_k, H, Hkv, d, float(tau), 128,
+                                 float(scale), _ptr(kept), _ptr(bits), _stream(stream))
+    _raise(code, "mala_fwd_varlen")
+    return (o, lse_t, kept, bits) if trace else (o, lse_t)
 
 
 def bwd_workspace_bytes(B, H, L, d) -> int:

@@ -89,6 +89,24 @@ inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t Z
   return r == CUDA_SUCCESS;
 }
 
+// Packed bf16 tensor [tokens][heads][128] seen as 3-D (x = d, y = token,
+// z = head), box 64 x box_rows x 1, 128-byte swizzle; tokens outside
+// [0, tokens) read as zero.
+inline bool make_map_packed(CUtensorMap* m, const void* base, uint64_t tokens, uint64_t heads,
+                            uint32_t box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, tokens, heads};
+  cuuint64_t strides[2] = {heads * 128 * 2, 128 * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  memset(m, 0, sizeof(*m));
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 inline int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -123,6 +141,16 @@ inline mala_status fwd_f32(const float* Q, const float* K, const float* V, float
   return launch_status();
 }
 
+template <bool VARLEN>
+inline mala_status launch_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                               const fwd2::Params& p, int npairs, int Z, cudaStream_t s);
+
+// Trace words per query block of a chunk: key tiles k < nbq + ceil(off / 128).
+inline int varlen_trace_words(int max_q, int max_k) {
+  const int nkt = (max_q + 127) / 128 + (max_k + 127) / 128;
+  return (nkt + 31) / 32;
+}
+
 inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O, float* LSE,
                             float* O32, float* rowmax, int B, int Hq, int Hkv, int L, float scale,
                             float tau, int32_t* kept, uint32_t* bits, cudaStream_t s) {
@@ -148,11 +176,17 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
   p.rm_bits = rowmax ? rowmax_flags(rowmax, Z, L, fwd2::T) : nullptr;
   p.Hq = Hq;
   p.G = Hq / Hkv;
-  MALA_CUDA_TRY(cudaFuncSetAttribute(fwd2::fwd_pair_kernel,
+  return launch_pair<false>(mq, mk, mv, p, p.npairs, Z, s);
+}
+
+template <bool VARLEN>
+inline mala_status launch_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                               const fwd2::Params& p, int npairs, int Z, cudaStream_t s) {
+  MALA_CUDA_TRY(cudaFuncSetAttribute(fwd2::fwd_pair_kernel<VARLEN>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)fwd2::SMEM_BYTES));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * p.npairs, Z, 1);
+  cfg.gridDim = dim3(2 * npairs, Z, 1);
   cfg.blockDim = dim3(fwd2::NT, 1, 1);
   cfg.dynamicSmemBytes = fwd2::SMEM_BYTES;
   cfg.stream = s;
@@ -163,8 +197,37 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  MALA_CUDA_TRY(cudaLaunchKernelEx(&cfg, fwd2::fwd_pair_kernel, mq, mk, mv, p));
+  MALA_CUDA_TRY(cudaLaunchKernelEx(&cfg, fwd2::fwd_pair_kernel<VARLEN>, mq, mk, mv, p));
   return launch_status();
+}
+
+// Chunks appended to KV caches, packed tokens (see mala_fwd_varlen).
+inline mala_status fwd_varlen_bf16(const void* Q, const void* K, const void* V, void* O,
+                                   float* LSE, const int32_t* cu_q, const int32_t* cu_k,
+                                   int batch, int max_q, int max_k, int total_q, int total_k,
+                                   int Hq, int Hkv, float scale, float tau, int32_t* kept,
+                                   uint32_t* bits, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map_packed(&mq, Q, total_q, Hq, 128) || !make_map_packed(&mk, K, total_k, Hkv, 64) ||
+      !make_map_packed(&mv, V, total_k, Hkv, 128))
+    return MALA_ERR_CUDA;
+  fwd2::Params p;
+  memset(&p, 0, sizeof(p));
+  p.O = reinterpret_cast<__nv_bfloat16*>(O);
+  p.LSE = LSE;
+  p.scale_log2 = scale * kLog2e;
+  p.never_skip = tau == 0.f;
+  p.log2_tau = tau > 0.f ? log2f(tau) : 0.f;
+  p.kept_tiles = kept;
+  p.keep_bits = bits;
+  p.Hq = Hq;
+  p.G = Hq / Hkv;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.total_q = total_q;
+  p.nbq_max = (max_q + fwd2::T - 1) / fwd2::T;
+  p.nw = varlen_trace_words(max_q, max_k);
+  return launch_pair<true>(mq, mk, mv, p, (p.nbq_max + 1) / 2, batch * Hq, s);
 }
 
 // ---------------------------------------------------------------- backward
@@ -504,6 +567,34 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
   }
   return fwd_bf16(Q, K, V, O, LSE, O_f32, tile_rowmax, B, H, Hkv, L, sc, tau, kept_tiles,
                   keep_bits, s);
+}
+
+mala_status mala_fwd_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                            int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int H,
+                            int Hkv, int d, float tau, int tile, float scale,
+                            int32_t* kept_tiles, uint32_t* keep_bits, void* stream) {
+  if (batch < 1 || H < 1 || Hkv < 1 || d < 1 || total_q < 0 || total_k < 0 ||
+      max_seqlen_q < 0 || max_seqlen_k < 0)
+    return MALA_ERR_INVALID_ARG;
+  if (H % Hkv != 0 || !tau_ok(tau)) return MALA_ERR_INVALID_ARG;
+  if (d != 128 || tile != 128) return MALA_ERR_UNSUPPORTED;
+  if ((long long)batch * H > 65535) return MALA_ERR_INVALID_ARG;
+  if (total_q == 0 || max_seqlen_q == 0) return MALA_OK;
+  if (!Q || !K || !V || !O || !LSE || !cu_seqlens_q || !cu_seqlens_k) return MALA_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, K, V, O, LSE};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MALA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return MALA_ERR_INVALID_ARG;
+  return fwd_varlen_bf16(Q, K, V, O, LSE, cu_seqlens_q, cu_seqlens_k, batch, max_seqlen_q,
+                         max_seqlen_k, total_q, total_k, H, Hkv, resolve_scale(scale, d), tau,
+                         kept_tiles, keep_bits, as_stream(stream));
+}
+
+int mala_varlen_trace_words(int max_seqlen_q, int max_seqlen_k) {
+  if (max_seqlen_q < 0 || max_seqlen_k < 0) return 0;
+  return varlen_trace_words(max_seqlen_q, max_seqlen_k);
 }
 
 size_t mala_bwd_workspace_bytes(int B, int H, int L, int d) {

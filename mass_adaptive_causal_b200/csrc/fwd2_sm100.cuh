@@ -97,6 +97,17 @@ struct Params {
   float* rowmax;
   uint32_t* rm_bits;
   int Hq, G;  // query heads; G query heads share each key/value head
+  // Chunks appended to a KV cache, packed (the VARLEN instantiation):
+  // sequence b's queries are tokens [cu_q[b], cu_q[b+1]) of Q [total_q][Hq][d],
+  // its keys / values tokens [cu_k[b], cu_k[b+1]) of K, V [total_k][Hkv][d];
+  // its query r sits at position off + r, off = Lk - Lq. Key tiles are
+  // aligned to the chunk's query blocks: tile k starts at position
+  // off + T (k - koff), koff = ceil(off / T); positions below 0 are masked.
+  const int* cu_q;
+  const int* cu_k;
+  int total_q;
+  int nbq_max;  // trace rows per (b, h)
+  int nw;       // trace words per row
 };
 
 struct Bars {
@@ -135,6 +146,7 @@ __device__ __forceinline__ int vote_or(int pred) {
 }
 __device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+template <bool VARLEN>
 __global__ void __launch_bounds__(NT, 1)
     fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -150,17 +162,45 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
 
-  const int c = p.npairs - 1 - (int)(blockIdx.x >> 1);  // longest pairs first
   const int z = blockIdx.y;  // (b, query head)
-  const int zkv = (z / p.Hq) * (p.Hq / p.G) + (z % p.Hq) / p.G;  // its key/value head
+  // this (b, head)'s sequence: query rows, cache offset, TMA coordinates
+  int Lq, off, zq, zkv, yq0, yk0;
+  if (VARLEN) {
+    const int b = z / p.Hq, h = z % p.Hq;
+    yq0 = p.cu_q[b];
+    yk0 = p.cu_k[b];
+    Lq = p.cu_q[b + 1] - yq0;
+    off = (p.cu_k[b + 1] - yk0) - Lq;
+    zq = h;
+    zkv = h / p.G;
+  } else {
+    Lq = p.L;
+    off = 0;
+    zq = z;
+    zkv = (z / p.Hq) * (p.Hq / p.G) + (z % p.Hq) / p.G;  // its key/value head
+    yq0 = yk0 = 0;
+  }
+  const int nb = (Lq + T - 1) / T;
+  const int npairs = (nb + 1) / 2;
+  const int koff = (off + T - 1) / T;
+  // a cluster beyond this sequence's pairs, or of a sequence with fewer
+  // keys than queries (not a cache append), has nothing to do: both CTAs
+  // leave together, before any barrier
+  if ((int)(blockIdx.x >> 1) >= npairs || off < 0) return;
+  // a sequence longer than the stated maxima would overrun the trace rows
+  if (VARLEN && (nb > p.nbq_max || nb + koff > 32 * p.nw)) return;
+  const int c = npairs - 1 - (int)(blockIdx.x >> 1);  // longest pairs first
   const int i0 = 2 * c, i1 = 2 * c + 1;
-  const bool hasB = i1 < p.nb;
+  const bool hasB = i1 < nb;
   const bool mine = leader || hasB;  // this CTA has a query block
   const int iX = i0 + (int)rank;
-  const int jtop = hasB ? i1 : i0;
-  const int ntiles = jtop + 1;  // tile t <-> key block jtop - t
-  // the CTA's block takes part in tile t iff its query block >= key block
-  auto part = [&](int t) { return mine && jtop - t <= iX; };
+  const int ktop = (hasB ? i1 : i0) + koff;
+  const int ntiles = ktop + 1;  // tile t <-> key tile ktop - t
+  // first key position of key tile k (below 0 for the oldest tile of a
+  // chunk whose cache is not a whole number of tiles)
+  auto kpos = [&](int k) { return off + T * (k - koff); };
+  // the CTA's block takes part in tile t iff the tile is not past its diagonal
+  auto part = [&](int t) { return mine && ktop - t <= iX + koff; };
   // PVs whose V the producers load without a request: the diagonal tiles,
   // always kept (t = 0 for rank 1's block, t = 1 for rank 0's), or every
   // tile when nothing is skipped.
@@ -206,14 +246,14 @@ __global__ void __launch_bounds__(NT, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       if (leader) mbar_expect_tx(smem_u32(&bars.q_full), 2 * Q_BYTES);
-      tma_load_3d_pair(sbase + OFF_Q, &tmQ, 0, iX * T, z, lead(&bars.q_full));
-      tma_load_3d_pair(sbase + OFF_Q + QH_BYTES, &tmQ, 64, iX * T, z, lead(&bars.q_full));
+      tma_load_3d_pair(sbase + OFF_Q, &tmQ, 0, yq0 + iX * T, zq, lead(&bars.q_full));
+      tma_load_3d_pair(sbase + OFF_Q + QH_BYTES, &tmQ, 64, yq0 + iX * T, zq, lead(&bars.q_full));
       for (int t = 0; t < ntiles; ++t) {
         const int s = t % NSK;
         if (t >= NSK && !mbar_wait(smem_u32(&bars.k_empty[s]), ((t / NSK) - 1) & 1, abort, 0x211))
           break;
         if (leader) mbar_expect_tx(smem_u32(&bars.k_full[s]), 2 * KH_BYTES);
-        const int row = (jtop - t) * T + 64 * (int)rank;
+        const int row = yk0 + kpos(ktop - t) + 64 * (int)rank;
         const uint32_t dst = sbase + OFF_K + s * KH_BYTES;
         tma_load_3d_pair(dst, &tmK, 0, row, zkv, lead(&bars.k_full[s]));
         tma_load_3d_pair(dst + KH_BLK, &tmK, 64, row, zkv, lead(&bars.k_full[s]));
@@ -228,7 +268,7 @@ __global__ void __launch_bounds__(NT, 1)
         const int vs = n % NSV;
         int j;
         if (n < npre) {
-          j = jtop - n;  // PV n is tile n
+          j = ktop - n;  // PV n is tile n
         } else {
           if (!mbar_wait_cluster(smem_u32(&bars.v_req[vs]), ((n - npre) / NSV) & 1, abort, 0x212))
             break;
@@ -238,7 +278,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (n >= NSV && !mbar_wait(smem_u32(&bars.v_empty[vs]), ((n / NSV) - 1) & 1, abort, 0x213))
           break;
         if (leader) mbar_expect_tx(smem_u32(&bars.v_full[vs]), 2 * VH_BYTES);
-        tma_load_3d_pair(sbase + OFF_V + vs * VH_BYTES, &tmV, 64 * (int)rank, j * T, zkv,
+        tma_load_3d_pair(sbase + OFF_V + vs * VH_BYTES, &tmV, 64 * (int)rank, yk0 + kpos(j), zkv,
                          lead(&bars.v_full[vs]));
       }
     }
@@ -309,7 +349,7 @@ __global__ void __launch_bounds__(NT, 1)
           const int vs = vcount % NSV;
           if (vcount >= npre) {  // ask both V producers for tile t
             for (uint32_t r = 0; r < 2; ++r) {
-              st_cluster_u32(mapa_rank(smem_u32(&bars.req_j[vs]), r), (uint32_t)(jtop - t));
+              st_cluster_u32(mapa_rank(smem_u32(&bars.req_j[vs]), r), (uint32_t)(ktop - t));
               mbar_arrive_cluster(mapa_rank(smem_u32(&bars.v_req[vs]), r));
             }
           }
@@ -351,9 +391,11 @@ __global__ void __launch_bounds__(NT, 1)
   } else {
     // ----------------------------------------------------- softmax / test (4 warps)
     const int r = tid;  // 0..127
-    const int row = iX * T + r;
-    const bool row_valid = mine && row < p.L;
-    const float thr = p.never_skip ? 0.f : (p.log2_tau - __log2f((float)(row + 1)));
+    const int row = iX * T + r;  // row of the chunk; position off + row
+    // (packed chunks: a row past the packed tensor is never written, whatever
+    // the offsets say)
+    const bool row_valid = mine && row < Lq && (!VARLEN || yq0 + row < p.total_q);
+    const float thr = p.never_skip ? 0.f : (p.log2_tau - __log2f((float)(off + row + 1)));
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const uint32_t t_o = tmem + lane_base + TMEM_O;
     auto signal = [&](int u, int keep) {  // thread 0: this CTA's decision for slot u
@@ -374,19 +416,22 @@ __global__ void __launch_bounds__(NT, 1)
     // score bound, refreshed whenever (m_ref, l) change
     float bound_raw = kNegInf;
     int n_kept = 0;
-    const int nw = (p.nb + 31) >> 5;
+    // trace row of this block: bit k of word k / 32 = key tile k kept
+    const int nw = VARLEN ? p.nw : (nb + 31) >> 5;
+    const size_t brow = (size_t)z * (VARLEN ? p.nbq_max : nb) + iX;
     KeepBits kb, kbs;
-    kb.init(r == 0 && mine ? p.keep_bits : nullptr, ((size_t)z * p.nb + iX) * nw);
-    kbs.init(r == 0 && mine ? p.rm_bits : nullptr, ((size_t)z * p.nb + iX) * nw);
+    kb.init(r == 0 && mine ? p.keep_bits : nullptr, brow * nw);
+    kbs.init(r == 0 && mine && !VARLEN ? p.rm_bits : nullptr, brow * nw);
     if (r == 0 && mine) {
-      for (int w = iX / 32 + 1; w < nw; ++w) {
-        if (p.keep_bits) p.keep_bits[((size_t)z * p.nb + iX) * nw + w] = 0u;
-        if (p.rm_bits) p.rm_bits[((size_t)z * p.nb + iX) * nw + w] = 0u;
+      for (int w = (iX + koff) / 32 + 1; w < nw; ++w) {
+        if (p.keep_bits) p.keep_bits[brow * nw + w] = 0u;
+        if (p.rm_bits && !VARLEN) p.rm_bits[brow * nw + w] = 0u;
       }
     }
-    float* rm = (p.rowmax && mine) ? p.rowmax + ((size_t)z * ((size_t)p.nb * (p.nb + 1) / 2) +
-                                                 (size_t)iX * (iX + 1) / 2) * T + r
-                                   : nullptr;
+    float* rm = (p.rowmax && mine && !VARLEN)
+                    ? p.rowmax + ((size_t)z * ((size_t)nb * (nb + 1) / 2) +
+                                  (size_t)iX * (iX + 1) / 2) * T + r
+                    : nullptr;
     softmax_sync();  // O zeroed by every thread before any decision leaves
 
     for (int t = 0; t < ntiles; ++t) {
@@ -399,11 +444,13 @@ __global__ void __launch_bounds__(NT, 1)
         if (r == 0) signal(u, 0);
         continue;
       }
-      const int j = jtop - t;
-      const bool diag = (j == iX);
+      const int j = ktop - t;  // key tile
+      const bool diag = (j == iX + koff);
+      const int lo = VARLEN ? max(0, -kpos(j)) : 0;  // columns below lo: no key
       const uint32_t t_s = tmem + lane_base + u * 128;
       // ---- row max of the tile (raw scores: the positive scale commutes)
-      const float mraw = tmem_rowmax128(t_s, diag, r);
+      const float mraw = (VARLEN && lo > 0) ? tmem_rowmax128_from(t_s, lo)
+                                            : tmem_rowmax128(t_s, diag, r);
       const float mt = mraw * p.scale_log2;
       int want = diag || p.never_skip;
       if (!want && row_valid) want = mraw >= bound_raw;
@@ -458,8 +505,11 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int col = ch * 32 + e;
-          const float p0 = (diag && col > r) ? 0.f : exp2f(sv[e] * p.scale_log2 - m_ref);
-          const float p1 = (diag && col + 1 > r) ? 0.f : exp2f(sv[e + 1] * p.scale_log2 - m_ref);
+          const float p0 = ((diag && col > r) || col < lo) ? 0.f
+                                                           : exp2f(sv[e] * p.scale_log2 - m_ref);
+          const float p1 = ((diag && col + 1 > r) || col + 1 < lo)
+                               ? 0.f
+                               : exp2f(sv[e + 1] * p.scale_log2 - m_ref);
           lsum += p0 + p1;
           const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
           const float2 hf = __bfloat1622float2(h);
@@ -486,7 +536,8 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_wait(smem_u32(&bars.pv_done), (n_kept - 1) & 1, abort, 0x21b);
       tc_fence_after();
       const float inv = 1.f / l;
-      const size_t orow = ((size_t)z * p.L + (row_valid ? row : 0)) * D;
+      const size_t orow = VARLEN ? ((size_t)(yq0 + (row_valid ? row : 0)) * p.Hq + zq) * D
+                                 : ((size_t)z * p.L + (row_valid ? row : 0)) * D;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         float o[32];
@@ -511,8 +562,11 @@ __global__ void __launch_bounds__(NT, 1)
           }
         }
       }
-      if (row_valid) p.LSE[(size_t)z * p.L + row] = (m_ref + __log2f(l)) * kLn2;
-      if (r == 0 && p.kept_tiles) p.kept_tiles[(size_t)z * p.nb + iX] = n_kept;
+      if (row_valid) {
+        const size_t li = VARLEN ? (size_t)zq * p.total_q + yq0 + row : (size_t)z * p.L + row;
+        p.LSE[li] = (m_ref + __log2f(l)) * kLn2;
+      }
+      if (r == 0 && p.kept_tiles) p.kept_tiles[brow] = n_kept;
     }
   }
   // both CTAs finish every access to the other's shared memory and TMEM

@@ -411,6 +411,23 @@ __device__ __forceinline__ float tmem_rowmax128(uint32_t taddr, bool diag, int r
   return fmaxf(fmaxf(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5])), fmaxf(a[6], a[7]));
 }
 
+// Row max over TMEM columns lo .. 127 of this thread's lane (the columns
+// below lo are keys that do not exist).
+__device__ __forceinline__ float tmem_rowmax128_from(uint32_t taddr, int lo) {
+  uint32_t v[128];
+  tmem_ld128(taddr, v);
+  const float ninf = -__builtin_huge_valf();
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = ninf;
+#pragma unroll
+  for (int e = 0; e < 128; e += 8) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], e + k < lo ? ninf : __uint_as_float(v[e + k]));
+  }
+  return fmaxf(fmaxf(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5])), fmaxf(a[6], a[7]));
+}
+
 // Row max over 64 TMEM columns of this thread's lane (columns col0 .. col0+63
 // of the tile). With `diag`, tile columns c > r are excluded.
 __device__ __forceinline__ float tmem_rowmax64(uint32_t taddr, bool diag, int r, int col0) {

@@ -128,3 +128,20 @@ def test_tile_rowmax_bytes(lib):
         8 * 1024 * 1025 // 2 * 512 + 8 * 1024 * 32 * 4
     assert lib.mala_tile_rowmax_bytes(0, 1, 10, 128) == 0
     assert lib.mala_tile_rowmax_bytes(1, 1, 0, 128) == 0
+
+
+def test_fwd_varlen_argument_checks(lib):
+    v = ctypes.c_void_p(256)
+    f = lambda batch=2, mq=100, mk=200, tq=150, tk=300, H=2, Hkv=1, d=128, tau=1.0, tile=128: \
+        lib.mala_fwd_varlen(v, v, v, v, v, v, v, batch, mq, mk, tq, tk, H, Hkv, d, tau, tile, 0.0,
+                            None, None, None)
+    assert f(batch=0) == 1
+    assert f(H=3, Hkv=2) == 1
+    assert f(tau=-1.0) == 1
+    assert f(d=64) == 2
+    assert f(tile=64) == 2
+    assert f(tq=0) == 0
+    assert lib.mala_fwd_varlen(None, v, v, v, v, v, v, 2, 100, 200, 150, 300, 2, 1, 128, 1.0, 128,
+                               0.0, None, None, None) == 1
+    assert lib.mala_varlen_trace_words(100, 200) == 1
+    assert lib.mala_varlen_trace_words(4096, 131072) == (32 + 1024 + 31) // 32

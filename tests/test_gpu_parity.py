@@ -406,3 +406,54 @@ def test_bf16_grouped_query_heads(L, tau, use_rowmax):
         for g in range(2):
             assert rel_l2(as_f64(dK[0, g]), refK[g]) <= TOL["bf16"]["grad"]
             assert rel_l2(as_f64(dV[0, g]), refV[g]) <= TOL["bf16"]["grad"]
+
+
+@pytest.mark.parametrize("tau", [1.0, 0.25])
+def test_bf16_varlen_cache_append(tau):
+    """Three packed sequences with (new queries, all keys) = (300, 300),
+    (200, 500) (a cache of 300 keys: not a whole number of tiles) and
+    (384, 640), two query heads on one key/value head: every (sequence,
+    head) against the oracle's chunk forward (outputs, LSE, keep sets)."""
+    lens = [(300, 300), (200, 500), (384, 640)]
+    H, Hkv, d = 2, 1, 128
+    rng = np.random.default_rng(91)
+    cfg = synth.CONFIGS["matched_8k"]
+    qs, ks, vs = [], [], []
+    for s_i, (lq, lk) in enumerate(lens):
+        x = synth.prefill_inputs(cfg, L=lk, heads=[s_i])
+        K, V, Qall = x["K"][0, 0], x["V"][0, 0], x["Q"][0, 0]
+        Qh = [Qall[lk - lq:], Qall[lk - lq:] * 0.8 + 0.2 * rng.standard_normal((lq, d))]
+        qs.append(np.stack(Qh, axis=1))          # [lq, H, d]
+        ks.append(K[:, None, :])
+        vs.append(V[:, None, :])
+    q = dev_tensor(np.concatenate(qs), torch.bfloat16)
+    k = dev_tensor(np.concatenate(ks), torch.bfloat16)
+    v = dev_tensor(np.concatenate(vs), torch.bfloat16)
+    cq = torch.tensor(np.cumsum([0] + [a for a, _ in lens]), dtype=torch.int32).cuda()
+    ck = torch.tensor(np.cumsum([0] + [b for _, b in lens]), dtype=torch.int32).cuda()
+    mq, mk = max(a for a, _ in lens), max(b for _, b in lens)
+    O, LSE, kept, bits = mala.mala_fwd_varlen(q, k, v, cq, ck, mq, mk, tau=tau, trace=True)
+    mala.mala_check()
+    cqh, ckh = cq.cpu().numpy(), ck.cpu().numpy()
+    for b, (lq, lk) in enumerate(lens):
+        Kd = rounded(k[ckh[b]:ckh[b + 1], 0])
+        Vd = rounded(v[ckh[b]:ckh[b + 1], 0])
+        for h in range(H):
+            Qd = rounded(q[cqh[b]:cqh[b + 1], h])
+            ref = oracle.fwd_chunk(Qd, Kd, Vd, tile=128, tau=tau, want_margin=True)
+            nbq, nkt = ref["keep"].shape
+            gk = mala.unpack_bits(bits[b, h], nkt)[:nbq]
+            bad = []
+            for i in range(nbq):
+                diff = np.nonzero(gk[i] != ref["keep"][i])[0]
+                if len(diff):
+                    assert all(abs(ref["margin"][i, kk]) <= np.log1p(1e-3) for kk in diff), (b, h, i)
+                    bad.append(i)
+            rows = np.ones(lq, bool)
+            for i in bad:  # a near-threshold flip changes that block's later tiles
+                rows[i * 128:(i + 1) * 128] = False
+            o = as_f64(O[cqh[b]:cqh[b + 1], h])
+            assert rel_l2(o[rows], ref["O"][rows]) <= TOL["bf16"]["O"]
+            assert rel_l2(as_f64(LSE[h, cqh[b]:cqh[b + 1]])[rows], ref["LSE"][rows]) <= TOL["bf16"]["LSE"]
+            if not bad:
+                assert np.array_equal(kept[b, h, :nbq].cpu().numpy(), ref["keep"].sum(axis=1))
