@@ -12,7 +12,6 @@
 #include "bwd_test_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "fwd2_sm100.cuh"
-#include "fwd_sm100.cuh"
 #include "mala.h"
 #include "simt_f32.cuh"
 

@@ -22,17 +22,32 @@
 // Warps 0-3 test A, warps 4-7 test B, warp 8 loads, warp 9 issues the MMAs.
 #pragma once
 
-#include "fwd_sm100.cuh"
+#include "sm100.cuh"
 
 namespace mala {
 namespace bwdtest {
 
 using namespace sm100;
-using fwd100::D;
-using fwd100::HALF_BYTES;
-using fwd100::IDESC_QK;
-using fwd100::T;
-using fwd100::TILE_BYTES;
+
+constexpr int T = 128;
+constexpr int D = 128;
+constexpr uint32_t TILE_BYTES = T * D * 2;   // 32 KB
+constexpr uint32_t HALF_BYTES = T * 64 * 2;  // one 64-column swizzled block
+constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, false, false);
+
+// OR-vote over one 128-thread warpgroup on named barrier `id`.
+__device__ __forceinline__ int wg_vote_or(int pred, int id) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "barrier.cta.red.or.pred po, %2, 128, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(out)
+      : "r"(pred), "r"(id)
+      : "memory");
+  return (int)out;
+}
 
 constexpr int NT = 320;
 constexpr int WARP_PRODUCER = 8;
@@ -207,7 +222,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
           for (int e = 0; e < 64; ++e) mraw = fmaxf(mraw, 64 + e > r ? kNegInf : sb[e]);
         }
-        const int keep = fwd100::wg_vote_or(mraw >= craw, bar_id);
+        const int keep = wg_vote_or(mraw >= craw, bar_id);
         kb.set(j, keep != 0);
       }
       kb.flush();
