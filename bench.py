@@ -229,6 +229,18 @@ def load_profile_traffic():
     return {}
 
 
+def reduce_max(v: float, world: int, device) -> float:
+    """The largest of every rank's value (a device time: the job is as slow as
+    its slowest replica); the process group's backend decides the device."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
@@ -284,12 +296,7 @@ def run_mala(args, rank, world, local_rank):
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        import torch.distributed as dist
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, world, dev)
 
     def timed(tau, steps, warmup, rowmax=True):
         for _ in range(warmup):
