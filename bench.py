@@ -139,7 +139,11 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        # the raw samples go to MALA_BENCH_OUT (default: the system's temp
+        # directory); the JSON line carries their summary
+        import tempfile
+        out = os.environ.get("MALA_BENCH_OUT", tempfile.gettempdir())
+        self.path = os.path.join(out, f"clocks_gpu{gpu_index}.csv")
 
     def start(self):
         try:
