@@ -34,12 +34,14 @@ using namespace sm100;
 
 constexpr int T = 128;
 constexpr int D = 128;
-constexpr int NT = 128;
+constexpr int NT = 256;
+constexpr int NWARP = NT / 32;
 constexpr uint32_t TILE_BYTES = T * D * 2;
 constexpr uint32_t HALF_BYTES = T * 64 * 2;
 constexpr int LIST_CHUNK = 1024;  // query blocks listed per round
-constexpr uint32_t SMEM_BYTES = 6 * TILE_BYTES + 1024 /*align*/ + 2048 /*LSE, D*/ + 256 +
-                                LIST_CHUNK * 4 + 64;
+constexpr int LIST_ROUNDS = LIST_CHUNK / NT;
+constexpr uint32_t SMEM_BYTES = 6 * TILE_BYTES + 1024 /*align*/ + 2048 /*LSE, D*/ + 64 /*bars*/ +
+                                LIST_CHUNK * 4 + LIST_ROUNDS * NWARP * 4;
 constexpr uint32_t TMEM_COLS = 512;
 // S^T, dP^T: A = K_j or V_j (K-major over d), B = Q_i or dO_i (K-major over d)
 constexpr uint32_t IDESC_KQ = idesc_bf16(128, 128, false, false);
@@ -99,27 +101,37 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t da = ka + 3 * TILE_BYTES;   // dO_i
   const uint32_t pta = ka + 4 * TILE_BYTES;  // P^T
   const uint32_t sta = ka + 5 * TILE_BYTES;  // dS^T
-  float* lse_s = reinterpret_cast<float*>(base + 6 * TILE_BYTES);  // [128] LSE2
-  float* dd_s = lse_s + T;                                          // [128] D
-  uint64_t* bars = reinterpret_cast<uint64_t*>(dd_s + T + 256);
+  // per-query LSE * log2(e) and D, two buffers each: the next kept tile's
+  // values land in one while the current tile reads the other
+  float* lse_s = reinterpret_cast<float*>(base + 6 * TILE_BYTES);  // [2][128]
+  float* dd_s = lse_s + 2 * T;                                      // [2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(dd_s + 2 * T);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* list = reinterpret_cast<int*>(bars + 8);  // [LIST_CHUNK]
-  int* wcount = list + LIST_CHUNK;               // [4]
+  int* wcount = list + LIST_CHUNK;               // [LIST_ROUNDS][NWARP]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int lane = tid & 31;
+  // Warps w and w + 4 share TMEM lanes 32 (w mod 4) .. +31 and split the
+  // 128 columns of each accumulator into halves: row = this thread's lane
+  // of the tile (a key for S^T / dP^T, a query for dQ), half = which 64.
+  const int row = tid & (T - 1);
+  const int half = warp >> 2;
   const int j = blockIdx.x;   // key block 0 has the most query blocks: first
   const int zkv = blockIdx.y;  // (b, key/value head): K_j, V_j, dK_j, dV_j
   // dK_j and dV_j sum over the G query heads that share this key/value head
   const int zq0 = (zkv / p.Hkv) * p.Hq + (zkv % p.Hkv) * p.G;
   const uint32_t bar_kv = smem_u32(&bars[0]);
   const uint32_t bar_q = smem_u32(&bars[1]);
+  const uint32_t bar_do = smem_u32(&bars[2]);
   const uint32_t bar_mma = smem_u32(&bars[3]);
 
   if (tid == 0) {
     mbar_init(bar_kv, 1);
     mbar_init(bar_q, 1);
+    mbar_init(bar_do, 1);
     mbar_init(bar_mma, 1);
     *abort = 0;
     fence_mbar_init();
@@ -133,12 +145,14 @@ __global__ void __launch_bounds__(NT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const uint32_t t_st = tmem + lane_base;         // S^T, then dQ
-  const uint32_t t_dpt = tmem + lane_base + 128;  // dP^T
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const uint32_t t_st = tmem + lane_base + half * 64;         // S^T, then dQ
+  const uint32_t t_dpt = tmem + lane_base + 128 + half * 64;  // dP^T
   const uint32_t t_dk = tmem + lane_base + 256;
   const uint32_t t_dv = tmem + lane_base + 384;
 
+  // K_j, V_j: waited for before the first product, so the load overlaps the
+  // listing of the kept query blocks
   if (tid == 0) {
     mbar_expect_tx(bar_kv, 2 * TILE_BYTES);
     tma_load_3d(ka, &tmK, 0, j * T, zkv, bar_kv);
@@ -146,50 +160,100 @@ __global__ void __launch_bounds__(NT, 1)
     tma_load_3d(va, &tmV, 0, j * T, zkv, bar_kv);
     tma_load_3d(va + HALF_BYTES, &tmV, 64, j * T, zkv, bar_kv);
   }
-  uint32_t ph_q = 0, ph_mma = 0;
+  // Phases and copies/MMAs in flight; thread 0 issues every copy and MMA,
+  // so its own view is the one that the exit path settles.
+  uint32_t ph_q = 0, ph_do = 0, ph_mma = 0;
+  bool kv_pend = true, q_pend = false, do_pend = false, mma_pend = false;
+  bool kv_ready = false;
   int kept_count = 0;
-  bool ok = mbar_wait(bar_kv, 0, abort, 0x201);
+  int tcount = 0;  // tiles done by this CTA: picks the LSE / D buffer
+  bool ok = true;
   const int nw = (p.nb + 31) >> 5;
-  const int lane = tid & 31;
 
   for (int hg = 0; hg < p.G && ok; ++hg) {
   const int z = zq0 + hg;  // query head: Q_i, dO_i, LSE, D, dQ, the keep bits
   const int kept_before = kept_count;
   for (int i0 = j; i0 < p.nb && ok; i0 += LIST_CHUNK) {
-    // ---- list the kept query blocks i in [i0, i0 + LIST_CHUNK), ascending
-    int n_list = 0;
-    for (int k = 0; k < LIST_CHUNK / NT; ++k) {
+    // ---- list the kept query blocks i in [i0, i0 + LIST_CHUNK), ascending:
+    // every bit word is loaded first, then one barrier orders the counts
+    bool fk[LIST_ROUNDS];
+    unsigned bal[LIST_ROUNDS];
+#pragma unroll
+    for (int k = 0; k < LIST_ROUNDS; ++k) {
       const int i = i0 + k * NT + tid;
-      bool f = false;
-      if (i < p.nb)
-        f = p.never_skip ||
-            ((p.bits[((size_t)z * p.nb + i) * nw + (j >> 5)] >> (j & 31)) & 1u);
-      const unsigned bal = __ballot_sync(0xffffffffu, f);
-      if (lane == 0) wcount[warp] = __popc(bal);
-      __syncthreads();
-      int off = n_list;
-      for (int w = 0; w < warp; ++w) off += wcount[w];
-      if (f) list[off + __popc(bal & ((1u << lane) - 1u))] = i;
-      n_list += wcount[0] + wcount[1] + wcount[2] + wcount[3];
-      __syncthreads();
+      const bool in = i < p.nb;
+      const uint32_t w =
+          (in && !p.never_skip) ? p.bits[((size_t)z * p.nb + i) * nw + (j >> 5)] : 0u;
+      fk[k] = in && (p.never_skip || ((w >> (j & 31)) & 1u));
     }
+#pragma unroll
+    for (int k = 0; k < LIST_ROUNDS; ++k) {
+      bal[k] = __ballot_sync(0xffffffffu, fk[k]);
+      if (lane == 0) wcount[k * NWARP + warp] = __popc(bal[k]);
+    }
+    __syncthreads();
+    int n_list = 0;
+#pragma unroll
+    for (int k = 0; k < LIST_ROUNDS; ++k) {
+      int off = n_list, tot = 0;
+#pragma unroll
+      for (int w = 0; w < NWARP; ++w) {
+        const int c = wcount[k * NWARP + w];
+        off += w < warp ? c : 0;
+        tot += c;
+      }
+      if (fk[k]) list[off + __popc(bal[k] & ((1u << lane) - 1u))] = i0 + k * NT + tid;
+      n_list += tot;
+    }
+    __syncthreads();
+    // Within a list, tile li + 1's Q, dO, LSE and D are fetched while tile li
+    // is still being worked on: dO once the dP / dV products have read it,
+    // Q once the dK / dQ products have, LSE and D into the other buffer.
+    // Threads 0-127 move the LSE of query `row`, threads 128-255 its D.
+    bool prefetched = false;
     for (int li = 0; li < n_list && ok; ++li) {
     const int i = list[li];
-    {
-      const int q = i * T + tid;
+    const bool has_next = li + 1 < n_list;
+    const int inext = has_next ? list[li + 1] : 0;
+    float* lse_c = lse_s + (tcount & 1) * T;
+    float* dd_c = dd_s + (tcount & 1) * T;
+    if (!prefetched) {
+      const int q = i * T + row;
       const bool qv = q < p.L;
-      lse_s[tid] = qv ? p.LSE[(size_t)z * p.L + q] * kLog2e : 0.f;
-      dd_s[tid] = qv ? p.Dterm[(size_t)z * p.L + q] : 0.f;
+      if (half == 0)
+        lse_c[row] = qv ? p.LSE[(size_t)z * p.L + q] * kLog2e : 0.f;
+      else
+        dd_c[row] = qv ? p.Dterm[(size_t)z * p.L + q] : 0.f;
+      if (tid == 0) {
+        mbar_expect_tx(bar_q, TILE_BYTES);
+        tma_load_3d(qa, &tmQ, 0, i * T, z, bar_q);
+        tma_load_3d(qa + HALF_BYTES, &tmQ, 64, i * T, z, bar_q);
+        mbar_expect_tx(bar_do, TILE_BYTES);
+        tma_load_3d(da, &tmdO, 0, i * T, z, bar_do);
+        tma_load_3d(da + HALF_BYTES, &tmdO, 64, i * T, z, bar_do);
+        q_pend = do_pend = true;
+      }
     }
-    if (tid == 0) {
-      mbar_expect_tx(bar_q, 2 * TILE_BYTES);
-      tma_load_3d(qa, &tmQ, 0, i * T, z, bar_q);
-      tma_load_3d(qa + HALF_BYTES, &tmQ, 64, i * T, z, bar_q);
-      tma_load_3d(da, &tmdO, 0, i * T, z, bar_q);
-      tma_load_3d(da + HALF_BYTES, &tmdO, 64, i * T, z, bar_q);
+    // next tile's LSE or D: loaded now, stored once this tile is done
+    float next_val = 0.f;
+    if (has_next) {
+      const int q = inext * T + row;
+      if (q < p.L) next_val = (half == 0 ? p.LSE : p.Dterm)[(size_t)z * p.L + q];
     }
-    if (!mbar_wait(bar_q, ph_q, abort, 0x202)) ok = false;
-    ph_q ^= 1;
+    if (!kv_ready) {
+      if (mbar_wait(bar_kv, 0, abort, 0x201)) {
+        kv_pend = false;
+      } else {
+        ok = false;
+      }
+      kv_ready = true;
+    }
+    if (mbar_wait(bar_q, ph_q, abort, 0x202)) {
+      ph_q ^= 1;
+      q_pend = false;
+    } else {
+      ok = false;
+    }
     if (__syncthreads_or(!ok)) { ok = false; break; }
     // ---- S^T = K_j Q_i^T -----------------------------------------------------
     if (tid == 0) {
@@ -201,36 +265,47 @@ __global__ void __launch_bounds__(NT, 1)
                  IDESC_KQ, kk > 0);
       }
       mma_commit(bar_mma);
+      mma_pend = true;
     }
-    if (!mbar_wait(bar_mma, ph_mma, abort, 0x203)) ok = false;
-    ph_mma ^= 1;
+    if (mbar_wait(bar_mma, ph_mma, abort, 0x203)) {
+      ph_mma ^= 1;
+      mma_pend = false;
+    } else {
+      ok = false;
+    }
     if (__syncthreads_or(!ok)) { ok = false; break; }
     tc_fence_after();
     const bool diag = (i == j);
     {
-      // P^T row (key tid) over the block's queries, fp32 kept for dS
-      float pr[T];
+      // P^T row (key `row`) over this thread's 64 queries, fp32 kept for dS
+      float pr[T / 2];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float s[32];
         tmem_ld32(t_st + c * 32, s);
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int qc = c * 32 + e;
-          const bool legal = (!diag || qc >= tid) && (i * T + qc) < p.L;
-          pr[qc] = legal ? exp2f(s[e] * p.scale_log2 - lse_s[qc]) : 0.f;
+          const int qc = half * 64 + c * 32 + e;
+          const bool legal = (!diag || qc >= row) && (i * T + qc) < p.L;
+          pr[c * 32 + e] = legal ? exp2f(s[e] * p.scale_log2 - lse_c[qc]) : 0.f;
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int q0 = c * 32 + q * 8;
-          st_shared_v4(pta + sw128_chunk_off(tid, q0, T), pack_bf16(pr[q0], pr[q0 + 1]),
-                       pack_bf16(pr[q0 + 2], pr[q0 + 3]), pack_bf16(pr[q0 + 4], pr[q0 + 5]),
-                       pack_bf16(pr[q0 + 6], pr[q0 + 7]));
+          st_shared_v4(pta + sw128_chunk_off(row, half * 64 + q0, T),
+                       pack_bf16(pr[q0], pr[q0 + 1]), pack_bf16(pr[q0 + 2], pr[q0 + 3]),
+                       pack_bf16(pr[q0 + 4], pr[q0 + 5]), pack_bf16(pr[q0 + 6], pr[q0 + 7]));
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      __syncthreads();
+      if (mbar_wait(bar_do, ph_do, abort, 0x204)) {
+        ph_do ^= 1;
+        do_pend = false;
+      } else {
+        ok = false;
+      }
+      if (__syncthreads_or(!ok)) { ok = false; break; }
       // ---- dP^T = V_j dO_i^T ; dV += P^T dO_i ---------------------------------
       if (tid == 0) {
         tc_fence_after();
@@ -248,18 +323,30 @@ __global__ void __launch_bounds__(NT, 1)
                    (kept_count > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar_mma);
+        mma_pend = true;
       }
-      if (!mbar_wait(bar_mma, ph_mma, abort, 0x205)) ok = false;
-      ph_mma ^= 1;
+      if (mbar_wait(bar_mma, ph_mma, abort, 0x205)) {
+        ph_mma ^= 1;
+        mma_pend = false;
+      } else {
+        ok = false;
+      }
       if (__syncthreads_or(!ok)) { ok = false; break; }
       tc_fence_after();
+      // dO_i has been read: the next tile's dO goes into its buffer now
+      if (tid == 0 && has_next) {
+        mbar_expect_tx(bar_do, TILE_BYTES);
+        tma_load_3d(da, &tmdO, 0, inext * T, z, bar_do);
+        tma_load_3d(da + HALF_BYTES, &tmdO, 64, inext * T, z, bar_do);
+        do_pend = true;
+      }
       // ---- dS^T = P^T o (dP^T - D) * scale as a bf16 pair hi + lo --------------
       // dQ sums dS K over keys whose rows of dS cancel (each full row of dS
       // sums to zero), so a single bf16 rounding of dS costs several percent
       // of dQ; hi + lo carries ~16 significant bits. lo goes into the P^T
       // buffer, free now that the dV product has completed.
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float dp[32];
         tmem_ld32(t_dpt + c * 32, dp);
 #pragma unroll
@@ -267,15 +354,16 @@ __global__ void __launch_bounds__(NT, 1)
           uint32_t whi[4], wlo[4];
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
-            const int q0 = c * 32 + q * 8 + e;
-            const float a = pr[q0] * (dp[q * 8 + e] - dd_s[q0]) * p.scale;
-            const float b = pr[q0 + 1] * (dp[q * 8 + e + 1] - dd_s[q0 + 1]) * p.scale;
+            const int lc = c * 32 + q * 8 + e;  // this thread's column
+            const int qc = half * 64 + lc;      // the tile's query column
+            const float a = pr[lc] * (dp[q * 8 + e] - dd_c[qc]) * p.scale;
+            const float b = pr[lc + 1] * (dp[q * 8 + e + 1] - dd_c[qc + 1]) * p.scale;
             const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
             const float2 hf = __bfloat1622float2(h);
             whi[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
             wlo[e >> 1] = pack_bf16(a - hf.x, b - hf.y);
           }
-          const uint32_t off = sw128_chunk_off(tid, c * 32 + q * 8, T);
+          const uint32_t off = sw128_chunk_off(row, half * 64 + c * 32 + q * 8, T);
           st_shared_v4(sta + off, whi[0], whi[1], whi[2], whi[3]);
           st_shared_v4(pta + off, wlo[0], wlo[1], wlo[2], wlo[3]);
         }
@@ -308,18 +396,32 @@ __global__ void __launch_bounds__(NT, 1)
           }
         }
         mma_commit(bar_mma);
+        mma_pend = true;
       }
-      if (!mbar_wait(bar_mma, ph_mma, abort, 0x206)) ok = false;
-      ph_mma ^= 1;
+      if (mbar_wait(bar_mma, ph_mma, abort, 0x206)) {
+        ph_mma ^= 1;
+        mma_pend = false;
+      } else {
+        ok = false;
+      }
       if (__syncthreads_or(!ok)) { ok = false; break; }
       tc_fence_after();
+      // Q_i has been read: the next tile's Q goes into its buffer now
+      if (tid == 0 && has_next) {
+        mbar_expect_tx(bar_q, TILE_BYTES);
+        tma_load_3d(qa, &tmQ, 0, inext * T, z, bar_q);
+        tma_load_3d(qa + HALF_BYTES, &tmQ, 64, inext * T, z, bar_q);
+        q_pend = true;
+      }
       ++kept_count;
-      // ---- dQ_i rows (lane = query) added into the float32 workspace ----------
-      // tcgen05.ld is warp-collective: every lane loads, only valid rows add.
-      const int q = i * T + tid;
-      float4* dst = reinterpret_cast<float4*>(p.dQacc + ((size_t)z * p.L + (q < p.L ? q : 0)) * D);
+      // ---- dQ_i rows (lane = query `row`, this thread's 64 of d) added into
+      // the float32 workspace; tcgen05.ld is warp-collective: every lane
+      // loads, only valid rows add.
+      const int q = i * T + row;
+      float4* dst = reinterpret_cast<float4*>(p.dQacc + ((size_t)z * p.L + (q < p.L ? q : 0)) * D +
+                                              half * 64);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float v[32];
         tmem_ld32(t_st + c * 32, v);
         if (q < p.L) {
@@ -329,31 +431,48 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
     }
-    // Q_i, dO_i and the TMEM columns are free once every MMA above completed
+    if (has_next) {
+      if (half == 0)
+        lse_s[((tcount + 1) & 1) * T + row] = next_val * kLog2e;
+      else
+        dd_s[((tcount + 1) & 1) * T + row] = next_val;
+    }
+    prefetched = has_next;
+    ++tcount;
+    // the TMEM columns (and the LSE / D buffer just filled) are ready for
+    // the next tile once every thread is here
     tc_fence_before();
     __syncthreads();
     }
   }
   if (tid == 0 && p.kept_tiles) p.kept_tiles[(size_t)z * p.nb + j] = kept_count - kept_before;
   }
+  // thread 0's copies and MMAs still in flight (K_j, V_j when no tile was
+  // kept; anything on the error path) land before the CTA releases its
+  // shared memory and TMEM
+  if (tid == 0) {
+    if (kv_pend) mbar_settle(bar_kv, 0);
+    if (!ok) {
+      if (q_pend) mbar_settle(bar_q, ph_q);
+      if (do_pend) mbar_settle(bar_do, ph_do);
+      if (mma_pend) mbar_settle(bar_mma, ph_mma);
+    }
+  }
 
-  // ---- epilogue: dK_j, dV_j (bf16); zero if no tile was kept ----------------
-  // (TMEM loads are warp-collective: all lanes load, valid key rows store)
-  const int key = j * T + tid;
+  // ---- epilogue: dK_j (warps 0-3), dV_j (warps 4-7) in bf16; zero if no
+  // tile was kept (TMEM loads are warp-collective: all lanes load, valid key
+  // rows store)
+  const int key = j * T + row;
   if (ok) {
-    __nv_bfloat16* dk = p.dK + ((size_t)zkv * p.L + (key < p.L ? key : 0)) * D;
-    __nv_bfloat16* dv = p.dV + ((size_t)zkv * p.L + (key < p.L ? key : 0)) * D;
+    __nv_bfloat16* dst =
+        (half == 0 ? p.dK : p.dV) + ((size_t)zkv * p.L + (key < p.L ? key : 0)) * D;
     if (kept_count > 0) {
       tc_fence_after();
-      store_row_bf16(dk, t_dk, key < p.L);
-      store_row_bf16(dv, t_dv, key < p.L);
+      store_row_bf16(dst, half == 0 ? t_dk : t_dv, key < p.L);
     } else if (key < p.L) {
       uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
-        reinterpret_cast<uint4*>(dk)[c] = zero;
-        reinterpret_cast<uint4*>(dv)[c] = zero;
-      }
+      for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = zero;
     }
   }
   tc_fence_before();

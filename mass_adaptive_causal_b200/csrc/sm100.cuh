@@ -62,6 +62,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Bounded wait that ignores the abort flag: on an error path, lets this
+// CTA's own copies or MMAs still in flight land before it releases its
+// shared memory and TMEM.
+__device__ __forceinline__ void mbar_settle(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kWaitLimitNs) {
+  }
+}
+
 // Same as mbar_wait but polls with the non-suspending test_wait: for a
 // single thread whose only job is to react to the phase (the MMA issuer),
 // this avoids the wake-up latency of a suspended try_wait.
