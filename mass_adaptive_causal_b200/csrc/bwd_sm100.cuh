@@ -11,10 +11,13 @@
 //   P = exp(S - LSE), dV_j += P^T dO_i, dP = dO_i V_j^T, dS = P o (dP - D),
 //   dK_j += scale dS^T Q_i, dQ_i += scale dS K_j.
 //
-// CTA (128 threads) = one key block j: it lists the kept query blocks
-// i >= j of its column of the bit matrix, then for each: loads Q_i and dO_i,
-// recomputes S^T = K_j Q_i^T with keys in TMEM lanes (thread t owns key t),
-// and accumulates dK_j, dV_j in TMEM:
+// CTA (256 threads) = one key block j: it lists the kept query blocks
+// i >= j of its column of the bit matrix, then for each: loads Q_i and dO_i
+// (the next kept block's while the current one is worked on), recomputes
+// S^T = K_j Q_i^T with keys in TMEM lanes, and accumulates dK_j, dV_j in
+// TMEM. Threads t and t + 128 own TMEM lane t mod 128 and split the 128
+// columns of each accumulator into halves, so the elementwise work of a
+// tile (P, dS, the dQ readout) is spread over 8 warps:
 //   TMEM [  0,128): S^T, later reused for dQ_i = dS K_j
 //   TMEM [128,256): dP^T = V_j dO_i^T
 //   TMEM [256,384): dK_j accumulator      TMEM [384,512): dV_j accumulator
