@@ -31,6 +31,17 @@ MUTATIONS = {
                                                 "const double crit = (mx - LSE[r0]) - log_threshold(tau, (double)(row + 1));"),
     "decode threshold length": ("const double lthr = log_threshold(tau, (double)Lc);",
                                 "const double lthr = log_threshold(tau, (double)T);"),
+    "decode group test reads the first head only": (
+        "for (int r = 0; r < rows; ++r) {\n          const double crit = (mt[r] - m[r] - log(l[r])) - lthr;",
+        "for (int r = 0; r < 1; ++r) {\n          const double crit = (mt[r] - m[r] - log(l[r])) - lthr;"),
+    "decode group test needs every head": (
+        "kept = 0;\n        for (int r = 0; r < rows; ++r) {\n          const double crit = (mt[r] - m[r] - log(l[r])) - lthr;\n          if (crit > mu) mu = crit;\n          if (crit >= 0.0) kept = 1;",
+        "kept = 1;\n        for (int r = 0; r < rows; ++r) {\n          const double crit = (mt[r] - m[r] - log(l[r])) - lthr;\n          if (crit > mu) mu = crit;\n          if (crit < 0.0) kept = 0;"),
+    "decode traversal oldest first": ("for (int t = nt - 1; t >= 0; --t) {\n      const int c0 = t * T, c1 = imin(Lc, (t + 1) * T);",
+                                      "for (int t = 0; t < nt; ++t) {\n      const int c0 = t * T, c1 = imin(Lc, (t + 1) * T);"),
+    "decode scores use the group's first head": (
+        "const double v = scale * dot(q + (size_t)(h0 + r) * d, Kg + (size_t)c * d, d);",
+        "const double v = scale * dot(q + (size_t)h0 * d, Kg + (size_t)c * d, d);"),
     "chunk threshold ignores the cache": (
         "const double crit = lhs - log_threshold(tau, (double)(off + r0 + r + 1));",
         "const double crit = lhs - log_threshold(tau, (double)(r0 + r + 1));"),

@@ -362,6 +362,89 @@ def test_decode_group_rows():
         assert np.allclose(grp["o"][h], (w / w.sum()) @ Vc[g][kept_cols], rtol=0, atol=1e-12)
 
 
+def decode_consistent_sets(S, T, tau):
+    """All subsets of a cache's key tiles (the newest always in) consistent
+    with the sequential decode test, re-derived from the definition: rows are
+    the heads in S ([rows][Lc] scores), a tile is kept when any row's ratio
+    exp(tile max) / (sum of exp over the kept tiles visited earlier) reaches
+    tau / Lc; plain sums, no online update."""
+    Lc = len(S[0])
+    nt = -(-Lc // T)
+    found = []
+    for bits in itertools.product([0, 1], repeat=nt - 1):
+        kept = {nt - 1} | {t for t in range(nt - 1) if bits[t]}
+        ok = True
+        for t in range(nt - 2, -1, -1):
+            earlier = [tt for tt in kept if tt > t]
+            keep_t = False
+            for s in S:
+                z = sum(math.exp(s[c]) for tt in earlier for c in range(tt * T, min((tt + 1) * T, Lc)))
+                mt = max(s[c] for c in range(t * T, min((t + 1) * T, Lc)))
+                if math.exp(mt) / z >= tau / Lc:
+                    keep_t = True
+            if (t in kept) != keep_t:
+                ok = False
+                break
+        if ok:
+            found.append(kept)
+    return found
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_decode_bruteforce_keep_sets(T):
+    """Tiny caches: exactly one keep set per KV group (group rows) and per head
+    (per-head rows) is consistent with the sequential rule, it is the
+    oracle's, and each head's output is the softmax over the kept keys."""
+    Hq, Hkv, Lc, d, tau = 6, 2, 11, 3, 1.0
+    G = Hq // Hkv
+    nt = -(-Lc // T)
+    skipped = kept_old = 0
+    for seed in range(3):
+        rng = np.random.default_rng(5100 + seed)
+        q = rng.standard_normal((Hq, d)) * 1.8
+        Kc = rng.standard_normal((Hkv, Lc, d)) * 1.8
+        Vc = rng.standard_normal((Hkv, Lc, d))
+        S = [q[h] @ Kc[h // G].T / math.sqrt(d) for h in range(Hq)]
+        for per_head in (False, True):
+            out = oracle.decode(q, Kc, Vc, tau=tau, tile=T, per_head=per_head)
+            for u in range(Hq if per_head else Hkv):
+                heads = [u] if per_head else list(range(u * G, (u + 1) * G))
+                sets = decode_consistent_sets([S[h] for h in heads], T, tau)
+                assert len(sets) == 1
+                assert sets[0] == {t for t in range(nt) if out["keep"][u, t]}
+                skipped += nt - len(sets[0])
+                kept_old += len(sets[0]) - 1
+                for h in heads:
+                    cols = [c for t in sets[0] for c in range(t * T, min((t + 1) * T, Lc))]
+                    w = np.exp(S[h][cols] - S[h][cols].max())
+                    assert np.allclose(out["o"][h], (w / w.sum()) @ Vc[h // G][cols], rtol=0,
+                                       atol=1e-12)
+    assert skipped > 0 and kept_old > 0  # both branches of the test were taken
+
+
+def test_decode_head_permutation():
+    """Permuting the query heads inside each KV group leaves the group's keep
+    set unchanged and permutes the outputs; permuting the KV groups together
+    with their query heads permutes both."""
+    Hq, Hkv, Lc, d = 8, 2, 700, 16
+    G = Hq // Hkv
+    rng = np.random.default_rng(29)
+    q = rng.standard_normal((Hq, d)) * 2.5
+    Kc = rng.standard_normal((Hkv, Lc, d)) * 2.5
+    Vc = rng.standard_normal((Hkv, Lc, d))
+    base = oracle.decode(q, Kc, Vc, tau=1.0, tile=32)
+    assert 0 < base["keep"].sum() < base["keep"].size
+    inner = np.concatenate([g * G + rng.permutation(G) for g in range(Hkv)])
+    p = oracle.decode(q[inner], Kc, Vc, tau=1.0, tile=32)
+    assert np.array_equal(p["keep"], base["keep"])
+    assert np.array_equal(p["o"], base["o"][inner])
+    gp = np.array([1, 0])
+    heads = np.concatenate([np.arange(g * G, (g + 1) * G) for g in gp])
+    p = oracle.decode(q[heads], Kc[gp], Vc[gp], tau=1.0, tile=32)
+    assert np.array_equal(p["keep"], base["keep"][gp])
+    assert np.array_equal(p["o"], base["o"][heads])
+
+
 def test_tile_row_max_bruteforce():
     """Pure-Python enumeration of every (row, legal key) score on a tiny
     ragged case (L = 7, tile 3: blocks of 3, 3, 1 rows)."""
