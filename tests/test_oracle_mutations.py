@@ -27,6 +27,8 @@ MUTATIONS = {
                         "const double ds = p * (dp + D[row]);\n          for (int k = 0; k < d; ++k) {"),
     "backward dK transposed operand": ("dK[(size_t)c * d + k] += scale * ds * Q[(size_t)row * d + k];",
                                        "dK[(size_t)c * d + k] += scale * ds * K[(size_t)row * d + k];"),
+    "backward forces the diagonal tile": ("if (force_first && j == i) { *mu_out = INFINITY; return 1; }",
+                                          "if (j == i) { *mu_out = INFINITY; return 1; }"),
     "backward test uses row max of wrong row": ("const double crit = (mx - LSE[row]) - log_threshold(tau, (double)(row + 1));",
                                                 "const double crit = (mx - LSE[r0]) - log_threshold(tau, (double)(row + 1));"),
     "decode threshold length": ("const double lthr = log_threshold(tau, (double)Lc);",
