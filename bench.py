@@ -132,29 +132,66 @@ def generate_inputs(workers: int, seed_shift: int = 0):
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """nvidia-smi sampling of one GPU's SM clock and throttle reasons.
+
+    start() launches the sampler and waits (at most a few seconds) until it
+    has written a first sample, so that the timed region that follows is
+    covered; mark("begin") / mark("end") bracket the timed region on the
+    host clock; stop() summarises the samples whose timestamps fall inside
+    that window (all samples when none does, and the line says which).
+    Throttle reasons are collected over every sample of the run."""
+
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "timestamp")
+    PERIOD_MS = 50
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, tool: str = "nvidia-smi"):
         self.gpu = gpu_index
+        self.tool = tool
         self.proc = None
+        self.marks = {}
         # the raw samples go to MALA_BENCH_OUT (default: the system's temp
         # directory); the JSON line carries their summary
         import tempfile
         out = os.environ.get("MALA_BENCH_OUT", tempfile.gettempdir())
         self.path = os.path.join(out, f"clocks_gpu{gpu_index}.csv")
 
-    def start(self):
+    def start(self, first_sample_timeout: float = 3.0):
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                [self.tool, "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)], stdout=self.fh,
                 stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        t0 = time.time()
+        while time.time() - t0 < first_sample_timeout and self.proc.poll() is None:
+            try:
+                if os.path.getsize(self.path) > 0:
+                    break
+            except OSError:
+                break
+            time.sleep(0.01)
+
+    def mark(self, which: str):
+        import datetime
+        self.marks[which] = datetime.datetime.now()
+
+    @staticmethod
+    def _timestamp(text: str):
+        import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(text, fmt)
+            except ValueError:
+                pass
+        return None
 
     def stop(self):
         if self.proc is None:
@@ -165,24 +202,33 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.fh.close()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows, reasons = [], set()
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
+                sm, smax = float(f[1]), float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(self.REASONS, f[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        if not sm:
+            rows.append((self._timestamp(f[9]) if len(f) > 9 else None, sm, smax))
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        import datetime
+        b, e = self.marks.get("begin"), self.marks.get("end")
+        inside = []
+        if b is not None and e is not None:
+            # a sample stands for the period that ends at its timestamp
+            late = e + datetime.timedelta(milliseconds=self.PERIOD_MS)
+            inside = [r for r in rows if r[0] is not None and b <= r[0] <= late]
+        use = inside or rows
+        return {"sm_mhz": statistics.median(r[1] for r in use),
+                "sm_max_mhz": max(r[2] for r in use), "reasons": sorted(reasons),
+                "samples": len(use),
+                "window": "timed region" if inside else "whole run (none inside the timed region)"}
 
 
 # ---------------------------------------------------------------------------
@@ -302,7 +348,7 @@ def run_mala(args, rank, world, local_rank):
     def max_over_ranks(v: float) -> float:
         return reduce_max(v, world, dev)
 
-    def timed(tau, steps, warmup, rowmax=True):
+    def timed(tau, steps, warmup, rowmax=True, clock=None):
         for _ in range(warmup):
             step(tau, rowmax=rowmax)
         mala.mala_check()
@@ -311,11 +357,15 @@ def run_mala(args, rank, world, local_rank):
         torch.cuda.synchronize()
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
+        if clock is not None:
+            clock.mark("begin")
         start.record(stream)
         for k in range(steps):
             step(tau, evs[k], rowmax=rowmax)
         end.record(stream)
         torch.cuda.synchronize()
+        if clock is not None:
+            clock.mark("end")
         barrier()
         mala.mala_check()
         total = start.elapsed_time(end)
@@ -343,7 +393,7 @@ def run_mala(args, rank, world, local_rank):
 
     clock = ClockSampler(local_rank)
     clock.start()
-    t1 = timed(1.0, args.steps, args.warmup)
+    t1 = timed(1.0, args.steps, args.warmup, clock=clock)
     clocks = clock.stop()
     work1 = trace(1.0)
     # the backward that recomputes every tile's scores for its test (no row maxima)
