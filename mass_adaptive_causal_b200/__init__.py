@@ -107,23 +107,126 @@ def _dtype_code(t):
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def _check_prefill(q, k, v, *rest):
+# ---------------------------------------------------------------------------
+# host checks: the C ABI receives bare pointers, so every size it relies on
+# is checked here against the tensors before a pointer crosses. Each check
+# takes ``require_cuda`` so that its logic runs on CPU tensors in the tests.
+# ---------------------------------------------------------------------------
+def _inputs(ts, dev, require_cuda, what):
+    for t in ts:
+        if require_cuda and not t.is_cuda:
+            raise ValueError(f"{what} must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError(f"{what} must be contiguous")
+        if t.device != dev:
+            raise ValueError("every tensor of a call must be on one device")
+    if require_cuda and dev.index != _torch().cuda.current_device():
+        raise ValueError(f"the tensors are on {dev}, not on the current CUDA device "
+                         "(torch.cuda.set_device)")
+
+
+def _buf(t, name, dev, dtype, shape=None, min_bytes=None):
+    """A caller-supplied output or scratch tensor: contiguous, on ``dev``, of
+    ``dtype`` (any when None), exactly ``shape`` and/or at least ``min_bytes``."""
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != dev:
+        raise ValueError(f"{name} must be on {dev}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if min_bytes is not None and t.numel() * t.element_size() < min_bytes:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, needs {min_bytes}")
+    return t
+
+
+def _check_prefill(q, k, v, *rest, require_cuda=True):
     """q (and o, do in rest): [B, H, L, d]; k, v: [B, Hkv, L, d] with H % Hkv == 0
     (grouped query heads; Hkv = H is multi-head attention)."""
     torch = _torch()
+    _inputs((q, k, v) + rest, q.device, require_cuda, "Q, K, V, O, dO")
     for t in (q, k, v) + rest:
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("tensors must be contiguous CUDA tensors")
         if t.dtype != q.dtype or t.dim() != 4:
             raise ValueError("expected [B, H, L, d] tensors of one dtype")
     if k.shape != v.shape or k.shape[0] != q.shape[0] or k.shape[2:] != q.shape[2:]:
         raise ValueError("K and V must be [B, Hkv, L, d] matching Q's B, L, d")
-    if q.shape[1] % k.shape[1] != 0:
+    if k.shape[1] == 0 or q.shape[1] % k.shape[1] != 0:
         raise ValueError("the query heads must be a multiple of the key/value heads")
     for t in rest:
         if t.shape != q.shape:
             raise ValueError("O and dO must have Q's shape")
     return torch
+
+
+def _check_fwd_buffers(q, tile, out=None, lse=None, o32=None, rowmax=None):
+    torch = _torch()
+    B, H, L, _ = q.shape
+    if out is not None:
+        _buf(out, "out", q.device, q.dtype, q.shape)
+    if lse is not None:
+        _buf(lse, "lse", q.device, torch.float32, (B, H, L))
+    if o32 is not None:
+        _buf(o32, "o32", q.device, torch.float32, q.shape)
+    if rowmax is not None:
+        _buf(rowmax, "rowmax", q.device, torch.float32,
+             min_bytes=tile_rowmax_bytes(B, H, L, tile))
+
+
+def _check_bwd_buffers(q, k, lse, tile, o32=None, rowmax=None, grads=None, workspace=None):
+    torch = _torch()
+    B, H, L, _ = q.shape
+    _buf(lse, "lse", q.device, torch.float32, (B, H, L))
+    if o32 is not None:
+        _buf(o32, "o32", q.device, torch.float32, q.shape)
+    if rowmax is not None:
+        _buf(rowmax, "rowmax", q.device, torch.float32,
+             min_bytes=tile_rowmax_bytes(B, H, L, tile))
+    if grads is not None:
+        dq, dk, dv = grads
+        _buf(dq, "dQ", q.device, q.dtype, q.shape)
+        _buf(dk, "dK", q.device, q.dtype, k.shape)
+        _buf(dv, "dV", q.device, q.dtype, k.shape)
+    if workspace is not None:
+        _buf(workspace, "workspace", q.device, None)
+
+
+def _check_decode(q, k_cache, v_cache, out=None, workspace=None, require_cuda=True):
+    """q: [B, Hq, d] bf16; caches: [B, Hkv, Lc, d] bf16, the same shape."""
+    torch = _torch()
+    _inputs((q, k_cache, v_cache), q.device, require_cuda, "decode tensors")
+    for t in (q, k_cache, v_cache):
+        if t.dtype != torch.bfloat16:
+            raise ValueError("decode tensors must be bf16")
+    if q.dim() != 3 or k_cache.dim() != 4 or k_cache.shape != v_cache.shape:
+        raise ValueError("q must be [B, Hq, d], the caches [B, Hkv, Lc, d] of one shape")
+    if k_cache.shape[0] != q.shape[0] or k_cache.shape[3] != q.shape[2]:
+        raise ValueError("the caches' B and d must match q's")
+    if out is not None:
+        _buf(out, "out", q.device, q.dtype, q.shape)
+    if workspace is not None:
+        _buf(workspace, "workspace", q.device, None)
+
+
+def _check_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, out=None, lse=None, require_cuda=True):
+    """q: [total_q, H, d]; k, v: [total_k, Hkv, d] of one shape; cu_seqlens:
+    int32 [batch + 1] each."""
+    torch = _torch()
+    _inputs((q, k, v, cu_seqlens_q, cu_seqlens_k), q.device, require_cuda, "varlen tensors")
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or t.dim() != 3:
+            raise ValueError("q, k, v must be [tokens, heads, d] bf16 tensors")
+    if k.shape != v.shape or k.shape[2] != q.shape[2]:
+        raise ValueError("k and v must be [total_k, Hkv, d] of one shape, d matching q's")
+    for t in (cu_seqlens_q, cu_seqlens_k):
+        if t.dtype != torch.int32 or t.dim() != 1:
+            raise ValueError("cu_seqlens must be 1-D int32 tensors")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold batch + 1 >= 2 offsets")
+    if out is not None:
+        _buf(out, "out", q.device, q.dtype, q.shape)
+    if lse is not None:
+        _buf(lse, "lse", q.device, torch.float32, (q.shape[1], q.shape[0]))
 
 
 def _raise(code, where):
@@ -171,6 +274,7 @@ def mala_fwd(q, k, v, tau: float = 1.0, tile: int | None = None, scale: float = 
                            device=q.device)
     elif rowmax is not None and rowmax is not False:
         rm_t = rowmax
+    _check_fwd_buffers(q, tile, out=o, lse=lse_t, o32=o32_t, rowmax=rm_t)
     kept = bits = None
     if trace:
         nb = n_blocks(L, tile)
@@ -195,12 +299,7 @@ def mala_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
     total_q]) or, with ``trace=True``, also kept_tiles [batch, H, nbq] and
     keep_bits [batch, H, nbq, nw] (bit k = key tile k)."""
     torch = _torch()
-    for t in (q, k, v):
-        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16 or t.dim() != 3:
-            raise ValueError("q, k, v must be contiguous [tokens, heads, d] bf16 CUDA tensors")
-    for t in (cu_seqlens_q, cu_seqlens_k):
-        if not t.is_cuda or t.dtype != torch.int32 or not t.is_contiguous():
-            raise ValueError("cu_seqlens must be contiguous int32 CUDA tensors")
+    _check_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, out=out, lse=lse)
     total_q, H, d = q.shape
     total_k, Hkv, _ = k.shape
     batch = cu_seqlens_q.numel() - 1
@@ -247,10 +346,11 @@ def mala_bwd(q, k, v, o, do, lse, tau: float = 1.0, tile: int | None = None,
         nb = n_blocks(L, tile)
         kept = torch.empty((B, H, nb), dtype=torch.int32, device=q.device)
         bits = torch.empty((B, H, nb, (nb + 31) // 32), dtype=torch.int32, device=q.device)
-    if rowmax is not None and rowmax.numel() * 4 < tile_rowmax_bytes(B, H, L, tile):
-        raise ValueError("rowmax is smaller than tile_rowmax_bytes")
+    _check_bwd_buffers(q, k, lse, tile, o32=o32, rowmax=rowmax, grads=(dq, dk, dv),
+                       workspace=ws)
     code = lib().mala_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(o32), _ptr(do), _ptr(lse),
-                          _ptr(rowmax), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), B, H,
+                          _ptr(rowmax), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                          ws.numel() * ws.element_size(), B, H,
                           k.shape[1], L, d, _dtype_code(q),
                           float(tau), int(tile), float(scale), _ptr(kept), _ptr(bits),
                           _stream(stream))
@@ -269,9 +369,7 @@ def mala_decode(q, k_cache, v_cache, tau: float = 1.0, scale: float = 0.0, trace
     keep_bits [B, Hkv, nw]); with ``per_head=True`` every query head applies
     the test alone and the trace is per query head ([B, Hq], [B, Hq, nw])."""
     torch = _torch()
-    for t in (q, k_cache, v_cache):
-        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
-            raise ValueError("decode tensors must be contiguous bf16 CUDA tensors")
+    _check_decode(q, k_cache, v_cache, out=out, workspace=workspace)
     B, Hq, d = q.shape
     _, Hkv, Lc, _ = k_cache.shape
     o = torch.empty_like(q) if out is None else out
@@ -285,7 +383,8 @@ def mala_decode(q, k_cache, v_cache, tau: float = 1.0, scale: float = 0.0, trace
         kept = torch.empty((B, rows), dtype=torch.int32, device=q.device)
         bits = torch.empty((B, rows, (nt + 31) // 32), dtype=torch.int32, device=q.device)
     code = lib().mala_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), B, Hq, Hkv, Lc, d,
-                             float(tau), float(scale), int(bool(per_head)), _ptr(ws), ws.numel(),
+                             float(tau), float(scale), int(bool(per_head)), _ptr(ws),
+                             ws.numel() * ws.element_size(),
                              _ptr(kept), _ptr(bits), _stream(stream))
     _raise(code, "mala_decode")
     return (o, kept, bits) if trace else o
@@ -304,9 +403,7 @@ def mala_decode_noalloc(q, k_cache, v_cache, tau: float = 1.0, scale: float = 0.
     holds. The output (and trace) tensors are the caller's: pass ``out`` to
     avoid allocating here too."""
     torch = _torch()
-    for t in (q, k_cache, v_cache):
-        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
-            raise ValueError("decode tensors must be contiguous bf16 CUDA tensors")
+    _check_decode(q, k_cache, v_cache, out=out)
     B, Hq, d = q.shape
     _, Hkv, Lc, _ = k_cache.shape
     o = torch.empty_like(q) if out is None else out
