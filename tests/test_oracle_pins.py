@@ -445,6 +445,51 @@ def test_decode_head_permutation():
     assert np.array_equal(p["o"], base["o"][heads])
 
 
+@pytest.mark.parametrize("tau,T", [(1.0, 8), (0.25, 8), (4.0, 4), (0.0, 8)])
+def test_forward_from_maxima_then_scan_then_pv(tau, T):
+    """The forward's rule re-derived in another order (numpy): every legal
+    tile's row maxima first; then, per query block, the sequential test on
+    those maxima alone, a kept tile's row sums exp(S - max) taken from its
+    scores only when it is kept; then O = sum over kept tiles of
+    exp(S - m) V / l with the final (m, l). It must give the oracle's keep
+    set, LSE and output."""
+    L, d = 203, 8
+    Q, K, V, _ = rand_inputs(L, d, 61, scale_qk=2.5)
+    scale = 1.0 / math.sqrt(d)
+    S = scale * Q @ K.T
+    S[np.triu(np.ones((L, L), bool), 1)] = -np.inf
+    nb = oracle.n_blocks(L, T)
+    f = oracle.fwd(Q, K, V, tile=T, tau=tau)
+    O = np.zeros((L, d))
+    LSE = np.zeros(L)
+    for i in range(nb):
+        rows = np.arange(i * T, min(L, (i + 1) * T))
+        tiles = [np.arange(j * T, min(L, (j + 1) * T)) for j in range(i + 1)]
+        mt = [S[np.ix_(rows, c)].max(axis=1) for c in tiles]        # phase A
+        m = np.full(len(rows), -np.inf)
+        l = np.zeros(len(rows))
+        kept = []
+        for j in range(i, -1, -1):                                    # phase B
+            if j != i and tau > 0:
+                lhs = mt[j] - m - np.log(l)
+                if np.all(lhs < math.log(tau) - np.log(rows + 1)):
+                    continue
+            kept.append(j)
+            lt = np.exp(S[np.ix_(rows, tiles[j])] - mt[j][:, None]).sum(axis=1)
+            mn = np.maximum(m, mt[j])
+            l = l * np.exp(m - mn) + lt * np.exp(mt[j] - mn)
+            m = mn
+        assert sorted(kept) == [j for j in range(i + 1) if f["keep"][i, j]]
+        cols = np.concatenate([tiles[j] for j in kept])               # phase C
+        P = np.exp(S[np.ix_(rows, cols)] - m[:, None])
+        O[rows] = P @ V[cols] / l[:, None]
+        LSE[rows] = m + np.log(l)
+    assert np.allclose(LSE, f["LSE"], rtol=0, atol=1e-12)
+    assert np.allclose(O, f["O"], rtol=0, atol=1e-12)
+    if tau > 0:
+        assert f["keep"][np.tril_indices(nb)].min() == 0  # something was skipped
+
+
 def test_tile_row_max_bruteforce():
     """Pure-Python enumeration of every (row, legal key) score on a tiny
     ragged case (L = 7, tile 3: blocks of 3, 3, 1 rows)."""
