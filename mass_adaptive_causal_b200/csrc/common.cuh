@@ -40,8 +40,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegInf = -__builtin_huge_valf();
 
-__device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
-
 // Keep-bit bookkeeping shared by the prefill kernels: row `rowblk` of the
 // [nb][nw] bit matrix of slice z. Thread 0 of a CTA accumulates 32 decisions
 // at a time and stores whole words, so no atomics are needed.

@@ -182,18 +182,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem]; A is M lanes x K columns of packed bf16
-// pairs (column c holds k = 2c, 2c+1, the even element in the low half).
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Arrive (count 1) on `bar` once every tcgen05 op this thread issued so far
 // has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -435,39 +423,6 @@ __device__ __forceinline__ float tmem_rowmax128_from(uint32_t taddr, int lo) {
     for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], e + k < lo ? ninf : __uint_as_float(v[e + k]));
   }
   return fmaxf(fmaxf(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5])), fmaxf(a[6], a[7]));
-}
-
-// Row max over 64 TMEM columns of this thread's lane (columns col0 .. col0+63
-// of the tile). With `diag`, tile columns c > r are excluded.
-__device__ __forceinline__ float tmem_rowmax64(uint32_t taddr, bool diag, int r, int col0) {
-  float s[64];
-  tmem_ld64(taddr, s);
-  float m = -__builtin_huge_valf();
-  if (!diag) {
-#pragma unroll
-    for (int e = 0; e < 63; e += 2) m = fmax3f(m, s[e], s[e + 1]);
-  } else {
-#pragma unroll
-    for (int e = 0; e < 64; ++e) m = fmaxf(m, (col0 + e > r) ? -__builtin_huge_valf() : s[e]);
-  }
-  return m;
-}
-
-// OR-vote / barrier over `count` threads on named barrier `id` (1..15).
-__device__ __forceinline__ int bar_vote_or(int pred, int id, int count) {
-  uint32_t out;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "barrier.cta.red.or.pred po, %2, %3, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}\n"
-      : "=r"(out)
-      : "r"(pred), "r"(id), "r"(count)
-      : "memory");
-  return (int)out;
-}
-__device__ __forceinline__ void bar_sync_n(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Byte offset of the 16-byte chunk holding element (row, col) of a bf16
