@@ -145,3 +145,18 @@ def test_fwd_varlen_argument_checks(lib):
                                0.0, None, None, None) == 1
     assert lib.mala_varlen_trace_words(100, 200) == 1
     assert lib.mala_varlen_trace_words(4096, 131072) == (32 + 1024 + 31) // 32
+
+
+def test_header_is_c_and_the_library_links_from_c(lib, tmp_path):
+    """A C11 program (tests/c/abi_host.c) includes include/mala.h, links
+    libmala.so and checks the calls that need no GPU."""
+    import subprocess
+    src = os.path.join(ROOT, "tests", "c", "abi_host.c")
+    exe = tmp_path / "abi_host"
+    libdir = os.path.dirname(mala.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I",
+                    os.path.join(ROOT, "include"), src, "-o", str(exe), f"-L{libdir}",
+                    f"-Wl,-rpath,{libdir}", "-l:libmala.so"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == "ok"
