@@ -283,6 +283,17 @@ mala_status mala_decode_noalloc(const void* q, const void* Kcache,
  */
 mala_status mala_check(void* stream);
 
+/*
+ * Diagnostic of the timeout path (no counterpart in the pages): launches one
+ * thread on `stream` that waits, with the bounded wait every kernel uses
+ * (about two seconds of %globaltimer), on a barrier that nothing arrives on.
+ * The wait runs out and records a timeout in the device status word, so the
+ * next mala_check returns MALA_ERR_TIMEOUT and clears it. Nothing traps, no
+ * memory is touched but the status word, and the context stays usable.
+ * Returns MALA_ERR_CUDA if the launch fails, MALA_OK otherwise.
+ */
+mala_status mala_selftest_wait(void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* mala_status_string(mala_status s);
 

@@ -19,7 +19,7 @@ import ctypes
 import os
 
 __all__ = ["mala_fwd", "mala_fwd_varlen", "mala_bwd", "mala_decode", "mala_decode_noalloc", "mala_check",
-           "MalaError", "lib",
+           "mala_selftest_wait", "MalaError", "lib",
            "LIB_PATH", "MALA_F32", "MALA_BF16", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.mala_decode_noalloc.restype = ci
         L.mala_check.argtypes = [_vp]
         L.mala_check.restype = ci
+        L.mala_selftest_wait.argtypes = [_vp]
+        L.mala_selftest_wait.restype = ci
         L.mala_status_string.argtypes = [ci]
         L.mala_status_string.restype = ctypes.c_char_p
         L.mala_version.argtypes = []
@@ -423,6 +425,13 @@ def mala_check(stream=None):
     """Synchronize the stream and raise MalaError if a kernel reported a
     timeout or the stream holds a CUDA error."""
     _raise(lib().mala_check(_stream(stream)), "mala_check")
+
+
+def mala_selftest_wait(stream=None):
+    """Diagnostic of the timeout path: one device thread waits, with the
+    kernels' bounded wait (about two seconds), on a barrier nothing arrives
+    on, so the next mala_check raises MalaError (MALA_ERR_TIMEOUT) once."""
+    _raise(lib().mala_selftest_wait(_stream(stream)), "mala_selftest_wait")
 
 
 def unpack_bits(bits, n: int):

@@ -62,3 +62,31 @@ extern "C" mala_status mala_decode_noalloc(const void* q, const void* Kcache, co
   return decode_bf16(q, Kcache, Vcache, o, B, Hq, Hkv, Lc, resolve_scale(scale, d), tau, 0, w,
                      kept_tiles, keep_bits, as_stream(stream));
 }
+
+// -------------------------------------------------------------------------
+// mala_selftest_wait: a wait that runs out on purpose, through the same
+// bounded mbarrier wait as every kernel, so that the status path
+// (record_timeout -> mala_check) can be tested without a fault.
+// -------------------------------------------------------------------------
+namespace {
+
+__global__ void selftest_wait_kernel() {
+  using namespace mala::sm100;
+  __shared__ uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // phase 0 never completes: nothing arrives on `bar`
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort, 0x7f0);
+}
+
+}  // namespace
+
+extern "C" mala_status mala_selftest_wait(void* stream) {
+  selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>();
+  return launch_status();
+}

@@ -16,7 +16,7 @@ bf16, f32 = torch.bfloat16, torch.float32
 
 class Recorder:
     COMPUTE = ("mala_fwd", "mala_fwd_varlen", "mala_bwd", "mala_decode", "mala_decode_noalloc",
-               "mala_check")
+               "mala_check", "mala_selftest_wait")
 
     def __init__(self, real):
         self.real = real
@@ -131,3 +131,8 @@ def test_varlen(rec):
     assert a[7:15] == [2, 100, 200, 150, 300, 4, 2, 128]
     assert LSE.shape == (4, 150) and kept.shape == (2, 4, 1)
     assert bits.shape == (2, 4, 1, mala.lib().mala_varlen_trace_words(100, 200))
+
+
+def test_selftest_wait(rec):
+    mala.mala_selftest_wait()
+    assert rec.calls[-1][0] == "mala_selftest_wait"

@@ -1,8 +1,8 @@
 """mala_decode_noalloc (the decode step whose scratch is the library's static
 device array) against mala_decode (caller-provided workspace), through the C
 ABI, on two calls in a row with different shapes, so that the second call
-runs over the first call's leftovers in the shared array. The file sorts last
-so that it runs after every other test as well as alone."""
+runs over the first call's leftovers in the shared array. The file sorts
+after the parity tests so that it runs after them as well as alone."""
 
 from __future__ import annotations
 
