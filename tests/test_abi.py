@@ -97,7 +97,6 @@ def test_bwd_and_decode_argument_checks(lib):
 
 
 def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
-    import importlib
     monkeypatch.setattr(mala, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(mala, "_lib", None)
     with pytest.raises(RuntimeError):

@@ -3,7 +3,6 @@ same seeded inputs. Every test here needs a B200 and the built library."""
 
 from __future__ import annotations
 
-import math
 
 import numpy as np
 import pytest

@@ -16,7 +16,6 @@ Every policy keeps exactly MALA's number of tiles in each query block.
 from __future__ import annotations
 
 import numpy as np
-import pytest
 
 import oracle
 import synth
