@@ -621,7 +621,7 @@ def tau_study(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mala", choices=["mala", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
