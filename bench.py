@@ -293,6 +293,22 @@ def reduce_max(v: float, world: int, device) -> float:
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
+def count_launches(fn):
+    """Kernels of this library launched by one call of ``fn``, counted from
+    the CUDA activity trace (torch.profiler / CUPTI): every kernel whose name
+    is in the library's namespaces."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    ours = [n for n in names if any(k in n for k in ("fwd2::", "bwd100::", "bwdtest::", "dec::",
+                                                          "aux::", "simt::"))]
+    return len(ours), sorted(set(n.split("(")[0] for n in ours))
+
+
 def run_mala(args, rank, world, local_rank):
     import torch
     import mass_adaptive_causal_b200 as mala
@@ -300,7 +316,6 @@ def run_mala(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     P, Dc = PREFILL, DECODE
-    G = Dc.Hq // Dc.Hkv
 
     def to_dev(u16, shape):
         t = torch.from_numpy(u16.view(np.int16)).view(torch.bfloat16).reshape(shape)
@@ -317,22 +332,20 @@ def run_mala(args, rank, world, local_rank):
     LSE = torch.empty((P.B, P.H, P.L), dtype=torch.float32, device=dev)
     dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
     o = torch.empty_like(q)
-    RM = torch.empty(mala.tile_rowmax_bytes(P.B, P.H, P.L, P.tile) // 4, dtype=torch.float32,
-                     device=dev)
     ws_b = torch.empty(mala.bwd_workspace_bytes(P.B, P.H, P.L, P.d), dtype=torch.uint8, device=dev)
     ws_d = torch.empty(mala.decode_workspace_bytes(Dc.B, Dc.Hq, Dc.Hkv, Dc.Lc, Dc.d),
                        dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(tau, ev=None, rowmax=True):
-        rm = RM if rowmax else None
+    def step(tau, ev=None):
+        # the training chain: only O (its float32 copy) and LSE go from the
+        # forward to the backward
         if ev is not None:
             ev[0].record(stream)
-        mala.mala_fwd(Q, K, V, tau=tau, out=O, lse=LSE, o32=O32, rowmax=rm)
+        mala.mala_fwd(Q, K, V, tau=tau, out=O, lse=LSE, o32=O32)
         if ev is not None:
             ev[1].record(stream)
-        mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, workspace=ws_b, grads=(dQ, dK, dV), o32=O32,
-                      rowmax=rm)
+        mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, workspace=ws_b, grads=(dQ, dK, dV), o32=O32)
         if ev is not None:
             ev[2].record(stream)
         mala.mala_decode(q, Kc, Vc, tau=tau, workspace=ws_d, out=o)
@@ -347,9 +360,9 @@ def run_mala(args, rank, world, local_rank):
     def max_over_ranks(v: float) -> float:
         return reduce_max(v, world, dev)
 
-    def timed(tau, steps, warmup, rowmax=True, clock=None):
+    def timed(tau, steps, warmup, clock=None):
         for _ in range(warmup):
-            step(tau, rowmax=rowmax)
+            step(tau)
         mala.mala_check()
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
         barrier()
@@ -360,7 +373,7 @@ def run_mala(args, rank, world, local_rank):
             clock.mark("begin")
         start.record(stream)
         for k in range(steps):
-            step(tau, evs[k], rowmax=rowmax)
+            step(tau, evs[k])
         end.record(stream)
         torch.cuda.synchronize()
         if clock is not None:
@@ -376,12 +389,11 @@ def run_mala(args, rank, world, local_rank):
                 "bwd_ms": max_over_ranks(sum(bwd) / steps),
                 "decode_us": max_over_ranks(1000 * sum(dec) / steps)}
 
-    # trace pass (untimed): retained work and kept decode tiles at tau=1 and 0
+    # trace pass (untimed): retained work and kept decode tiles at tau=1
     def trace(tau):
-        _, _, kept_f, bits_f = mala.mala_fwd(Q, K, V, tau=tau, trace=True, out=O, lse=LSE, o32=O32,
-                                             rowmax=RM)[:4]
-        _, _, _, kept_b, bits_b = mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, trace=True, o32=O32,
-                                                rowmax=RM)
+        _, _, kept_f, bits_f, _ = mala.mala_fwd(Q, K, V, tau=tau, trace=True, out=O, lse=LSE,
+                                                o32=O32)
+        _, _, _, kept_b, bits_b = mala.mala_bwd(Q, K, V, O, dO, LSE, tau=tau, trace=True, o32=O32)
         _, kept_d, _ = mala.mala_decode(q, Kc, Vc, tau=tau, trace=True)
         mala.mala_check()
         nt = (Dc.Lc + 127) // 128
@@ -395,12 +407,13 @@ def run_mala(args, rank, world, local_rank):
     t1 = timed(1.0, args.steps, args.warmup, clock=clock)
     clocks = clock.stop()
     work1 = trace(1.0)
-    # the backward that recomputes every tile's scores for its test (no row maxima)
-    recompute = timed(1.0, max(1, min(args.steps, 3)), 1, rowmax=False)
-    work1["bwd_recompute_ms"] = recompute["bwd_ms"]
-    work1["fwd_no_rowmax_ms"] = recompute["fwd_ms"]
+    launches, kernels = count_launches(lambda: step(1.0))
+    work1["launches_per_step"] = launches
+    work1["kernels"] = kernels
     dense = timed(0.0, max(1, min(args.steps, 3)), 1) if not args.no_dense else None
     e2e = None if args.no_e2e else run_e2e(args, x, dev, world, max_over_ranks)
+    del Q, K, V, dO, q, Kc, Vc, O, O32, LSE, dQ, dK, dV, o, ws_b, ws_d
+    torch.cuda.empty_cache()
     return t1, work1, dense, clocks, e2e
 
 
@@ -435,10 +448,9 @@ def run_e2e(args, x, dev, world, max_over_ranks):
         q_.copy_(hq, non_blocking=True)
         Kc_.copy_(hKc, non_blocking=True)
         Vc_.copy_(hVc, non_blocking=True)
-        O, LSE, O32, RM = mala.mala_fwd(dQ_["Q"], dQ_["K"], dQ_["V"], tau=1.0, o32=True,
-                                        rowmax=True)
-        dQ, dK, dV = mala.mala_bwd(dQ_["Q"], dQ_["K"], dQ_["V"], O, dQ_["dO"], LSE, tau=1.0, o32=O32,
-                                   rowmax=RM)
+        O, LSE, O32 = mala.mala_fwd(dQ_["Q"], dQ_["K"], dQ_["V"], tau=1.0, o32=True)
+        dQ, dK, dV = mala.mala_bwd(dQ_["Q"], dQ_["K"], dQ_["V"], O, dQ_["dO"], LSE, tau=1.0,
+                                   o32=O32)
         o = mala.mala_decode(q_, Kc_, Vc_, tau=1.0)
         for n, t in (("O", O), ("dQ", dQ), ("dK", dK), ("dV", dV)):
             outs_h[n].copy_(t, non_blocking=True)
@@ -529,12 +541,11 @@ def profile_case(args):
     if args.profile in ("fwd", "bwd"):
         x = synth.prefill_inputs(PREFILL, L=args.L)
         t = {n: torch.tensor(x[n]).to(torch.bfloat16).cuda() for n in ("Q", "K", "V", "dO")}
-        O, LSE, O32, RM = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, o32=True, rowmax=True)
-        run = (lambda: mala.mala_fwd(t["Q"], t["K"], t["V"], tau=1.0, out=O, lse=LSE, o32=O32,
-                                     rowmax=RM)) \
+        tau = args.tau
+        O, LSE, O32 = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, o32=True)
+        run = (lambda: mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, out=O, lse=LSE, o32=O32)) \
             if args.profile == "fwd" else \
-            (lambda: mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=1.0, o32=O32,
-                                   rowmax=RM))
+            (lambda: mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau, o32=O32))
     else:
         cfg = synth.DecodeConfig("profile", 4, 4, DECODE.Hq, DECODE.Hkv, DECODE.Lc, DECODE.d,
                                  128, DECODE.rho, DECODE.n_pairs, DECODE.n_query_targets)
@@ -551,7 +562,7 @@ def profile_case(args):
     e.record()
     torch.cuda.synchronize()
     mala.mala_check()
-    print(json.dumps({"profile": args.profile, "L": args.L,
+    print(json.dumps({"profile": args.profile, "L": args.L, "tau": args.tau,
                       "ms_per_launch": s.elapsed_time(e) / args.launches}), flush=True)
 
 
@@ -618,6 +629,155 @@ def tau_study(args):
                       "decode": {"workload": "decode_128k", "rows": drows}}), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# per-workload report: configurations 0-2 (the tiny float32 case, the
+# matched-work shape and the length sweep), each at tau=1 and tau=0
+# ---------------------------------------------------------------------------
+PER_WORKLOAD = ["tiny_f32", "matched_8k"] + [f"sweep_L{L}" for L in (1024, 2048, 4096, 8192, 16384,
+                                                                       32768)]
+# heads whose keep sets the oracle recomputes (near-threshold flip counts and
+# the oracle's own time on this workload); "fwd" = forward only
+ORACLE_HEADS = {"tiny_f32": (1, "both"), "matched_8k": (8, "both"), "sweep_L1024": (16, "both"),
+                "sweep_L2048": (16, "both"), "sweep_L4096": (16, "both"),
+                "sweep_L8192": (4, "both"), "sweep_L16384": (1, "both"),
+                "sweep_L32768": (1, "fwd")}
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 148 SMs x 128 FP32 FMA/clk at 1965 MHz
+
+
+def workload_oracle(cfg, host, gbits_f, gbits_b, n_heads, which, tau=1.0):
+    """The CPU oracle on ``n_heads`` heads of this workload (the values the GPU
+    sees, rounded on the host): its wall time on this host's cores, and the
+    GPU keep sets compared with its own -- mismatches inside the
+    near-threshold band are counted (both decisions are correct there), any
+    other mismatch is counted separately (it must be 0)."""
+    import mass_adaptive_causal_b200 as mala
+    import oracle
+    sys.path.insert(0, ROOT)
+    from tests.parity import NEAR
+    cores = oracle.threads(len(os.sched_getaffinity(0)))
+    nb = (cfg.L + cfg.tile - 1) // cfg.tile
+    tril = np.tril(np.ones((nb, nb), bool))
+    flips_f = flips_b = other = 0
+    t_cpu = 0.0
+    for h in range(n_heads):
+        Qd, Kd, Vd, dOd = (host[n][0, h] for n in ("Q", "K", "V", "dO"))
+        t0 = time.perf_counter()
+        ref = oracle.fwd(Qd, Kd, Vd, tile=cfg.tile, tau=tau, want_margin=True)
+        g = None
+        if which == "both":
+            g = oracle.bwd(Qd, Kd, Vd, ref["O"], dOd, ref["LSE"], tile=cfg.tile, tau=tau,
+                           want_margin=True)
+        t_cpu += time.perf_counter() - t0
+        gk = mala.unpack_bits(gbits_f[0, h], nb)
+        bad = set()
+        for i in range(nb):
+            for j in range(i, -1, -1):
+                if gk[i, j] != ref["keep"][i, j]:
+                    if abs(ref["margin"][i, j]) <= NEAR:
+                        flips_f += 1
+                    else:
+                        other += 1
+                    bad.add(i)
+                    break  # later tiles of this block follow a different state
+        if g is not None:
+            gb = mala.unpack_bits(gbits_b[0, h], nb)
+            diff = (gb.astype(bool) != g["keep"].astype(bool)) & tril
+            for i, j in zip(*np.nonzero(diff)):
+                if i in bad:
+                    continue
+                if abs(g["margin"][i, j]) <= NEAR:
+                    flips_b += 1
+                else:
+                    other += 1
+    per_head = t_cpu / max(1, n_heads)
+    return {"heads": n_heads, "passes": "fwd+bwd" if which == "both" else "fwd", "cpu_s": t_cpu,
+            "cores": cores, "cpu_s_all_heads_extrapolated": per_head * cfg.B * cfg.H,
+            "near_threshold_flips_fwd": flips_f, "near_threshold_flips_bwd": flips_b,
+            "mismatches_outside_band": other}
+
+
+def per_workload(dev, peaks, oracle_leg=True, reps=5):
+    """Configurations 0-2 on the GPU kernels, each at tau=1 and at tau=0
+    (the in-house dense comparison): ms, effective TFLOP/s and fraction of
+    the roofline, retained slots per query, omitted mass and O/dQ/dK/dV error
+    against tau=0, and (oracle_leg) the oracle's time and the near-threshold
+    flip counts on sampled heads."""
+    import torch
+    import mass_adaptive_causal_b200 as mala
+    out = []
+    for name in PER_WORKLOAD:
+        cfg = synth.CONFIGS[name]
+        x = synth.prefill_inputs(cfg)
+        dt = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
+        host = {n: torch.tensor(x[n]).to(dt) for n in ("Q", "K", "V", "dO")}
+        t = {n: v.to(dev) for n, v in host.items()}
+        res = {"workload": name, "shape": f"B{cfg.B} H{cfg.H} L{cfg.L} d{cfg.d} tile{cfg.tile}",
+               "dtype": "f32" if cfg.dtype == "f32" else "bf16"}
+        d, L = cfg.d, cfg.L
+        P_legal = cfg.B * cfg.H * legal_pairs(L)
+        runs = {}
+        for tau in (1.0, 0.0):
+            o32 = dt == torch.bfloat16
+            O, LSE, kept, bits, *r = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True,
+                                                   o32=o32)
+            O32 = r[0] if o32 else O
+            dQ, dK, dV, kept_b, bits_b = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE,
+                                                       tau=tau, trace=True,
+                                                       o32=O32 if o32 else None)
+            mala.mala_check()
+
+            def ev_time(fn):
+                fn()
+                ts = []
+                for _ in range(reps):
+                    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    s.record()
+                    fn()
+                    e.record()
+                    torch.cuda.synchronize()
+                    ts.append(s.elapsed_time(e))
+                return statistics.median(ts)
+            f_ms = ev_time(lambda: mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, out=O, lse=LSE,
+                                                 o32=O32 if o32 else None))
+            b_ms = ev_time(lambda: mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
+                                                 o32=O32 if o32 else None))
+            fret = retained_pairs(bits, L, cfg.tile)
+            bret = retained_pairs(bits_b, L, cfg.tile)
+            f_fl = 2 * d * P_legal + 2 * d * fret
+            b_fl = 2 * d * P_legal + 8 * d * bret
+            peak = FP32_SIMT_TFLOPS if cfg.dtype == "f32" else peaks["bf16_tflops"]
+            f_tf, b_tf = f_fl / (f_ms * 1e-3) / 1e12, b_fl / (b_ms * 1e-3) / 1e12
+            runs[tau] = {"O": O32.float(), "LSE": LSE.double(), "dQ": dQ.float(), "dK": dK.float(),
+                         "dV": dV.float(), "bits": bits, "bits_b": bits_b}
+            res[f"tau{int(tau)}"] = {
+                "fwd_ms": f_ms, "bwd_ms": b_ms, "fwd_tflops_eff": f_tf, "bwd_tflops_eff": b_tf,
+                "fwd_frac": f_tf / peak, "bwd_frac": b_tf / peak,
+                "peak": "fp32 SIMT nominal" if cfg.dtype == "f32" else "bf16 burst (measured)",
+                "fwd_slots_per_query": fret / (cfg.B * cfg.H * L),
+                "bwd_slots_per_query": bret / (cfg.B * cfg.H * L)}
+        a, z = runs[1.0], runs[0.0]
+        om = (1.0 - torch.exp(a["LSE"] - z["LSE"])).clamp_min(0.0).flatten()
+
+        def rel(n):
+            return float(torch.linalg.norm((a[n] - z[n]).flatten()) /
+                         torch.linalg.norm(z[n].flatten()))
+        res["tau1_vs_tau0"] = {"omitted_mass_mean": float(om.mean()),
+                               "omitted_mass_p95": float(torch.quantile(om.float(), 0.95))
+                               if om.numel() <= 1 << 24 else None,
+                               "omitted_mass_max": float(om.max()), "O_rel_l2": rel("O"),
+                               "dQ_rel_l2": rel("dQ"), "dK_rel_l2": rel("dK"), "dV_rel_l2": rel("dV"),
+                               "fwd_speedup": res["tau0"]["fwd_ms"] / res["tau1"]["fwd_ms"],
+                               "bwd_speedup": res["tau0"]["bwd_ms"] / res["tau1"]["bwd_ms"]}
+        if oracle_leg:
+            nh, which = ORACLE_HEADS[name]
+            hostd = {n: v.double().numpy() for n, v in host.items()}
+            res["oracle"] = workload_oracle(cfg, hostd, a["bits"], a["bits_b"], nh, which)
+        out.append(res)
+        del t, runs, a, z
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -632,6 +792,9 @@ def main():
                     help="run only a small case of one call (for ncu captures)")
     ap.add_argument("--L", type=int, default=32768, help="sequence length of --profile")
     ap.add_argument("--launches", type=int, default=2, help="timed launches of --profile")
+    ap.add_argument("--tau", type=float, default=1.0, help="tau of --profile")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the per-workload report of configurations 0-2")
     ap.add_argument("--study", choices=["tau"], default=None,
                     help="tau sweep: slots, omitted mass and error against dense, one JSON line")
     args = ap.parse_args()
@@ -681,11 +844,10 @@ def main():
     peaks = load_peaks()
     d = P.d
     P_legal = P.B * P.H * legal_pairs(P.L)
+    # effective work: every legal QK plus the retained post-score work
+    # (forward P.V: 2d per retained pair; backward P, dV, dP, dK, dQ: 8d)
     fwd_flop = 2 * d * P_legal + 2 * d * work["fwd_ret"]
-    # with the forward's tile row maxima the backward's test reads 512 bytes per
-    # legal tile and recomputes no score; kept tiles then cost S, dP, dV, dK, dQ
-    bwd_flop = 10 * d * work["bwd_ret"]
-    rm_bytes = 4 * 128 * P.B * P.H * legal_tiles(P.L, P.tile)
+    bwd_flop = 2 * d * P_legal + 8 * d * work["bwd_ret"]
     fwd_tf = fwd_flop / (t1["fwd_ms"] * 1e-3) / 1e12
     bwd_tf = bwd_flop / (t1["bwd_ms"] * 1e-3) / 1e12
     kc_bytes = Dc.B * Dc.Hkv * Dc.Lc * Dc.d * 2
@@ -694,18 +856,23 @@ def main():
     dec_bytes = kc_bytes + 2 * work["decode_kept_tiles"] * tile_bytes + \
         Dc.B * Dc.Hq * (2 * Dc.d * 2 + nt * 8 * 2)
     dec_gbs = dec_bytes / (t1["decode_us"] * 1e-6) / 1e9
-    dominant = "fwd" if t1["fwd_ms"] >= t1["bwd_ms"] else "bwd"
     traffic = load_profile_traffic()
-    if dominant == "fwd":
-        roof = {"bound": "tensor", "kernel": "mala::fwd2::fwd_pair_kernel", "achieved": fwd_tf,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": fwd_tf / peaks["bf16_tflops"],
-                "traffic": traffic.get("fwd_pair_kernel")}
-    else:
-        roof = {"bound": "tensor", "kernel": "mala::bwd100::bwd_bf16_kernel", "achieved": bwd_tf,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": bwd_tf / peaks["bf16_tflops"],
-                "traffic": traffic.get("bwd_bf16_kernel")}
-    roof["peak_source"] = peaks["source"] + " (burst bf16 cuBLAS)"
-    roof["frac_of_sustained"] = roof["achieved"] / (peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"])
+    sus = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
+    src = peaks["source"] + " (burst bf16 cuBLAS)"
+    # the forward is one kernel per call, so its CUDA-event bracket is that
+    # kernel's launch time; the backward call is four kernels, the
+    # recomputing skip test among them, and its bracket covers them all
+    roof = {"bound": "tensor", "kernel": "mala::fwd2::fwd_pair_kernel", "achieved": fwd_tf,
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": fwd_tf / peaks["bf16_tflops"],
+            "traffic": traffic.get("fwd_pair_kernel"), "peak_source": src,
+            "frac_of_sustained": fwd_tf / sus}
+    roof_bwd = {"bound": "tensor", "call": "mala_bwd (row terms, skip test, work pass, dQ convert)",
+                "achieved": bwd_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": bwd_tf / peaks["bf16_tflops"], "traffic": traffic.get("bwd_call"),
+                "peak_source": src, "frac_of_sustained": bwd_tf / sus}
+    roof_dec = {"bound": "hbm", "call": "mala_decode", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
+                "traffic": traffic.get("decode_call")}
 
     line = {
         "metric": "ms per step (fwd+bwd at 128K + one decode step at 128K)",
@@ -715,10 +882,6 @@ def main():
         "config": {"workload": WORKLOAD, "tau": 1.0, "l2": "inputs larger than L2 (no flush)",
                    "parallelism": f"replicas x{world} (independent heads/sequences per rank)"},
         "fwd_ms": t1["fwd_ms"], "bwd_ms": t1["bwd_ms"], "decode_us": t1["decode_us"],
-        "bwd_recompute_ms": work["bwd_recompute_ms"], "fwd_no_rowmax_ms": work["fwd_no_rowmax_ms"],
-        "bwd_recompute_tflops_eff": (2 * d * P_legal + 8 * d * work["bwd_ret"]) /
-        (work["bwd_recompute_ms"] * 1e-3) / 1e12,
-        "rowmax_bytes": rm_bytes,
         "fwd_tflops_eff": fwd_tf, "bwd_tflops_eff": bwd_tf,
         "fwd_frac_bf16": fwd_tf / peaks["bf16_tflops"], "bwd_frac_bf16": bwd_tf / peaks["bf16_tflops"],
         "decode_gbs": dec_gbs, "decode_frac_hbm": dec_gbs / peaks["hbm_gbs"],
@@ -726,9 +889,10 @@ def main():
         "fwd_slots_per_query": work["fwd_ret"] / (P.B * P.H * P.L),
         "bwd_slots_per_query": work["bwd_ret"] / (P.B * P.H * P.L),
         "decode_kept_tile_frac": work["decode_kept_tiles"] / work["decode_tiles"],
-        "roofline": roof,
+        "roofline": roof, "roofline_bwd": roof_bwd, "roofline_decode": roof_dec,
         "clocks": clocks,
-        "gpu_launches": args.steps * (1 + 5 + 4),  # fwd 1; bwd row-dot, zero, test, work, convert; decode 4
+        "gpu_launches": args.steps * work["launches_per_step"],
+        "gpu_launches_per_step": work["launches_per_step"], "kernels": work["kernels"],
     }
     if dense is not None:
         line["dense_tau0"] = {"fwd_ms": dense["fwd_ms"], "bwd_ms": dense["bwd_ms"],
@@ -738,8 +902,14 @@ def main():
                               "decode_speedup": dense["decode_us"] / t1["decode_us"],
                               "fwd_tflops": 4 * d * P_legal / (dense["fwd_ms"] * 1e-3) / 1e12,
                               "bwd_tflops": 10 * d * P_legal / (dense["bwd_ms"] * 1e-3) / 1e12}
+        for k in ("fwd", "bwd"):
+            line["dense_tau0"][k + "_frac_bf16"] = line["dense_tau0"][k + "_tflops"] / peaks["bf16_tflops"]
     if e2e is not None:
         line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_per_workload:
+        import torch
+        line["per_workload"] = per_workload(torch.device("cuda", local_rank), peaks,
+                                            oracle_leg=not args.no_cpu_baseline)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ms, cores, desc = oracle_sample(x, 30.0)
         line["cpu_baseline"] = {"value": ms, "unit": "ms", "cores": cores, "kind": "oracle",

@@ -83,37 +83,24 @@ typedef enum { MALA_F32 = 0, MALA_BF16 = 1 } mala_dtype;
  *         D = <dO, O> feed dQ through a sum over keys whose rows cancel, so
  *         D computed from a bf16-rounded O costs dQ percents of accuracy when
  *         keys share a large common component.
- *         tile_rowmax (may be NULL; MALA_BF16 only; mala_tile_rowmax_bytes
- *         bytes): what the backward's skip test needs from this pass. Part
- *         1, float32 [B][H][i(i+1)/2 + j][tile]: for legal tile (query block
- *         i, key block j <= i) and row r of block i, the largest raw score
- *         q_r . k_c (unscaled) over the tile's keys c <= row. Part 2 (from
- *         the next 256-byte boundary), uint32 [B][H][nb][ceil(nb/32)]: bit j
- *         of row i set iff tile (i, j)'s maxima were stored. They are stored
- *         for every kept tile and for skipped tiles with some row within a
- *         relative 1e-3 of the forward's bound; every other tile fails the
- *         backward's test (the final normalizer only raises the bound), so
- *         its maxima are not needed. Rows past L are unspecified. Pass the
- *         buffer to mala_bwd: its skip test then reads the stored maxima
- *         instead of recomputing every tile's scores.
  * Trace   kept_tiles: [B][H][nb] kept key tiles per query block;
  *         keep_bits: [B][H][nb][ceil(nb/32)], row = query block, bit = key
  *         block. nb = ceil(L / tile).
  * Supported: (dt, d, tile) in {(MALA_BF16, 128, 128), (MALA_F32, 32|64|128, 64)};
  *            any L >= 0 (a ragged last block is masked), B, H >= 1, H % Hkv
- *            == 0 (Hkv < H: MALA_BF16 only); with tile_rowmax, L <= 4194304
- *            (else MALA_ERR_UNSUPPORTED).
+ *            == 0 (Hkv < H: MALA_BF16 only).
+ * Memory: nothing but O, LSE (and O_f32 when given) is written; no score,
+ *         row maximum or selection mask outlives the call.
  */
 mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O,
-                     float* LSE, float* O_f32, float* tile_rowmax, int B, int H,
-                     int Hkv, int L, int d, mala_dtype dt, float tau, int tile,
-                     float scale, int32_t* kept_tiles, uint32_t* keep_bits,
-                     void* stream);
+                     float* LSE, float* O_f32, int B, int H, int Hkv, int L,
+                     int d, mala_dtype dt, float tau, int tile, float scale,
+                     int32_t* kept_tiles, uint32_t* keep_bits, void* stream);
 
 /*
- * Prefill of chunks appended to KV caches, several sequences packed
- * (SURVEY's next row "varlen prefill": prefill uses the same tau;
- * agihunt.info summary, "one tau for prefill and decode").
+ * Prefill of chunks appended to KV caches, several sequences packed (prefill
+ * and decode use the same tau: agihunt.info summary, "one tau for prefill and
+ * decode").
  *
  * Sequence b's new queries are tokens [cu_seqlens_q[b], cu_seqlens_q[b+1])
  * of Q; its keys and values, cached ones first, are tokens
@@ -150,13 +137,6 @@ mala_status mala_fwd_varlen(const void* Q, const void* K, const void* V, void* O
 /* 32-bit words per query block in mala_fwd_varlen's keep_bits. */
 int mala_varlen_trace_words(int max_seqlen_q, int max_seqlen_k);
 
-/* Bytes of the forward's optional tile_rowmax output: B * H * nb(nb+1)/2 *
- * tile * 4 (maxima) plus B * H * nb * ceil(nb/32) * 4 (flags), each rounded
- * up to 256, for nb = ceil(L / tile): 2 GiB for B = 1, H = 8, L = 131072,
- * tile = 128, of which the forward writes only the flagged tiles (a few
- * percent when most tiles are skipped). 0 for invalid sizes. */
-size_t mala_tile_rowmax_bytes(int B, int H, int L, int tile);
-
 /* Bytes of device workspace mala_bwd needs: the row terms D (float32
  * [B][H][L]), the float32 dQ accumulator [B][H][L][d] and the per-tile keep
  * bits of the backward's test pass (B*H*nb*ceil(nb/32) words for nb =
@@ -167,12 +147,12 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
  * Backward pass.
  *
  * Uses the forward's final LSE instead of replaying its partial normalizers.
- * Tile (i, j) is skipped iff every valid row r satisfies
+ * Every legal tile's scores are recomputed, and tile (i, j) is skipped iff
+ * every valid row r satisfies
  *     max_c S_rc - LSE_r  <  ln tau - ln (r + 1).
- * The row maxima come from tile_rowmax when given (the forward recorded them
- * from the same scores), else every legal tile's scores are recomputed;
- * both give the same decisions. There is no forced keep and no stored mask;
- * in exact arithmetic the kept set is inside the forward's. Kept tiles do the standard work with
+ * Only O and LSE (or O_f32) come from the forward: no mask, score or row
+ * maximum is carried between the passes, and there is no forced keep. In
+ * exact arithmetic the kept set is inside the forward's. Kept tiles do the standard work with
  * P = exp(S - LSE), D_r = <dO_r, O_r>: dV_j += P^T dO_i, dP = dO_i V_j^T,
  * dS = P o (dP - D), dQ_i += scale dS K_j, dK_j += scale dS^T Q_i.
  * Sources: agihunt.info summary, backward paragraph; jaehun.me review,
@@ -181,9 +161,7 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
  * Inputs  Q, O, dO: [B][H][L][d], K, V: [B][Hkv][L][d] of dtype dt (grouped
  *         heads as in mala_fwd); LSE from mala_fwd;
  *         O_f32 (may be NULL): the float32 output of mala_fwd, used for the
- *         row terms D instead of O when given;
- *         tile_rowmax (may be NULL; MALA_BF16 only): the forward's tile row
- *         maxima for the same Q, K (read only when tau > 0).
+ *         row terms D instead of O when given.
  * Outputs dQ: [B][H][L][d]; dK, dV: [B][Hkv][L][d], summed over the query
  *         heads of each group; dtype dt (fully overwritten).
  * workspace: device buffer of at least mala_bwd_workspace_bytes(B,H,L,d)
@@ -195,8 +173,8 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
  */
 mala_status mala_bwd(const void* Q, const void* K, const void* V,
                      const void* O, const float* O_f32, const void* dO,
-                     const float* LSE, const float* tile_rowmax, void* dQ,
-                     void* dK, void* dV, void* workspace,
+                     const float* LSE, void* dQ, void* dK, void* dV,
+                     void* workspace,
                      size_t workspace_bytes, int B, int H, int Hkv, int L, int d,
                      mala_dtype dt, float tau, int tile, float scale,
                      int32_t* kept_tiles, uint32_t* keep_bits, void* stream);
@@ -254,8 +232,10 @@ mala_status mala_decode(const void* q, const void* Kcache, const void* Vcache,
  * Scratch: a file-scope __device__ array of MALA_DECODE_NOALLOC_SCRATCH_BYTES
  * bytes inside this library. Every GPU that loads the library holds it until
  * the process exits. The first call on a device, with that device current,
- * looks up the array's device address (cudaGetSymbolAddress) and caches it;
- * make that first call before any stream capture begins. The call itself
+ * looks up the array's device address (cudaGetSymbolAddress) and caches it
+ * with the unique ID of the current context; a call in another context of
+ * that device (after cudaDeviceReset, say) looks it up again. Make the first
+ * call in a context before any stream capture begins. The call itself
  * allocates nothing: no cudaMalloc, no cudaFree, no allocating library
  * routine.
  *

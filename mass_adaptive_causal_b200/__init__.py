@@ -50,19 +50,17 @@ def lib() -> ctypes.CDLL:
                 " (or __graft_entry__.build())")
         L = ctypes.CDLL(LIB_PATH)
         ci, cf, cs = ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-        L.mala_fwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _fp, _fp, ci, ci, ci, ci, ci, ci, cf, ci, cf,
+        L.mala_fwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _fp, ci, ci, ci, ci, ci, ci, cf, ci, cf,
                                _i32p, _u32p, _vp]
         L.mala_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _vp, ci, ci, ci, ci, ci, ci,
                                       ci, ci, cf, ci, cf, _i32p, _u32p, _vp]
         L.mala_fwd_varlen.restype = ci
         L.mala_varlen_trace_words.argtypes = [ci, ci]
         L.mala_varlen_trace_words.restype = ci
-        L.mala_tile_rowmax_bytes.argtypes = [ci, ci, ci, ci]
-        L.mala_tile_rowmax_bytes.restype = cs
         L.mala_fwd.restype = ci
         L.mala_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
         L.mala_bwd_workspace_bytes.restype = cs
-        L.mala_bwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _fp, _fp, _vp, _vp, _vp, _vp, cs, ci, ci,
+        L.mala_bwd.argtypes = [_vp, _vp, _vp, _vp, _fp, _vp, _fp, _vp, _vp, _vp, _vp, cs, ci, ci,
                                ci, ci, ci, ci, cf, ci, cf, _i32p, _u32p, _vp]
         L.mala_bwd.restype = ci
         L.mala_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
@@ -161,7 +159,7 @@ def _check_prefill(q, k, v, *rest, require_cuda=True):
     return torch
 
 
-def _check_fwd_buffers(q, tile, out=None, lse=None, o32=None, rowmax=None):
+def _check_fwd_buffers(q, out=None, lse=None, o32=None):
     torch = _torch()
     B, H, L, _ = q.shape
     if out is not None:
@@ -170,20 +168,14 @@ def _check_fwd_buffers(q, tile, out=None, lse=None, o32=None, rowmax=None):
         _buf(lse, "lse", q.device, torch.float32, (B, H, L))
     if o32 is not None:
         _buf(o32, "o32", q.device, torch.float32, q.shape)
-    if rowmax is not None:
-        _buf(rowmax, "rowmax", q.device, torch.float32,
-             min_bytes=tile_rowmax_bytes(B, H, L, tile))
 
 
-def _check_bwd_buffers(q, k, lse, tile, o32=None, rowmax=None, grads=None, workspace=None):
+def _check_bwd_buffers(q, k, lse, o32=None, grads=None, workspace=None):
     torch = _torch()
     B, H, L, _ = q.shape
     _buf(lse, "lse", q.device, torch.float32, (B, H, L))
     if o32 is not None:
         _buf(o32, "o32", q.device, torch.float32, q.shape)
-    if rowmax is not None:
-        _buf(rowmax, "rowmax", q.device, torch.float32,
-             min_bytes=tile_rowmax_bytes(B, H, L, tile))
     if grads is not None:
         dq, dk, dv = grads
         _buf(dq, "dQ", q.device, q.dtype, q.shape)
@@ -245,21 +237,14 @@ def n_blocks(L: int, tile: int) -> int:
     return (L + tile - 1) // tile
 
 
-def tile_rowmax_bytes(B, H, L, tile=128) -> int:
-    return int(lib().mala_tile_rowmax_bytes(B, H, L, tile))
-
-
 def mala_fwd(q, k, v, tau: float = 1.0, tile: int | None = None, scale: float = 0.0,
-             trace: bool = False, out=None, lse=None, o32=None, rowmax=None, stream=None):
+             trace: bool = False, out=None, lse=None, o32=None, stream=None):
     """Forward pass. q, k, v: [B, H, L, d] (bf16 with d = 128, or float32).
 
     Returns (O, LSE) or, with ``trace=True``, (O, LSE, kept_tiles, keep_bits)
     where kept_tiles is int32 [B, H, nb] and keep_bits int32 [B, H, nb, nw].
     ``o32=True`` (or a float32 tensor shaped like q) also writes the float32
-    output and appends it to the returned tuple (pass it to mala_bwd).
-    ``rowmax=True`` (or a float32 tensor of tile_rowmax_bytes / 4 elements)
-    also records every legal tile's row score maxima and appends them last
-    (pass them to mala_bwd to spare its score recomputation; bf16 only)."""
+    output and appends it to the returned tuple (pass it to mala_bwd)."""
     torch = _check_prefill(q, k, v)
     B, H, L, d = q.shape
     tile = default_tile(q.dtype) if tile is None else tile
@@ -270,26 +255,18 @@ def mala_fwd(q, k, v, tau: float = 1.0, tile: int | None = None, scale: float = 
         o32_t = torch.empty(q.shape, dtype=torch.float32, device=q.device)
     elif o32 is not None and o32 is not False:
         o32_t = o32
-    rm_t = None
-    if rowmax is True:
-        rm_t = torch.empty(tile_rowmax_bytes(B, H, L, tile) // 4, dtype=torch.float32,
-                           device=q.device)
-    elif rowmax is not None and rowmax is not False:
-        rm_t = rowmax
-    _check_fwd_buffers(q, tile, out=o, lse=lse_t, o32=o32_t, rowmax=rm_t)
+    _check_fwd_buffers(q, out=o, lse=lse_t, o32=o32_t)
     kept = bits = None
     if trace:
         nb = n_blocks(L, tile)
         kept = torch.empty((B, H, nb), dtype=torch.int32, device=q.device)
         bits = torch.empty((B, H, nb, (nb + 31) // 32), dtype=torch.int32, device=q.device)
-    code = lib().mala_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), _ptr(o32_t),
-                          _ptr(rm_t), B, H, k.shape[1], L, d, _dtype_code(q), float(tau), int(tile),
-                          float(scale), _ptr(kept), _ptr(bits), _stream(stream))
+    code = lib().mala_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), _ptr(o32_t), B, H,
+                          k.shape[1], L, d, _dtype_code(q), float(tau), int(tile), float(scale),
+                          _ptr(kept), _ptr(bits), _stream(stream))
     _raise(code, "mala_fwd")
     res = (o, lse_t, kept, bits) if trace else (o, lse_t)
-    if o32_t is not None:
-        res = res + (o32_t,)
-    return res + (rm_t,) if rm_t is not None else res
+    return res + (o32_t,) if o32_t is not None else res
 
 
 def mala_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
@@ -327,12 +304,11 @@ def bwd_workspace_bytes(B, H, L, d) -> int:
 
 def mala_bwd(q, k, v, o, do, lse, tau: float = 1.0, tile: int | None = None,
              scale: float = 0.0, trace: bool = False, workspace=None, grads=None, o32=None,
-             rowmax=None, stream=None):
+             stream=None):
     """Backward pass. Returns (dQ, dK, dV) or, with ``trace=True``,
     (dQ, dK, dV, kept_tiles [B, H, nb] per key block, keep_bits [B, H, nb, nw]).
     ``o32``: the float32 forward output (recommended for bf16), used for the
-    row terms D = <dO, O>. ``rowmax``: the forward's tile row maxima; the skip
-    test then reads them instead of recomputing every tile's scores."""
+    row terms D = <dO, O>. Only O (or o32) and lse come from the forward."""
     torch = _check_prefill(q, k, v, o, do)
     B, H, L, d = q.shape
     tile = default_tile(q.dtype) if tile is None else tile
@@ -348,10 +324,9 @@ def mala_bwd(q, k, v, o, do, lse, tau: float = 1.0, tile: int | None = None,
         nb = n_blocks(L, tile)
         kept = torch.empty((B, H, nb), dtype=torch.int32, device=q.device)
         bits = torch.empty((B, H, nb, (nb + 31) // 32), dtype=torch.int32, device=q.device)
-    _check_bwd_buffers(q, k, lse, tile, o32=o32, rowmax=rowmax, grads=(dq, dk, dv),
-                       workspace=ws)
+    _check_bwd_buffers(q, k, lse, o32=o32, grads=(dq, dk, dv), workspace=ws)
     code = lib().mala_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(o32), _ptr(do), _ptr(lse),
-                          _ptr(rowmax), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                          _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
                           ws.numel() * ws.element_size(), B, H,
                           k.shape[1], L, d, _dtype_code(q),
                           float(tau), int(tile), float(scale), _ptr(kept), _ptr(bits),

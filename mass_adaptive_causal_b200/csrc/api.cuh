@@ -24,26 +24,6 @@ namespace host {
     if (e_ != cudaSuccess) return MALA_ERR_CUDA; \
   } while (0)
 
-// The backward's row-maximum test keeps one query block's bits in 4 KB of
-// shared memory: nb <= 32768 blocks of 128 rows.
-constexpr int kMaxRowmaxL = 32768 * 128;
-
-// The forward's tile row maxima buffer: the maxima [Z][nb(nb+1)/2][tile]
-// float32, then one flag bit per tile [Z][nb][ceil(nb/32)] saying which
-// tiles' maxima were stored, each part rounded up to 256 bytes.
-inline size_t rowmax_maxima_bytes(size_t Z, size_t L, size_t tile) {
-  const size_t nb = (L + tile - 1) / tile;
-  return (Z * (nb * (nb + 1) / 2) * tile * sizeof(float) + 255) & ~size_t(255);
-}
-inline size_t rowmax_flag_bytes(size_t Z, size_t L, size_t tile) {
-  const size_t nb = (L + tile - 1) / tile;
-  return (Z * nb * ((nb + 31) / 32) * sizeof(uint32_t) + 255) & ~size_t(255);
-}
-inline uint32_t* rowmax_flags(const float* rowmax, size_t Z, size_t L, size_t tile) {
-  return reinterpret_cast<uint32_t*>(
-      const_cast<char*>(reinterpret_cast<const char*>(rowmax)) + rowmax_maxima_bytes(Z, L, tile));
-}
-
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline bool tau_ok(float tau) { return isfinite(tau) && tau >= 0.f; }
@@ -151,8 +131,8 @@ inline int varlen_trace_words(int max_q, int max_k) {
 }
 
 inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O, float* LSE,
-                            float* O32, float* rowmax, int B, int Hq, int Hkv, int L, float scale,
-                            float tau, int32_t* kept, uint32_t* bits, cudaStream_t s) {
+                            float* O32, int B, int Hq, int Hkv, int L, float scale, float tau,
+                            int32_t* kept, uint32_t* bits, cudaStream_t s) {
   const int Z = B * Hq, Zkv = B * Hkv;
   // Q and V in 128-row boxes; K in 64-row boxes (each CTA of a pair loads
   // half of every key tile)
@@ -171,8 +151,6 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
   p.log2_tau = tau > 0.f ? log2f(tau) : 0.f;
   p.kept_tiles = kept;
   p.keep_bits = bits;
-  p.rowmax = rowmax;
-  p.rm_bits = rowmax ? rowmax_flags(rowmax, Z, L, fwd2::T) : nullptr;
   p.Hq = Hq;
   p.G = Hq / Hkv;
   return launch_pair<false>(mq, mk, mv, p, p.npairs, Z, s);
@@ -315,7 +293,7 @@ inline mala_status bwd_f32(const float* Q, const float* K, const float* V, const
 }
 
 inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const void* dO,
-                            const float* LSE, const float* rowmax, BwdWorkspace w, void* dQ,
+                            const float* LSE, BwdWorkspace w, void* dQ,
                             void* dK, void* dV, int B, int Hq, int Hkv, int L, float scale,
                             float tau,
                             int32_t* kept, uint32_t* bits, cudaStream_t s) {
@@ -339,16 +317,11 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
     tp.scale_log2 = scale * kLog2e;
     tp.log2_tau = log2f(tau);
     tp.bits = tile_bits;
-    if (rowmax) {  // from the forward's recorded tile row maxima
-      bwdtest::rowmax_test_kernel<<<dim3(nb, Z), bwdtest::RM_NT, 0, s>>>(
-          rowmax, rowmax_flags(rowmax, Z, L, bwd100::T), tp);
-    } else {       // recompute every tile's scores
-      MALA_CUDA_TRY(cudaFuncSetAttribute(bwdtest::test_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)bwdtest::SMEM_BYTES));
-      bwdtest::test_kernel<<<dim3(tp.npairs, Z), bwdtest::NT, bwdtest::SMEM_BYTES, s>>>(mq, mk,
-                                                                                        tp);
-    }
+    // every legal tile's scores are recomputed against the final LSE
+    MALA_CUDA_TRY(cudaFuncSetAttribute(bwdtest::test_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bwdtest::SMEM_BYTES));
+    bwdtest::test_kernel<<<dim3(tp.npairs, Z), bwdtest::NT, bwdtest::SMEM_BYTES, s>>>(mq, mk, tp);
   } else if (bits) {
     const size_t nwords = (size_t)Z * nb * ((nb + 31) / 32);
     aux::lower_bits_kernel<<<blocks_for(nwords, 256, 4 * sm_count()), 256, 0, s>>>(bits, nb,
@@ -534,23 +507,16 @@ static mala_status check_prefill_shape(int B, int H, int Hkv, int L, int d, mala
   return MALA_OK;
 }
 
-size_t mala_tile_rowmax_bytes(int B, int H, int L, int tile) {
-  if (B < 1 || H < 1 || L < 0 || tile < 1) return 0;
-  return rowmax_maxima_bytes((size_t)B * H, L, tile) + rowmax_flag_bytes((size_t)B * H, L, tile);
-}
-
 mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE,
-                     float* O_f32, float* tile_rowmax, int B, int H, int Hkv, int L, int d,
-                     mala_dtype dt, float tau, int tile, float scale, int32_t* kept_tiles,
-                     uint32_t* keep_bits, void* stream) {
+                     float* O_f32, int B, int H, int Hkv, int L, int d, mala_dtype dt, float tau,
+                     int tile, float scale, int32_t* kept_tiles, uint32_t* keep_bits,
+                     void* stream) {
   mala_status st = check_prefill_shape(B, H, Hkv, L, d, dt, tau, tile);
   if (st != MALA_OK) return st;
-  if (tile_rowmax && dt != MALA_BF16) return MALA_ERR_UNSUPPORTED;
-  if (tile_rowmax && L > kMaxRowmaxL) return MALA_ERR_UNSUPPORTED;
   if (L == 0) return MALA_OK;
   if (!Q || !K || !V || !O || !LSE) return MALA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) ||
-      !aligned16(O_f32) || !aligned16(tile_rowmax))
+      !aligned16(O_f32))
     return MALA_ERR_INVALID_ARG;
   const int Z = B * H;
   const float sc = resolve_scale(scale, d);
@@ -564,8 +530,7 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
                                     cudaMemcpyDeviceToDevice, s));
     return st;
   }
-  return fwd_bf16(Q, K, V, O, LSE, O_f32, tile_rowmax, B, H, Hkv, L, sc, tau, kept_tiles,
-                  keep_bits, s);
+  return fwd_bf16(Q, K, V, O, LSE, O_f32, B, H, Hkv, L, sc, tau, kept_tiles, keep_bits, s);
 }
 
 mala_status mala_fwd_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
@@ -602,16 +567,12 @@ size_t mala_bwd_workspace_bytes(int B, int H, int L, int d) {
 }
 
 mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
-                     const float* O_f32, const void* dO, const float* LSE,
-                     const float* tile_rowmax, void* dQ, void* dK, void* dV, void* workspace,
-                     size_t workspace_bytes, int B, int H, int Hkv, int L, int d, mala_dtype dt,
-                     float tau, int tile, float scale, int32_t* kept_tiles, uint32_t* keep_bits,
-                     void* stream) {
+                     const float* O_f32, const void* dO, const float* LSE, void* dQ, void* dK,
+                     void* dV, void* workspace, size_t workspace_bytes, int B, int H, int Hkv,
+                     int L, int d, mala_dtype dt, float tau, int tile, float scale,
+                     int32_t* kept_tiles, uint32_t* keep_bits, void* stream) {
   mala_status st = check_prefill_shape(B, H, Hkv, L, d, dt, tau, tile);
   if (st != MALA_OK) return st;
-  if (tile_rowmax && dt != MALA_BF16) return MALA_ERR_UNSUPPORTED;
-  if (tile_rowmax && L > kMaxRowmaxL) return MALA_ERR_UNSUPPORTED;
-  if (!aligned16(tile_rowmax)) return MALA_ERR_INVALID_ARG;
   if (L == 0) return MALA_OK;
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace)
     return MALA_ERR_INVALID_ARG;
@@ -633,8 +594,8 @@ mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
                    reinterpret_cast<const float*>(V), reinterpret_cast<const float*>(dO), LSE, w,
                    reinterpret_cast<float*>(dQ), reinterpret_cast<float*>(dK),
                    reinterpret_cast<float*>(dV), Z, L, d, sc, tau, kept_tiles, keep_bits, s);
-  return bwd_bf16(Q, K, V, dO, LSE, tile_rowmax, w, dQ, dK, dV, B, H, Hkv, L, sc, tau,
-                  kept_tiles, keep_bits, s);
+  return bwd_bf16(Q, K, V, dO, LSE, w, dQ, dK, dV, B, H, Hkv, L, sc, tau, kept_tiles, keep_bits,
+                  s);
 }
 
 size_t mala_decode_workspace_bytes(int B, int Hq, int Hkv, int Lc, int d) {

@@ -236,51 +236,5 @@ __global__ void __launch_bounds__(NT, 1)
   }
 }
 
-// The same test from the tile row maxima the forward recorded
-// (rowmax[z][i(i+1)/2 + j][r], raw scores), for the tiles it flagged in
-// rm_bits; an unflagged tile is one the forward skipped with every row below
-// its bound by a margin, which the final log-normalizer can only widen, so
-// its bit is 0. No score is recomputed. CTA = query block i (largest first);
-// the flagged tiles are dealt out to the warps in turn; lane l holds the
-// bounds of rows 4l .. 4l+3 and reads their four maxima as one float4.
-constexpr int RM_NT = 256;
-
-__global__ void __launch_bounds__(RM_NT)
-    rowmax_test_kernel(const float* __restrict__ rowmax, const uint32_t* __restrict__ rm_bits,
-                       const Params p) {
-  __shared__ uint32_t words[1024];  // keep bits of this query block (nb <= 32768)
-  const int i = p.nb - 1 - (int)blockIdx.x;
-  const int z = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nw = (p.nb + 31) >> 5;
-  for (int w = tid; w < nw; w += RM_NT) words[w] = 0u;
-  float c[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e)
-    c[e] = bwd_keep_bound_raw(p.LSE, (size_t)z * p.L, i * T + 4 * lane + e, p.L, p.log2_tau,
-                              p.scale_log2);
-  __syncthreads();
-  const size_t ntri = (size_t)p.nb * (p.nb + 1) / 2;
-  const float4* src = reinterpret_cast<const float4*>(
-      rowmax + ((size_t)z * ntri + (size_t)i * (i + 1) / 2) * T) + lane;
-  const uint32_t* flags = rm_bits + ((size_t)z * p.nb + i) * nw;
-  constexpr int NWARP = RM_NT / 32;
-  int k = 0;  // running index of flagged tiles; warp (k % NWARP) takes tile k
-  for (int w = 0; w <= (i >> 5); ++w) {
-    uint32_t word = flags[w];
-    while (word) {
-      const int j = (w << 5) + __ffs(word) - 1;
-      word &= word - 1;
-      if ((k++ % NWARP) != warp || j > i) continue;
-      const float4 m = __ldcs(src + (size_t)j * (T / 4));
-      const bool want = m.x >= c[0] || m.y >= c[1] || m.z >= c[2] || m.w >= c[3];
-      if (__any_sync(0xffffffffu, want) && lane == 0) atomicOr(&words[j >> 5], 1u << (j & 31));
-    }
-  }
-  __syncthreads();
-  uint32_t* out = p.bits + ((size_t)z * p.nb + i) * nw;
-  for (int w = tid; w < nw; w += RM_NT) out[w] = words[w];
-}
-
 }  // namespace bwdtest
 }  // namespace mala

@@ -72,7 +72,6 @@ constexpr uint32_t TMEM_O = 384;
 constexpr uint32_t IDESC_QK = idesc_bf16(256, 128, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(256, 128, false, true);
 constexpr float kRescaleLog2 = 8.f;  // lazy O rescale threshold (log2 units)
-constexpr float kNearSkip = 1e-3f;   // see the row maxima below
 
 struct Params {
   __nv_bfloat16* O;
@@ -86,16 +85,6 @@ struct Params {
   int never_skip;
   int32_t* kept_tiles;
   uint32_t* keep_bits;
-  // optional, for the backward's test: raw score maxima of every row,
-  // [Z][i(i+1)/2 + j][T], written only for the tiles whose maxima can decide
-  // that test and flagged in rm_bits [Z][nb][ceil(nb/32)]. The backward
-  // keeps a tile iff some row's maximum reaches the bound set by the final
-  // log-normalizer, which is never below the partial one tested here; a tile
-  // skipped with every row below its bound by more than kNearSkip (relative)
-  // fails the backward's test too whatever the rounding of either bound, so
-  // only kept tiles and tiles skipped by less are stored.
-  float* rowmax;
-  uint32_t* rm_bits;
   int Hq, G;  // query heads; G query heads share each key/value head
   // Chunks appended to a KV cache, packed (the VARLEN instantiation):
   // sequence b's queries are tokens [cu_q[b], cu_q[b+1]) of Q [total_q][Hq][d],
@@ -419,19 +408,10 @@ __global__ void __launch_bounds__(NT, 1)
     // trace row of this block: bit k of word k / 32 = key tile k kept
     const int nw = VARLEN ? p.nw : (nb + 31) >> 5;
     const size_t brow = (size_t)z * (VARLEN ? p.nbq_max : nb) + iX;
-    KeepBits kb, kbs;
+    KeepBits kb;
     kb.init(r == 0 && mine ? p.keep_bits : nullptr, brow * nw);
-    kbs.init(r == 0 && mine && !VARLEN ? p.rm_bits : nullptr, brow * nw);
-    if (r == 0 && mine) {
-      for (int w = (iX + koff) / 32 + 1; w < nw; ++w) {
-        if (p.keep_bits) p.keep_bits[brow * nw + w] = 0u;
-        if (p.rm_bits && !VARLEN) p.rm_bits[brow * nw + w] = 0u;
-      }
-    }
-    float* rm = (p.rowmax && mine && !VARLEN)
-                    ? p.rowmax + ((size_t)z * ((size_t)nb * (nb + 1) / 2) +
-                                  (size_t)iX * (iX + 1) / 2) * T + r
-                    : nullptr;
+    if (r == 0 && mine && p.keep_bits)
+      for (int w = (iX + koff) / 32 + 1; w < nw; ++w) p.keep_bits[brow * nw + w] = 0u;
     softmax_sync();  // O zeroed by every thread before any decision leaves
 
     for (int t = 0; t < ntiles; ++t) {
@@ -459,13 +439,6 @@ __global__ void __launch_bounds__(NT, 1)
       kb.set(j, keep != 0);
       if (!keep) {
         if (r == 0) signal(u, 0);
-        if (rm) {  // after the decision, off the issuers' path
-          const bool near =
-              row_valid && mraw >= bound_raw - kNearSkip * (1.f + fabsf(bound_raw));
-          const int store = vote_or(near);
-          if (store) rm[(size_t)j * T] = mraw;
-          kbs.set(j, store != 0);
-        }
         continue;
       }
       // ---- kept tile ------------------------------------------------------
@@ -524,13 +497,8 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_before();
       softmax_sync();  // every row's P and O rescale are in TMEM
       if (r == 0) signal(u, 1);
-      if (rm) {
-        rm[(size_t)j * T] = mraw;
-        kbs.set(j, true);
-      }
     }
     kb.flush();
-    kbs.flush();
     if (mine && n_kept > 0) {
       // ---- epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2 -----------------
       mbar_wait(smem_u32(&bars.pv_done), (n_kept - 1) & 1, abort, 0x21b);

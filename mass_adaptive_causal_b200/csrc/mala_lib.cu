@@ -17,21 +17,60 @@ static __device__ __align__(256) unsigned char g_decode_scratch[MALA_DECODE_NOAL
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
-unsigned char* g_scratch_ptr[kMaxDevices];  // device address per device, once found
+// Per device: the array's device address and the unique ID of the context it
+// belongs to. A context destroyed and created again (cudaDeviceReset, or a
+// driver-API user replacing the current context) gets a new ID, so an address
+// from an earlier context is never reused.
+struct ScratchSlot {
+  unsigned long long ctx_id;
+  unsigned char* ptr;
+};
+ScratchSlot g_scratch[kMaxDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(ptr);
+}
+
+// The unique ID of the context current on this thread (0 if none yet).
+bool current_context_id(unsigned long long* id) {
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return false;
+  *id = 0;
+  return !ctx || get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 // In host code `g_decode_scratch` only names the array; its address on the
-// current device comes from the runtime, once per device, and is cached.
+// current device comes from the runtime, once per device and context, and is
+// cached.
 mala_status scratch_on_current_device(unsigned char** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MALA_ERR_CUDA;
+  unsigned long long id = 0;
+  if (!current_context_id(&id)) return MALA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
+  ScratchSlot& slot = g_scratch[dev];
+  if (id == 0 || slot.ptr == nullptr || slot.ctx_id != id) {
+    // the lookup makes the device's primary context current when none is
     unsigned char* ptr = nullptr;
     if (cudaGetSymbolAddress((void**)&ptr, g_decode_scratch) != cudaSuccess || !ptr)
       return MALA_ERR_CUDA;
-    g_scratch_ptr[dev] = ptr;
+    if (id == 0 && (!current_context_id(&id) || id == 0)) return MALA_ERR_CUDA;
+    slot.ptr = ptr;
+    slot.ctx_id = id;
   }
-  *out = g_scratch_ptr[dev];
+  *out = slot.ptr;
   return MALA_OK;
 }
 

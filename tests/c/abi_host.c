@@ -18,37 +18,31 @@
     }                                                              \
   } while (0)
 
-static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
-
 int main(void) {
   /* any 16-byte-aligned address: argument checks never dereference it */
   void* p = (void*)(uintptr_t)256;
   float* f = (float*)p;
-  const size_t nb = (1000 + 127) / 128;
 
   CHECK(mala_version() >= 100);
   CHECK(strcmp(mala_status_string(MALA_OK), "MALA_OK") == 0);
   CHECK(strcmp(mala_status_string(MALA_ERR_TOO_LARGE), "MALA_ERR_TOO_LARGE") == 0);
 
-  CHECK(mala_tile_rowmax_bytes(2, 3, 1000, 128) ==
-        round256(2 * 3 * nb * (nb + 1) / 2 * 128 * 4) + round256(2 * 3 * nb * ((nb + 31) / 32) * 4));
-  CHECK(mala_tile_rowmax_bytes(0, 1, 10, 128) == 0);
   CHECK(mala_bwd_workspace_bytes(1, 2, 1000, 128) > 0);
   CHECK(mala_decode_workspace_bytes(2, 8, 2, 1000, 128) > 0);
   CHECK(mala_varlen_trace_words(4096, 131072) == (32 + 1024 + 31) / 32);
 
-  CHECK(mala_fwd(p, p, p, p, f, NULL, NULL, 1, 1, 1, 256, 128, MALA_BF16, -1.0f, 128, 0.0f,
+  CHECK(mala_fwd(p, p, p, p, f, NULL, 1, 1, 1, 256, 128, MALA_BF16, -1.0f, 128, 0.0f,
                  NULL, NULL, NULL) == MALA_ERR_INVALID_ARG);
-  CHECK(mala_fwd(NULL, p, p, p, f, NULL, NULL, 1, 1, 1, 256, 128, MALA_BF16, 1.0f, 128, 0.0f,
+  CHECK(mala_fwd(NULL, p, p, p, f, NULL, 1, 1, 1, 256, 128, MALA_BF16, 1.0f, 128, 0.0f,
                  NULL, NULL, NULL) == MALA_ERR_INVALID_ARG);
-  CHECK(mala_fwd(p, p, p, p, f, NULL, NULL, 1, 1, 1, 256, 64, MALA_BF16, 1.0f, 128, 0.0f, NULL,
+  CHECK(mala_fwd(p, p, p, p, f, NULL, 1, 1, 1, 256, 64, MALA_BF16, 1.0f, 128, 0.0f, NULL,
                  NULL, NULL) == MALA_ERR_UNSUPPORTED);
-  CHECK(mala_fwd(p, p, p, p, f, NULL, NULL, 1, 4, 3, 256, 128, MALA_BF16, 1.0f, 128, 0.0f, NULL,
+  CHECK(mala_fwd(p, p, p, p, f, NULL, 1, 4, 3, 256, 128, MALA_BF16, 1.0f, 128, 0.0f, NULL,
                  NULL, NULL) == MALA_ERR_INVALID_ARG);
-  CHECK(mala_fwd(p, p, p, p, f, NULL, NULL, 1, 1, 1, 0, 128, MALA_BF16, 1.0f, 128, 0.0f, NULL,
+  CHECK(mala_fwd(p, p, p, p, f, NULL, 1, 1, 1, 0, 128, MALA_BF16, 1.0f, 128, 0.0f, NULL,
                  NULL, NULL) == MALA_OK);
 
-  CHECK(mala_bwd(p, p, p, p, NULL, p, f, NULL, p, p, p, p, 0, 1, 2, 2, 1000, 128, MALA_BF16,
+  CHECK(mala_bwd(p, p, p, p, NULL, p, f, p, p, p, p, 0, 1, 2, 2, 1000, 128, MALA_BF16,
                  1.0f, 128, 0.0f, NULL, NULL, NULL) == MALA_ERR_INVALID_ARG);
 
   CHECK(mala_decode(p, p, p, p, 2, 8, 3, 1000, 128, 1.0f, 0.0f, 0, p, 1 << 30, NULL, NULL,

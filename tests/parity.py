@@ -6,8 +6,14 @@ Tolerances (relative L2 over the compared tensor):
 Keep decisions must match exactly, except tiles whose contribution ratio is
 within 1e-3 relative of the threshold (|margin| <= ln(1 + 1e-3)) and, in the
 forward, the later tiles of the same query block after such a flip (their
-state differs). Rows of query blocks with an allowed flip are left out of the
-element comparison and counted.
+state differs). Such flips are counted and reported. Both decisions are
+correct there, so only what the flip does not touch is compared:
+  forward flip in query block i   -> O, LSE rows of block i; dQ rows of block
+                                     i; dK, dV rows of every key block that
+                                     block i keeps in the backward (either
+                                     side), since their sums include rows of i;
+  backward flip of tile (i, j)    -> dQ rows of block i, dK, dV rows of block j.
+Every other row is compared, and the callers assert how many were.
 """
 
 from __future__ import annotations
@@ -54,16 +60,65 @@ def compare_fwd_keep(gpu_keep, ref_keep, ref_margin, row_offset=0):
 
 
 def compare_bwd_keep(gpu_keep, ref_keep, ref_margin, skip_blocks=()):
+    """Backward keep sets of one slice (rows = query blocks, columns = key
+    blocks). Rows in ``skip_blocks`` (forward flips: their LSE differs) are
+    not compared. Returns the list of allowed near-threshold flips (i, j);
+    raises AssertionError on any other mismatch."""
     nb = ref_keep.shape[0]
-    n_near = 0
+    flips = []
     tril = np.tril(np.ones((nb, nb), bool))
     diff = (gpu_keep.astype(bool) != ref_keep.astype(bool)) & tril
     for i, j in zip(*np.nonzero(diff)):
         if i in skip_blocks:
             continue
         assert abs(ref_margin[i, j]) <= NEAR, f"bwd keep mismatch at ({i},{j}) margin {ref_margin[i, j]}"
-        n_near += 1
-    return n_near
+        flips.append((int(i), int(j)))
+    return flips
+
+
+def grad_row_masks(L, tile, fwd_bad, bwd_flips, gpu_bkeep, ref_bkeep):
+    """Rows of dQ (query rows) and of dK, dV (key rows) that no allowed flip
+    touches (see the module docstring)."""
+    qmask = np.ones(L, bool)
+    kmask = np.ones(L, bool)
+    either = gpu_bkeep.astype(bool) | ref_bkeep.astype(bool)
+    for i in fwd_bad:
+        qmask[i * tile:(i + 1) * tile] = False
+        for j in np.nonzero(either[i, :i + 1])[0]:
+            kmask[j * tile:(j + 1) * tile] = False
+    for i, j in bwd_flips:
+        qmask[i * tile:(i + 1) * tile] = False
+        kmask[j * tile:(j + 1) * tile] = False
+    return qmask, kmask
+
+
+class Coverage:
+    """What a test compared: rows per tensor (compared, total) and the
+    near-threshold flips it allowed. ``report()`` prints one line (visible
+    with pytest -s or in the failure output); ``require()`` asserts that at
+    least ``frac`` of the rows of every tensor were compared."""
+
+    def __init__(self, name):
+        self.name = name
+        self.rows = {}
+        self.flips = {"fwd": 0, "bwd": 0, "decode": 0}
+        self.slices = 0
+
+    def add(self, tensor, mask):
+        c, t = self.rows.get(tensor, (0, 0))
+        self.rows[tensor] = (c + int(np.count_nonzero(mask)), t + int(np.size(mask)))
+
+    def report(self):
+        parts = [f"{k} {c}/{t}" for k, (c, t) in sorted(self.rows.items())]
+        print(f"[coverage] {self.name}: slices {self.slices}; rows compared " + ", ".join(parts) +
+              f"; near-threshold flips fwd {self.flips['fwd']} bwd {self.flips['bwd']} "
+              f"decode {self.flips['decode']}", flush=True)
+
+    def require(self, frac):
+        self.report()
+        assert self.rows, "nothing compared"
+        for k, (c, t) in self.rows.items():
+            assert c >= frac * t, f"{self.name}: only {c} of {t} rows of {k} compared"
 
 
 def row_mask(L, tile, bad_blocks):
@@ -80,7 +135,9 @@ def as_f64(t):
 
 def compare_decode_keep(gpu_keep, ref_keep, ref_margin):
     """Decode keep sequence of one group: tiles visited newest first. Returns
-    True if an allowed near-threshold flip happened (later tiles unchecked)."""
+    True if an allowed near-threshold flip happened (later tiles unchecked;
+    the group's output then differs legitimately: its heads share the
+    decisions)."""
     nt = len(ref_keep)
     for t in range(nt - 1, -1, -1):
         if int(gpu_keep[t]) == int(ref_keep[t]):

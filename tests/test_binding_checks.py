@@ -46,23 +46,19 @@ def test_prefill_inputs():
 def test_forward_buffers():
     q, _, _ = prefill()
     B, H, L, _ = q.shape
-    need = mala.tile_rowmax_bytes(B, H, L, 128)
     good = dict(out=torch.empty_like(q), lse=torch.empty((B, H, L), dtype=f32),
-                o32=torch.empty(q.shape, dtype=f32), rowmax=torch.empty(need // 4, dtype=f32))
-    mala._check_fwd_buffers(q, 128, **good)
-    mala._check_fwd_buffers(q, 128)
+                o32=torch.empty(q.shape, dtype=f32))
+    mala._check_fwd_buffers(q, **good)
+    mala._check_fwd_buffers(q)
     for name, bad, msg in (
             ("out", torch.empty((B, H, L - 1, 128), dtype=bf16), "shape"),
             ("out", torch.empty(q.shape, dtype=f32), "must be"),
             ("lse", torch.empty((B, H, L), dtype=bf16), "must be"),
             ("lse", torch.empty((B * H * L,), dtype=f32), "shape"),
             ("o32", torch.empty(q.shape, dtype=bf16), "must be"),
-            ("rowmax", torch.empty(need // 4 - 1, dtype=f32), "bytes"),
-            # enough elements but half the bytes
-            ("rowmax", torch.empty(need // 4, dtype=bf16), "must be"),
             ("out", torch.empty(q.shape, dtype=bf16, device="meta"), "must be on")):
         with pytest.raises(ValueError, match=msg):
-            mala._check_fwd_buffers(q, 128, **dict(good, **{name: bad}))
+            mala._check_fwd_buffers(q, **dict(good, **{name: bad}))
 
 
 def test_backward_buffers():
@@ -71,20 +67,17 @@ def test_backward_buffers():
     lse = torch.empty((B, H, L), dtype=f32)
     grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(k))
     ws = torch.empty(mala.bwd_workspace_bytes(B, H, L, 128), dtype=torch.uint8)
-    mala._check_bwd_buffers(q, k, lse, 128, o32=torch.empty(q.shape, dtype=f32),
-                            rowmax=torch.empty(mala.tile_rowmax_bytes(B, H, L, 128) // 4,
-                                               dtype=f32), grads=grads, workspace=ws)
-    mala._check_bwd_buffers(q, k, lse, 128)
+    mala._check_bwd_buffers(q, k, lse, o32=torch.empty(q.shape, dtype=f32), grads=grads,
+                            workspace=ws)
+    mala._check_bwd_buffers(q, k, lse)
     with pytest.raises(ValueError, match="lse"):
-        mala._check_bwd_buffers(q, k, lse[:, :1].contiguous(), 128)
+        mala._check_bwd_buffers(q, k, lse[:, :1].contiguous())
     with pytest.raises(ValueError, match="o32"):
-        mala._check_bwd_buffers(q, k, lse, 128, o32=torch.empty(q.shape, dtype=bf16))
-    with pytest.raises(ValueError, match="rowmax"):
-        mala._check_bwd_buffers(q, k, lse, 128, rowmax=torch.empty(16, dtype=f32))
+        mala._check_bwd_buffers(q, k, lse, o32=torch.empty(q.shape, dtype=bf16))
     with pytest.raises(ValueError, match="dK"):  # grouped heads: dK has K's shape
-        mala._check_bwd_buffers(q, k, lse, 128, grads=(grads[0], torch.empty_like(q), grads[2]))
+        mala._check_bwd_buffers(q, k, lse, grads=(grads[0], torch.empty_like(q), grads[2]))
     with pytest.raises(ValueError, match="workspace"):
-        mala._check_bwd_buffers(q, k, lse, 128, workspace=torch.empty((64, 64))[:, ::2])
+        mala._check_bwd_buffers(q, k, lse, workspace=torch.empty((64, 64))[:, ::2])
 
 
 def decode(B=2, Hq=8, Hkv=2, Lc=1000, d=128):

@@ -57,34 +57,31 @@ def test_forward_and_backward(rec):
     q = torch.randn((B, H, L, d)).to(bf16)
     k = torch.randn((B, Hkv, L, d)).to(bf16)
     v, do = torch.randn_like(k.float()).to(bf16), torch.randn_like(q.float()).to(bf16)
-    O, LSE, kept, bits, O32, RM = mala.mala_fwd(q, k, v, tau=0.5, trace=True, o32=True,
-                                                rowmax=True)
+    O, LSE, kept, bits, O32 = mala.mala_fwd(q, k, v, tau=0.5, trace=True, o32=True)
     name, a = rec.calls[-1]
     assert name == "mala_fwd"
     a = [val(x) for x in a]
     assert a[0] == ptr(q) and a[1] == ptr(k) and a[2] == ptr(v) and a[3] == ptr(O)
-    assert a[4] == ptr(LSE) and a[5] == ptr(O32) and a[6] == ptr(RM)
-    assert a[7:14] == [B, H, Hkv, L, d, mala.MALA_BF16, 0.5] and a[14] == 128
-    assert a[16] == ptr(kept) and a[17] == ptr(bits)
+    assert a[4] == ptr(LSE) and a[5] == ptr(O32)
+    assert a[6:13] == [B, H, Hkv, L, d, mala.MALA_BF16, 0.5] and a[13] == 128
+    assert a[15] == ptr(kept) and a[16] == ptr(bits)
     assert kept.shape == (B, H, 3) and bits.shape == (B, H, 3, 1)
-    assert RM.numel() * 4 == mala.tile_rowmax_bytes(B, H, L, 128)
     # the benchmark's form: every buffer passed in
-    mala.mala_fwd(q, k, v, tau=1.0, out=O, lse=LSE, o32=O32, rowmax=RM)
-    assert [val(x) for x in rec.calls[-1][1][3:7]] == [ptr(O), ptr(LSE), ptr(O32), ptr(RM)]
+    mala.mala_fwd(q, k, v, tau=1.0, out=O, lse=LSE, o32=O32)
+    assert [val(x) for x in rec.calls[-1][1][3:6]] == [ptr(O), ptr(LSE), ptr(O32)]
 
-    dQ, dK, dV, kb, bb = mala.mala_bwd(q, k, v, O, do, LSE, tau=0.5, trace=True, o32=O32,
-                                       rowmax=RM)
+    dQ, dK, dV, kb, bb = mala.mala_bwd(q, k, v, O, do, LSE, tau=0.5, trace=True, o32=O32)
     name, a = rec.calls[-1]
     a = [val(x) for x in a]
     assert name == "mala_bwd" and dK.shape == k.shape and dQ.shape == q.shape
-    assert a[4] == ptr(O32) and a[5] == ptr(do) and a[6] == ptr(LSE) and a[7] == ptr(RM)
-    assert a[12] >= mala.bwd_workspace_bytes(B, H, L, d)
-    assert a[13:20] == [B, H, Hkv, L, d, mala.MALA_BF16, 0.5]
+    assert a[4] == ptr(O32) and a[5] == ptr(do) and a[6] == ptr(LSE)
+    assert a[11] >= mala.bwd_workspace_bytes(B, H, L, d)
+    assert a[12:19] == [B, H, Hkv, L, d, mala.MALA_BF16, 0.5]
     ws = torch.empty(mala.bwd_workspace_bytes(B, H, L, d), dtype=torch.uint8)
     grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(k))
-    mala.mala_bwd(q, k, v, O, do, LSE, workspace=ws, grads=grads, o32=O32, rowmax=RM)
+    mala.mala_bwd(q, k, v, O, do, LSE, workspace=ws, grads=grads, o32=O32)
     a = [val(x) for x in rec.calls[-1][1]]
-    assert a[8:13] == [ptr(grads[0]), ptr(grads[1]), ptr(grads[2]), ptr(ws), ws.numel()]
+    assert a[7:12] == [ptr(grads[0]), ptr(grads[1]), ptr(grads[2]), ptr(ws), ws.numel()]
     mala.mala_check()
     assert rec.calls[-1][0] == "mala_check"
 
@@ -93,7 +90,7 @@ def test_float32_and_empty(rec):
     q = torch.randn((1, 1, 200, 64))
     O, LSE = mala.mala_fwd(q, q, q, tau=1.0)
     a = [val(x) for x in rec.calls[-1][1]]
-    assert a[12] == mala.MALA_F32 and a[14] == 64 and O.dtype == f32
+    assert a[11] == mala.MALA_F32 and a[13] == 64 and O.dtype == f32
     z = torch.empty((1, 1, 0, 128), dtype=bf16)
     O, LSE = mala.mala_fwd(z, z, z)
     assert O.numel() == 0 and LSE.shape == (1, 1, 0)

@@ -9,8 +9,8 @@ import pytest
 
 import oracle
 import synth
-from tests.parity import (TOL, as_f64, compare_bwd_keep, compare_decode_keep, compare_fwd_keep,
-                          rel_l2, row_mask)
+from tests.parity import (TOL, Coverage, as_f64, compare_bwd_keep, compare_decode_keep,
+                          compare_fwd_keep, grad_row_masks, rel_l2, row_mask)
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -36,8 +36,10 @@ def prefill_case(cfg, L=None, heads=None, dtype=torch.bfloat16):
     return t
 
 
-def check_fwd_slice(Qd, Kd, Vd, O_gpu, LSE_gpu, bits_gpu, tile, tau, tol, qblocks=None):
-    """One (b, h) slice; returns (rows_compared, near_flips)."""
+def check_fwd_slice(Qd, Kd, Vd, O_gpu, LSE_gpu, bits_gpu, tile, tau, tol, qblocks=None,
+                    cov=None):
+    """One (b, h) slice; returns (rows_compared, near_flips, oracle result,
+    query blocks with an allowed flip)."""
     L = Qd.shape[0]
     nb = oracle.n_blocks(L, tile)
     ref = oracle.fwd(Qd, Kd, Vd, tile=tile, tau=tau, want_margin=True, qblocks=qblocks)
@@ -49,9 +51,14 @@ def check_fwd_slice(Qd, Kd, Vd, O_gpu, LSE_gpu, bits_gpu, tile, tau, tol, qblock
     sel = np.zeros(L, bool)
     sel[lo * tile:min(L, hi * tile)] = True
     rows &= sel
-    assert rel_l2(O_gpu[rows], ref["O"][rows]) <= tol["O"]
-    assert rel_l2(LSE_gpu[rows], ref["LSE"][rows]) <= tol["LSE"]
-    return int(rows.sum()), n_near, ref
+    if rows.any():
+        assert rel_l2(O_gpu[rows], ref["O"][rows]) <= tol["O"]
+        assert rel_l2(LSE_gpu[rows], ref["LSE"][rows]) <= tol["LSE"]
+    if cov is not None:
+        cov.add("O", rows[sel])
+        cov.flips["fwd"] += n_near
+        cov.slices += 1
+    return int(rows.sum()), n_near, ref, bad
 
 
 # ----------------------------------------------------------------------------
@@ -67,13 +74,13 @@ def test_f32_tiny_config_fwd_bwd(tau):
                                                trace=True)
     mala.mala_check()
     Qd, Kd, Vd, dOd = (rounded(t[n][0, 0]) for n in ("Q", "K", "V", "dO"))
-    _, n_near, ref = check_fwd_slice(Qd, Kd, Vd, as_f64(O[0, 0]), as_f64(LSE[0, 0]), bits[0, 0],
-                                     64, tau, TOL["f32"])
+    _, n_near, ref, _ = check_fwd_slice(Qd, Kd, Vd, as_f64(O[0, 0]), as_f64(LSE[0, 0]),
+                                        bits[0, 0], 64, tau, TOL["f32"])
     assert n_near == 0
     nb = 16
     assert np.array_equal(kept[0, 0].cpu().numpy(), ref["keep"].sum(axis=1))
     g = oracle.bwd(Qd, Kd, Vd, ref["O"], dOd, ref["LSE"], tile=64, tau=tau, want_margin=True)
-    assert compare_bwd_keep(mala.unpack_bits(bits_b[0, 0], nb), g["keep"], g["margin"]) == 0
+    assert compare_bwd_keep(mala.unpack_bits(bits_b[0, 0], nb), g["keep"], g["margin"]) == []
     assert np.array_equal(kept_b[0, 0].cpu().numpy(), g["keep"].sum(axis=0))
     for n, a in (("dQ", dQ), ("dK", dK), ("dV", dV)):
         assert rel_l2(as_f64(a[0, 0]), g[n]) <= TOL["f32"]["grad"], n
@@ -97,8 +104,8 @@ def test_f32_ragged_shapes(L, d, B, H):
     for b in range(B):
         for h in range(H):
             Qd, Kd, Vd, dOd = (rounded(t[n][b, h]) for n in ("Q", "K", "V", "dO"))
-            _, n_near, ref = check_fwd_slice(Qd, Kd, Vd, as_f64(O[b, h]), as_f64(LSE[b, h]),
-                                             bits[b, h], 64, 1.0, TOL["f32"])
+            _, n_near, ref, _ = check_fwd_slice(Qd, Kd, Vd, as_f64(O[b, h]), as_f64(LSE[b, h]),
+                                                bits[b, h], 64, 1.0, TOL["f32"])
             assert n_near == 0
             g = oracle.bwd(Qd, Kd, Vd, ref["O"], dOd, ref["LSE"], tile=64, tau=1.0)
             for n, a in (("dQ", dQ), ("dK", dK), ("dV", dV)):
@@ -108,15 +115,14 @@ def test_f32_ragged_shapes(L, d, B, H):
 # ----------------------------------------------------------------------------
 # bf16 tcgen05 path (128 x 128 tiles, d = 128)
 # ----------------------------------------------------------------------------
-def run_bf16_prefill(t, tau, use_o32=True, use_rowmax=False):
-    """The training chain: forward (with its float32 output when use_o32, its
-    tile row maxima when use_rowmax), then backward."""
+def run_bf16_prefill(t, tau, use_o32=True):
+    """The training chain: forward (with its float32 output when use_o32),
+    then backward; only O (or its float32 copy) and LSE pass between them."""
     O, LSE, kept, bits, *rest = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True,
-                                              o32=use_o32, rowmax=use_rowmax)
-    o32 = rest.pop(0) if use_o32 else None
-    rm = rest.pop(0) if use_rowmax else None
+                                              o32=use_o32)
+    o32 = rest[0] if use_o32 else None
     dQ, dK, dV, kept_b, bits_b = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
-                                               trace=True, o32=o32, rowmax=rm)
+                                               trace=True, o32=o32)
     mala.mala_check()
     if use_o32:  # the float32 output is the bf16 output before rounding
         assert torch.equal(o32.to(torch.bfloat16), O)
@@ -127,94 +133,46 @@ def bf16_round(a):
     return torch.tensor(a).to(torch.bfloat16).double().numpy()
 
 
-def check_bf16_slice(t, outs, b, h, tau, grads=True, o_rounded=False):
+def check_bf16_slice(t, outs, b, h, tau, cov, grads=True, o_rounded=False):
     """Forward against the oracle; backward against the oracle's backward fed
     the oracle's own forward output. With ``o_rounded`` (the chain without
     the float32 output) the backward's row terms D_r = <dO_r, O_r> are
     defined on the bf16 O it is given, so the oracle is fed its own O rounded
-    to bf16."""
+    to bf16. Rows touched by an allowed near-threshold flip are left out
+    (tests/parity.py); ``cov`` records what was compared."""
     O, LSE, kept, bits, dQ, dK, dV, kept_b, bits_b = outs
     Qd, Kd, Vd, dOd = (rounded(t[n][b, h]) for n in ("Q", "K", "V", "dO"))
     L = Qd.shape[0]
     nb = oracle.n_blocks(L, 128)
-    _, n_near, ref = check_fwd_slice(Qd, Kd, Vd, as_f64(O[b, h]), as_f64(LSE[b, h]), bits[b, h],
-                                     128, tau, TOL["bf16"])
+    _, _, ref, bad = check_fwd_slice(Qd, Kd, Vd, as_f64(O[b, h]), as_f64(LSE[b, h]), bits[b, h],
+                                     128, tau, TOL["bf16"], cov=cov)
+    if not bad:
+        assert np.array_equal(kept[b, h].cpu().numpy(), ref["keep"].sum(axis=1))
     if not grads:
-        return n_near, 0
-    gk = mala.unpack_bits(bits[b, h], nb)
-    _, bad = compare_fwd_keep(gk, ref["keep"], ref["margin"])
+        return
     O_in = bf16_round(ref["O"]) if o_rounded else ref["O"]
     g = oracle.bwd(Qd, Kd, Vd, O_in, dOd, ref["LSE"], tile=128, tau=tau, want_margin=True)
-    n_near_b = compare_bwd_keep(mala.unpack_bits(bits_b[b, h], nb), g["keep"], g["margin"],
-                                skip_blocks=bad)
-    if not bad:
-        for n, a in (("dQ", dQ), ("dK", dK), ("dV", dV)):
-            assert rel_l2(as_f64(a[b, h]), g[n]) <= TOL["bf16"]["grad"], n
-    return n_near, n_near_b
+    gb = mala.unpack_bits(bits_b[b, h], nb)
+    flips = compare_bwd_keep(gb, g["keep"], g["margin"], skip_blocks=bad)
+    cov.flips["bwd"] += len(flips)
+    qmask, kmask = grad_row_masks(L, 128, bad, flips, gb, g["keep"])
+    for n, a, m in (("dQ", dQ, qmask), ("dK", dK, kmask), ("dV", dV, kmask)):
+        if m.any():
+            assert rel_l2(as_f64(a[b, h])[m], g[n][m]) <= TOL["bf16"]["grad"], n
+        cov.add(n, m)
 
 
 @pytest.mark.parametrize("L", [128, 1000, 1536])
 @pytest.mark.parametrize("tau", [1.0, 0.0])
-@pytest.mark.parametrize("use_rowmax", [False, True])
-def test_bf16_small_fwd_bwd(L, tau, use_rowmax):
+def test_bf16_small_fwd_bwd(L, tau):
     cfg = synth.CONFIGS["matched_8k"]
     t = prefill_case(cfg, L=L, heads=[0, 1])
     t = {n: v[:, :2].contiguous() for n, v in t.items()}
-    outs = run_bf16_prefill(t, tau, use_rowmax=use_rowmax)
+    outs = run_bf16_prefill(t, tau)
+    cov = Coverage(f"small L={L} tau={tau}")
     for h in range(2):
-        check_bf16_slice(t, outs, 0, h, tau)
-
-
-def rowmax_parts(RM, Z, L, T=128):
-    """Split the forward's row-maxima buffer into maxima [Z, ntri, T] and the
-    per-tile stored flags [Z, nb, nb] (host numpy)."""
-    nb = oracle.n_blocks(L, T)
-    ntri = nb * (nb + 1) // 2
-    r256 = lambda x: (x + 255) // 256 * 256
-    nmax = r256(Z * ntri * T * 4) // 4
-    nw = (nb + 31) // 32
-    maxima = RM[:Z * ntri * T].view(Z, ntri, T).double().cpu().numpy()
-    flags = RM[nmax:nmax + Z * nb * nw].view(torch.int32).view(Z, nb, nw)
-    return maxima, mala.unpack_bits(flags, nb)
-
-
-@pytest.mark.parametrize("L,tau", [(1000, 1.0), (1536, 0.25), (2048, 1.0)])
-def test_bf16_tile_rowmax(L, tau):
-    """The forward's recorded tile row maxima against the oracle's (valid
-    rows of every stored tile; float32 sums of 128 exact bf16 products,
-    bounded by 128 ulp of |q| max|k|); every tile the forward kept is stored;
-    and the backward's test from them equals the test that recomputes every
-    score: the same bits, the same counts."""
-    cfg = synth.CONFIGS["matched_8k"]
-    t = prefill_case(cfg, L=L, heads=[0, 1])
-    t = {n: v[:, :2].contiguous() for n, v in t.items()}
-    O, LSE, kept, fbits, O32, RM = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True,
-                                                 o32=True, rowmax=True)
-    *_, kept_r, bits_r = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
-                                       trace=True, o32=O32, rowmax=RM)
-    *_, kept_s, bits_s = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
-                                       trace=True, o32=O32)
-    mala.mala_check()
-    assert torch.equal(bits_r, bits_s)
-    assert torch.equal(kept_r, kept_s)
-    nb = oracle.n_blocks(L, 128)
-    maxima, stored = rowmax_parts(RM, 2, L)
-    fkeep = mala.unpack_bits(fbits, nb)[0]
-    assert np.all(stored[fkeep == 1] == 1)
-    assert not np.any(np.triu(stored[0], 1)) and not np.any(np.triu(stored[1], 1))
-    n_checked = 0
-    for h in range(2):
-        Qd, Kd = rounded(t["Q"][0, h]), rounded(t["K"][0, h])
-        ref = oracle.tile_row_max(Qd, Kd, 128)
-        kmax = np.linalg.norm(Kd, axis=1).max()
-        for i in range(nb):
-            rows = min(L - i * 128, 128)
-            bound = 128 * 2.0 ** -24 * np.linalg.norm(Qd[i * 128:i * 128 + rows], axis=1) * kmax
-            for j in np.nonzero(stored[h, i, :i + 1])[0]:
-                got = maxima[h, i * (i + 1) // 2 + j, :rows]
-                assert np.all(np.abs(got - ref[i][j, :rows]) <= bound + 1e-30), (i, j)
-                n_checked += 1
-    assert n_checked > 0
+        check_bf16_slice(t, outs, 0, h, tau, cov)
+    cov.require(0.5)
 
 
 @pytest.mark.parametrize("L", [1000])
@@ -224,8 +182,10 @@ def test_bf16_chain_without_float32_output(L):
     t = prefill_case(cfg, L=L, heads=[0, 1])
     t = {n: v[:, :2].contiguous() for n, v in t.items()}
     outs = run_bf16_prefill(t, 1.0, use_o32=False)
+    cov = Coverage("chain without float32 output")
     for h in range(2):
-        check_bf16_slice(t, outs, 0, h, 1.0, o_rounded=True)
+        check_bf16_slice(t, outs, 0, h, 1.0, cov, o_rounded=True)
+    cov.require(0.5)
 
 
 def test_bf16_random_inputs_multi_batch():
@@ -234,39 +194,64 @@ def test_bf16_random_inputs_multi_batch():
     arrs = [rng.standard_normal((B, H, L, d)) * s for s in (1.5, 1.5, 1.0, 1.0)]
     t = {n: dev_tensor(a, torch.bfloat16) for n, a in zip(("Q", "K", "V", "dO"), arrs)}
     outs = run_bf16_prefill(t, 1.0)
+    cov = Coverage("random inputs B=2 H=2")
     for b in range(B):
         for h in range(H):
-            check_bf16_slice(t, outs, b, h, 1.0)
+            check_bf16_slice(t, outs, b, h, 1.0, cov)
+    cov.require(0.5)
 
 
 def test_bf16_matched_work_config_full():
     """B=1 H=8 L=8192 d=128 bf16 tile 128 tau=1: every head, every output."""
     cfg = synth.CONFIGS["matched_8k"]
     t = prefill_case(cfg)
-    outs = run_bf16_prefill(t, 1.0, use_rowmax=True)
+    outs = run_bf16_prefill(t, 1.0)
+    cov = Coverage("matched_8k")
     for h in range(cfg.H):
-        check_bf16_slice(t, outs, 0, h, 1.0)
+        check_bf16_slice(t, outs, 0, h, 1.0, cov)
+    cov.require(0.75)
 
 
-@pytest.mark.parametrize("L", [2048, 16384])
-def test_bf16_sweep_config_sampled_heads(L):
-    """Length-sweep configuration (H=16), tau=1 and tau=0, two heads checked."""
+@pytest.mark.parametrize("L", [1024, 2048, 4096, 8192])
+@pytest.mark.parametrize("tau", [1.0, 0.0])
+def test_bf16_sweep_config_all_heads(L, tau):
+    """Length-sweep configuration (B=1 H=16 d=128 bf16 tile 128) at the
+    lengths up to 8K: forward and backward of all 16 heads."""
     cfg = synth.CONFIGS[f"sweep_L{L}"]
+    t = prefill_case(cfg)
+    outs = run_bf16_prefill(t, tau)
+    cov = Coverage(f"sweep L={L} tau={tau}")
+    for h in range(cfg.H):
+        check_bf16_slice(t, outs, 0, h, tau, cov)
+    cov.require(0.75)
+
+
+@pytest.mark.parametrize("tau", [1.0, 0.0])
+def test_bf16_sweep_16k_two_heads(tau):
+    """Length-sweep configuration at L=16384 (H=16): heads 0 and 9, forward
+    and backward."""
+    cfg = synth.CONFIGS["sweep_L16384"]
     t = prefill_case(cfg, heads=[0, 9])
-    for tau in (1.0, 0.0):
-        outs = run_bf16_prefill(t, tau)
-        for h in (0, 9):
-            check_bf16_slice(t, outs, 0, h, tau, grads=(L <= 4096 or tau == 1.0))
+    outs = run_bf16_prefill(t, tau)
+    cov = Coverage(f"sweep L=16384 tau={tau}")
+    for h in range(2):
+        check_bf16_slice(t, outs, 0, h, tau, cov)
+    cov.require(0.75)
 
 
 # ----------------------------------------------------------------------------
 # decode
 # ----------------------------------------------------------------------------
-def check_decode(q, Kc, Vc, o, kept, bits, tau, groups):
+def check_decode(q, Kc, Vc, o, kept, bits, tau, groups, min_frac=0.75):
+    """Keep sets, kept counts and outputs of the given (b, kv head) groups. A
+    group with an allowed near-threshold flip is counted, not compared (its
+    heads share the decisions, so its whole output legitimately differs); at
+    least ``min_frac`` of the groups must be compared."""
     B, Hq, d = q.shape
     Hkv, Lc = Kc.shape[1], Kc.shape[2]
     G = Hq // Hkv
     nt = oracle.n_blocks(Lc, 128)
+    cov = Coverage(f"decode B={B} Hq={Hq} Hkv={Hkv} Lc={Lc} tau={tau}")
     for b in sorted(set(g // Hkv for g in groups)):
         ref = oracle.decode(rounded(q[b]), rounded(Kc[b]), rounded(Vc[b]), tau=tau,
                             want_margin=True)
@@ -274,11 +259,16 @@ def check_decode(q, Kc, Vc, o, kept, bits, tau, groups):
         for g in range(Hkv):
             if b * Hkv + g not in groups:
                 continue
+            cov.slices += 1
             if compare_decode_keep(gk[g], ref["keep"][g], ref["margin"][g]):
+                cov.flips["decode"] += 1
+                cov.add("o", np.zeros(G, bool))
                 continue
             assert kept[b, g].item() == int(ref["keep"][g].sum())
             sl = slice(g * G, (g + 1) * G)
             assert rel_l2(as_f64(o[b, sl]), ref["o"][sl]) <= TOL["bf16"]["decode"]
+            cov.add("o", np.ones(G, bool))
+    cov.require(min_frac)
 
 
 def test_decode_long_cache_wraps_the_ring():
@@ -342,16 +332,22 @@ def test_decode_per_head_rows(Lc, tau):
     B, Hq = q.shape[0], q.shape[1]
     gk = mala.unpack_bits(bits, nt)  # [B, Hq, nt]
     fewer = 0
+    cov = Coverage(f"decode per-head rows Lc={Lc} tau={tau}")
     for b in range(B):
         ref = oracle.decode(rounded(q[b]), rounded(Kc[b]), rounded(Vc[b]), tau=tau, per_head=True,
                             want_margin=True)
         for h in range(Hq):
+            cov.slices += 1
             if compare_decode_keep(gk[b, h], ref["keep"][h], ref["margin"][h]):
+                cov.flips["decode"] += 1
+                cov.add("o", np.zeros(1, bool))
                 continue
             assert kept[b, h].item() == int(ref["keep"][h].sum())
             assert rel_l2(as_f64(o[b, h]), ref["o"][h]) <= TOL["bf16"]["decode"]
+            cov.add("o", np.ones(1, bool))
             fewer += int(ref["keep"][h].sum())
     assert fewer > 0
+    cov.require(0.75)
 
 
 def gqa_case(L):
@@ -369,42 +365,45 @@ def gqa_case(L):
     return t
 
 
-@pytest.mark.parametrize("L,tau,use_rowmax", [(1000, 1.0, True), (1536, 0.25, False), (640, 0.0, False)])
-def test_bf16_grouped_query_heads(L, tau, use_rowmax):
+@pytest.mark.parametrize("L,tau", [(1000, 1.0), (1536, 0.25), (640, 0.0)])
+def test_bf16_grouped_query_heads(L, tau):
     """Grouped query heads (Hq = 4, Hkv = 2): per query head the rule on the
     shared K, V; dK, dV of a kv head are the sums over its query heads."""
     t = gqa_case(L)
-    O, LSE, kept, bits, *rest = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True,
-                                              o32=True, rowmax=use_rowmax)
-    O32 = rest[0]
-    rm = rest[1] if use_rowmax else None
+    O, LSE, kept, bits, O32 = mala.mala_fwd(t["Q"], t["K"], t["V"], tau=tau, trace=True,
+                                            o32=True)
     dQ, dK, dV, kept_b, bits_b = mala.mala_bwd(t["Q"], t["K"], t["V"], O, t["dO"], LSE, tau=tau,
-                                               trace=True, o32=O32, rowmax=rm)
+                                               trace=True, o32=O32)
     mala.mala_check()
     nb = oracle.n_blocks(L, 128)
     Kd, Vd = [rounded(t["K"][0, g]) for g in range(2)], [rounded(t["V"][0, g]) for g in range(2)]
     refK, refV = [np.zeros_like(Kd[0]), np.zeros_like(Kd[0])], [np.zeros_like(Vd[0]), np.zeros_like(Vd[0])]
-    clean = True
+    kmasks = [np.ones(L, bool), np.ones(L, bool)]
+    cov = Coverage(f"grouped heads L={L} tau={tau}")
     for h in range(4):
         g = h // 2
         Qd, dOd = rounded(t["Q"][0, h]), rounded(t["dO"][0, h])
-        _, n_near, ref = check_fwd_slice(Qd, Kd[g], Vd[g], as_f64(O[0, h]), as_f64(LSE[0, h]),
-                                         bits[0, h], 128, tau, TOL["bf16"])
-        gk = mala.unpack_bits(bits[0, h], nb)
-        _, bad = compare_fwd_keep(gk, ref["keep"], ref["margin"])
+        _, _, ref, bad = check_fwd_slice(Qd, Kd[g], Vd[g], as_f64(O[0, h]), as_f64(LSE[0, h]),
+                                         bits[0, h], 128, tau, TOL["bf16"], cov=cov)
         gr = oracle.bwd(Qd, Kd[g], Vd[g], ref["O"], dOd, ref["LSE"], tile=128, tau=tau,
                         want_margin=True)
-        compare_bwd_keep(mala.unpack_bits(bits_b[0, h], nb), gr["keep"], gr["margin"],
-                         skip_blocks=bad)
-        clean = clean and not bad
-        if not bad:
-            assert rel_l2(as_f64(dQ[0, h]), gr["dQ"]) <= TOL["bf16"]["grad"]
+        gb = mala.unpack_bits(bits_b[0, h], nb)
+        flips = compare_bwd_keep(gb, gr["keep"], gr["margin"], skip_blocks=bad)
+        cov.flips["bwd"] += len(flips)
+        qmask, kmask = grad_row_masks(L, 128, bad, flips, gb, gr["keep"])
+        if qmask.any():
+            assert rel_l2(as_f64(dQ[0, h])[qmask], gr["dQ"][qmask]) <= TOL["bf16"]["grad"]
+        cov.add("dQ", qmask)
+        kmasks[g] &= kmask  # a kv head's dK, dV sum over its query heads
         refK[g] += gr["dK"]
         refV[g] += gr["dV"]
-    if clean:
-        for g in range(2):
-            assert rel_l2(as_f64(dK[0, g]), refK[g]) <= TOL["bf16"]["grad"]
-            assert rel_l2(as_f64(dV[0, g]), refV[g]) <= TOL["bf16"]["grad"]
+    for g in range(2):
+        m = kmasks[g]
+        if m.any():
+            assert rel_l2(as_f64(dK[0, g])[m], refK[g][m]) <= TOL["bf16"]["grad"]
+            assert rel_l2(as_f64(dV[0, g])[m], refV[g][m]) <= TOL["bf16"]["grad"]
+        cov.add("dK, dV", m)
+    cov.require(0.5)
 
 
 @pytest.mark.parametrize("tau", [1.0, 0.25])
