@@ -258,8 +258,9 @@ mala_status mala_decode_noalloc(const void* q, const void* Kcache,
 
 /*
  * Synchronizes `stream`, then reads and clears this GPU's device status word.
- * Returns MALA_ERR_CUDA if the stream reported an error, MALA_ERR_TIMEOUT if
- * a kernel gave up on a wait since the last check, MALA_OK otherwise.
+ * Returns MALA_ERR_CUDA if the stream reported an error (or a kernel found
+ * its shared memory laid out unusably and did nothing), MALA_ERR_TIMEOUT if a
+ * kernel gave up on a wait since the last check, MALA_OK otherwise.
  */
 mala_status mala_check(void* stream);
 

@@ -120,7 +120,7 @@ inline mala_status fwd_f32(const float* Q, const float* K, const float* V, float
   return launch_status();
 }
 
-template <bool VARLEN>
+template <bool VARLEN, bool DENSE>
 inline mala_status launch_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                const fwd2::Params& p, int npairs, int Z, cudaStream_t s);
 
@@ -153,19 +153,21 @@ inline mala_status fwd_bf16(const void* Q, const void* K, const void* V, void* O
   p.keep_bits = bits;
   p.Hq = Hq;
   p.G = Hq / Hkv;
-  return launch_pair<false>(mq, mk, mv, p, p.npairs, Z, s);
+  // tau = 0 keeps every tile: the instantiation with two P buffers
+  return p.never_skip ? launch_pair<false, true>(mq, mk, mv, p, p.npairs, Z, s)
+                      : launch_pair<false, false>(mq, mk, mv, p, p.npairs, Z, s);
 }
 
-template <bool VARLEN>
+template <bool VARLEN, bool DENSE>
 inline mala_status launch_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                const fwd2::Params& p, int npairs, int Z, cudaStream_t s) {
-  MALA_CUDA_TRY(cudaFuncSetAttribute(fwd2::fwd_pair_kernel<VARLEN>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)fwd2::SMEM_BYTES));
+  constexpr uint32_t smem = fwd2::Plan<DENSE>::SMEM_BYTES;
+  MALA_CUDA_TRY(cudaFuncSetAttribute(fwd2::fwd_pair_kernel<VARLEN, DENSE>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * npairs, Z, 1);
   cfg.blockDim = dim3(fwd2::NT, 1, 1);
-  cfg.dynamicSmemBytes = fwd2::SMEM_BYTES;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -174,7 +176,7 @@ inline mala_status launch_pair(const CUtensorMap& mq, const CUtensorMap& mk, con
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  MALA_CUDA_TRY(cudaLaunchKernelEx(&cfg, fwd2::fwd_pair_kernel<VARLEN>, mq, mk, mv, p));
+  MALA_CUDA_TRY(cudaLaunchKernelEx(&cfg, fwd2::fwd_pair_kernel<VARLEN, DENSE>, mq, mk, mv, p));
   return launch_status();
 }
 
@@ -204,7 +206,7 @@ inline mala_status fwd_varlen_bf16(const void* Q, const void* K, const void* V, 
   p.total_q = total_q;
   p.nbq_max = (max_q + fwd2::T - 1) / fwd2::T;
   p.nw = varlen_trace_words(max_q, max_k);
-  return launch_pair<true>(mq, mk, mv, p, (p.nbq_max + 1) / 2, batch * Hq, s);
+  return launch_pair<true, false>(mq, mk, mv, p, (p.nbq_max + 1) / 2, batch * Hq, s);
 }
 
 // ---------------------------------------------------------------- backward
@@ -632,7 +634,7 @@ mala_status mala_check(void* stream) {
   if (st != 0) {
     if (cudaMemcpyToSymbol(mala::g_status, &zero, sizeof(zero)) != cudaSuccess)
       return MALA_ERR_CUDA;
-    return MALA_ERR_TIMEOUT;
+    return (st & mala::kStatusTimeout) ? MALA_ERR_TIMEOUT : MALA_ERR_CUDA;
   }
   return MALA_OK;
 }

@@ -20,6 +20,7 @@ __device__ unsigned int g_status_where = 0;
 
 enum : unsigned int {
   kStatusTimeout = 1u,
+  kStatusLayout = 2u,  // a kernel found its dynamic shared memory misaligned
 };
 
 // Wait limit for every device-side spin: about two seconds of %globaltimer.
@@ -33,6 +34,10 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 
 __device__ __forceinline__ void record_timeout(unsigned int where) {
   atomicOr(&g_status, kStatusTimeout);
+  atomicExch(&g_status_where, where);
+}
+__device__ __forceinline__ void record_layout_error(unsigned int where) {
+  atomicOr(&g_status, kStatusLayout);
   atomicExch(&g_status_where, where);
 }
 

@@ -16,27 +16,48 @@
 // (the leader): A is each CTA's own Q block, B (the key tile) is split by
 // rows, 64 keys in each CTA's shared memory, so each SM loads half of every
 // K tile; each CTA's TMEM receives its own 128 x 128 block of S. A kept
-// tile's PV is one M = 256 MMA as well (A = each CTA's P from its TMEM, B = V
-// split by columns, 64 of d in each CTA); the rows of a CTA that did not
-// keep the tile are masked out of D, so its O is untouched.
+// tile's PV is one M = 256 MMA as well (A = each CTA's P in its shared
+// memory, B = V split by columns, 64 of d in each CTA); the rows of a CTA
+// that did not keep the tile are masked out of D, so its O is untouched.
 //
-// TMEM (512 columns per SM): a ring of three S buffers [0, 384) and O
-// [384, 512). The ring lets the leader issue the next two tiles' QKs while a
-// tile is being tested, so the test's latency is off the tensor pipe's path.
+// With skipping, nearly every tile is a QK followed by a row-max test: per
+// tile a test thread waits for S, reads its row from TMEM, reduces it and
+// votes, a chain of dependent latencies longer than the tile's MMA. Two
+// warpgroups therefore take alternate key tiles of the block, so each has
+// two tiles' MMA time for its chain. Skipping stays exact although a group
+// tests against the running state it last saw: the bound
+// ln tau - ln Lq + m + ln l only grows as tiles are kept, so a tile below an
+// old bound is below the current one. A group that wants to keep a tile
+// first waits until every earlier tile is final, reloads the state the other
+// group may have advanced, tests again, and only then updates the state, so
+// the kept tiles are exactly those of the sequential rule. Each thread holds
+// its whole S row in registers and releases the S buffer right after the
+// TMEM load. At tau = 0 every tile is kept and the state is sequential, so
+// there the eight test warps instead split each row into two column halves.
 //
-// Warp roles (288 threads per CTA):
-//   warps 0-3  softmax / test of this CTA's block (thread r owns row r = TMEM lane r)
-//   warp  4    K producer: this CTA's Q block, then its half of each K tile (6 stages)
-//   warp  5    V producer: this CTA's half (64 columns of d) of each V tile a PV needs
-//   warps 6, 7 (leader) QK issuers for even / odd tiles. An issuing thread's own
+// The QK issuers wait for a tile's K and for the decision ring before they
+// wait for its S buffer, so the buffer's release is the last event before
+// the MMAs. Rank 1 sends buffer releases and decisions to the leader with
+// st.async (a store into the leader's shared memory counted on a leader
+// mbarrier), which does not hold up the sending warp.
+//
+// TMEM (512 columns per SM): three S buffers [0, 384) and O [384, 512).
+// Shared memory: Q, K-half stages, two V-half stages, P (hi, lo) buffers.
+//
+// Warp roles (384 threads per CTA, three warps per scheduler, so a thread
+// may use up to 168 registers):
+//   warps 0-7  softmax / test (thread t: row t % 128 = TMEM lane, group t / 128)
+//   warp  8    producer: this CTA's Q block, its half of each K tile, and its
+//              half (64 columns of d) of each V tile a PV needs
+//   warps 9, 10 (leader) QK issuers for even / odd tiles. An issuing thread's own
 //              shared-memory polls wait until its queued MMAs are dispatched, so
 //              two issuers keep the pipe fed while either one waits.
-//   warp  8    (leader) decisions: gathers both CTAs' votes per tile, requests V,
-//              issues PV, frees the S buffer for the QK four tiles later
+//   warp  11   (leader) decisions: reads both CTAs' decisions per tile, requests V,
+//              issues the PVs
 //
-// Every mbarrier wait is bounded; a wait that runs out records a timeout in
-// the device status word and the thread carries on, so every thread reaches
-// the final cluster barrier: the kernel always terminates.
+// Every wait is bounded; a wait that runs out records a timeout in the
+// device status word and the thread carries on, so every thread reaches the
+// final cluster barrier: the kernel always terminates.
 #pragma once
 
 #include "sm100.cuh"
@@ -48,25 +69,53 @@ using namespace sm100;
 
 constexpr int T = 128;
 constexpr int D = 128;
-constexpr int NT = 288;
-constexpr int WARP_KPROD = 4;
-constexpr int WARP_VPROD = 5;
-constexpr int WARP_QK0 = 6;  // also allocates TMEM (the same warp in both CTAs)
-constexpr int WARP_QK1 = 7;
-constexpr int WARP_DEC = 8;
-constexpr int NSK = 6;    // K half stages (even, so one stage's tiles share an issuer)
+constexpr int NT = 384;
+constexpr int NSOFT = 256;  // softmax / test threads
+constexpr int WARP_PROD = 8;
+constexpr int WARP_QK0 = 9;  // also allocates TMEM (the same warp in both CTAs)
+constexpr int WARP_QK1 = 10;
+constexpr int WARP_DEC = 11;
 constexpr int NSV = 2;    // V half stages
 constexpr int NSLOT = 3;  // S buffers
+constexpr int RD = 16;    // decision ring: tiles the PV issuer may fall behind the QKs
+constexpr int NFIN = 8;   // ring of "tile final" marks between the two test groups
 constexpr uint32_t Q_BYTES = T * D * 2;     // 32 KB: this CTA's query block
-constexpr uint32_t QH_BYTES = T * 64 * 2;   // one 64-column swizzled block of Q
+constexpr uint32_t QH_BYTES = T * 64 * 2;   // one 64-column swizzled block of Q (or P)
 constexpr uint32_t KH_BYTES = 64 * D * 2;   // 16 KB: 64 keys x 128 d
 constexpr uint32_t KH_BLK = 64 * 64 * 2;    // 8 KB: one 64-column block of a K half
 constexpr uint32_t VH_BYTES = T * 64 * 2;   // 16 KB: 128 keys x 64 columns of d
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
-constexpr uint32_t OFF_V = OFF_K + NSK * KH_BYTES;
-constexpr uint32_t OFF_BAR = OFF_V + NSV * VH_BYTES;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;
+constexpr uint32_t P_BYTES = T * T * 2;     // 32 KB: P_hi (then P_lo), 128 rows x 128 keys
+constexpr uint32_t BAR_BYTES = 3072;
+constexpr int NSK_MAX = 6;
+
+// Shared-memory plan. With skipping (DENSE = false) nearly every tile is a
+// 512-cycle QK, so six K stages cover the L2 latency and one P buffer
+// serves the kept tiles, which are rare and finalized in order. At tau = 0
+// every tile is kept and costs about three times as long, so two K stages
+// suffice and two P buffers let tile t + 1's P be written while tile t's PV
+// still reads its own.
+template <bool DENSE>
+struct Plan {
+  static constexpr int NSK = DENSE ? 2 : 6;  // even: one stage's tiles share an issuer
+  static constexpr int NPB = DENSE ? 2 : 1;  // P buffers, tile t uses t % NPB
+  // S buffer u's full / free barriers come in pairs, one per test group: tile
+  // t uses pair member t % 2 (DENSE: member 0 only, every warp reads every
+  // tile), so each barrier's phases are waited for in order by one consumer
+  static constexpr int SGRP_MASK = DENSE ? 0 : 1;
+  static constexpr int SPER = DENSE ? 3 : 6;            // tiles between uses of one barrier
+  static constexpr uint32_t REL_LOCAL = DENSE ? 8 : 4;  // releasing warps per CTA and tile
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+  static constexpr uint32_t OFF_V = OFF_K + NSK * KH_BYTES;
+  static constexpr uint32_t OFF_P = OFF_V + NSV * VH_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_P + NPB * 2 * P_BYTES;
+  // no alignment slack: the kernel requires (and checks) a 1024-byte
+  // aligned start, which dynamic shared memory has when a kernel declares
+  // no static shared memory
+  static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_BYTES;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(NSK % 2 == 0 && NSK <= NSK_MAX, "K stages");
+};
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_O = 384;
 constexpr uint32_t IDESC_QK = idesc_bf16(256, 128, false, false);
@@ -100,48 +149,245 @@ struct Params {
 };
 
 struct Bars {
-  uint64_t q_full;            // leader: both CTAs' Q blocks
-  uint64_t k_full[NSK];       // leader: both halves of a K tile
-  uint64_t k_empty[NSK];      // each CTA: stage free again
-  uint64_t s_full[NSLOT];     // each CTA: S of the slot's tile is in TMEM
-  // leader: a CTA's decision for a slot's tile arrives on exactly one of
-  // these two (per slot and rank), so the signal carries no data
-  uint64_t dec_keep[NSLOT][2];
-  uint64_t dec_skip[NSLOT][2];
-  uint64_t slot_free[NSLOT];  // leader: the slot may take the next QK
-  uint64_t v_req[NSV];        // each CTA: a V half to load (tile in req_j)
-  uint64_t v_full[NSV];       // leader: both V halves loaded
-  uint64_t v_empty[NSV];      // each CTA: V stage free again
-  uint64_t pv_done;           // each CTA: one arrival per PV that updated its O
-  int req_j[NSV];             // each CTA: key block of a V request, -1 = stop
+  uint64_t q_full;                 // leader: both CTAs' Q blocks
+  uint64_t k_full[NSK_MAX];        // leader: both halves of a K tile
+  uint64_t k_empty[NSK_MAX];       // each CTA: stage free again
+  uint64_t s_full[NSLOT][2];       // each CTA: S of a tile is in TMEM (see Plan::SGRP_MASK)
+  // leader: S read by both CTAs -- REL_LOCAL arrivals of its own test warps,
+  // and one of the QK issuer that arms 4 bytes for each of rank 1's stores
+  uint64_t slot_free[NSLOT][2];
+  // leader: rank r's decision for tile t is in dec_word[t % RD][r]; rank 0
+  // arrives on dec_full[][0] after writing it, rank 1's st.async completes
+  // 4 bytes on dec_full[][1], armed by the PV issuer
+  uint64_t dec_full[RD][2];
+  uint64_t v_req[NSV];             // each CTA: a V half to load (tile in req_j)
+  uint64_t v_full[NSV];            // leader: both V halves loaded
+  uint64_t v_empty[NSV];           // each CTA: V stage free again
+  uint64_t pv_done[2];             // each CTA: one arrival per PV that read P buffer b
+  int req_j[NSV];                  // each CTA: key block of a V request, -1 = stop
+  int dec_word[RD][2];             // leader: 1 = keep, 0 = skip
+  int sink;                        // leader: target of rank 1's buffer-release stores
+  int dec_done;                    // leader: tiles whose decisions the PV issuer has read
+  // each CTA, between its two test groups: fin[t % NFIN] = t + 1 once tile t
+  // is final, n_kept = kept tiles so far, and the running (m, l) per row
+  // after the last kept tile
+  int fin[NFIN];
+  int n_kept;
+  union {
+    struct {
+      float m[T];
+      float l[T];
+    } st;
+    struct {  // tau = 0: a kept tile's half-row maxima and sums
+      float max[2][T];
+      float sum[2][T];
+    } half;
+  } x;
   uint32_t tmem_slot;
   int abort;
 };
-static_assert(sizeof(Bars) <= 512, "barrier block");
-static_assert(NSK % 2 == 0, "a K stage's tiles must all belong to one issuer");
+static_assert(sizeof(Bars) <= BAR_BYTES, "barrier block");
 
-// OR-vote over the 128 softmax threads on named barrier 1.
-__device__ __forceinline__ int vote_or(int pred) {
+// OR-vote over 128 threads on named barrier ID (a compile-time constant).
+template <int ID>
+__device__ __forceinline__ int vote_or_128(int pred) {
   uint32_t out;
   asm volatile(
       "{\n\t.reg .pred pi, po;\n\t"
       "setp.ne.u32 pi, %1, 0;\n\t"
-      "barrier.cta.red.or.pred po, 1, 128, pi;\n\t"
+      "barrier.cta.red.or.pred po, %2, 128, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(out)
+      : "r"(pred), "n"(ID)
+      : "memory");
+  return (int)out;
+}
+// OR-vote over the 256 test threads on named barrier 3.
+__device__ __forceinline__ int vote_or_256(int pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "barrier.cta.red.or.pred po, 3, 256, pi;\n\t"
       "selp.u32 %0, 1, 0, po;\n\t}\n"
       : "=r"(out)
       : "r"(pred)
       : "memory");
   return (int)out;
 }
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+template <int ID>
+__device__ __forceinline__ void sync_128() {
+  asm volatile("barrier.cta.sync %0, 128;" ::"n"(ID) : "memory");
+}
+__device__ __forceinline__ void sync_256() { asm volatile("barrier.cta.sync 3, 256;" ::: "memory"); }
 
-template <bool VARLEN>
+// Row max of a 128-column S row held in registers (raw scores). Columns past
+// `hi` (the causal mask of a diagonal tile) and below `lo` (keys that do not
+// exist) are excluded. Eight independent max chains.
+__device__ __forceinline__ float row_max128(const uint32_t (&v)[128], int hi, int lo) {
+  const float ninf = -__builtin_huge_valf();
+  float a[8];
+  if (hi >= T - 1 && lo <= 0) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = __uint_as_float(v[k]);
+#pragma unroll
+    for (int e = 8; e < 128; e += 16) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        a[k] = fmax3f(a[k], __uint_as_float(v[e + k]), __uint_as_float(v[e + 8 + k]));
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = ninf;
+#pragma unroll
+    for (int e = 0; e < 128; e += 8) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        a[k] = fmaxf(a[k], (e + k > hi || e + k < lo) ? ninf : __uint_as_float(v[e + k]));
+    }
+  }
+  return fmaxf(fmaxf(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5])), fmaxf(a[6], a[7]));
+}
+
+// The same over a 64-column half row whose tile columns are c0 + e.
+__device__ __forceinline__ float half_row_max(const float (&v)[64], int c0, int hi, int lo) {
+  const float ninf = -__builtin_huge_valf();
+  float a[8];
+  if (c0 + 63 <= hi && c0 >= lo) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = v[k];
+#pragma unroll
+    for (int e = 8; e < 56; e += 16) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) a[k] = fmax3f(a[k], v[e + k], v[e + 8 + k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], v[56 + k]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = ninf;
+#pragma unroll
+    for (int e = 0; e < 64; e += 8) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int c = c0 + e + k;
+        a[k] = fmaxf(a[k], (c > hi || c < lo) ? ninf : v[e + k]);
+      }
+    }
+  }
+  return fmaxf(fmaxf(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5])), fmaxf(a[6], a[7]));
+}
+
+// P = exp2(s * scale_log2 - m) for 8 keys (tile columns col0 .. col0 + 7,
+// masked ones 0) as a bf16 pair hi + lo, stored into row r of the swizzled
+// P buffers; returns the 8 values' float sum.
+__device__ __forceinline__ float p_chunk8(const float* s, int col0, int hi, int lo, float scale_log2,
+                                          float m, uint32_t p_hi, uint32_t p_lo, int r) {
+  uint32_t hw[4], lw[4];
+  float sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    const int col = col0 + e;
+    const bool x0 = col > hi || col < lo, x1 = col + 1 > hi || col + 1 < lo;
+    const float p0 = x0 ? 0.f : exp2f(s[e] * scale_log2 - m);
+    const float p1 = x1 ? 0.f : exp2f(s[e + 1] * scale_log2 - m);
+    sum += p0 + p1;
+    const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+    const float2 hf = __bfloat1622float2(hb);
+    hw[e >> 1] = *reinterpret_cast<const uint32_t*>(&hb);
+    lw[e >> 1] = pack_bf16(p0 - hf.x, p1 - hf.y);
+  }
+  const uint32_t o = sw128_chunk_off(r, col0, T);
+  st_shared_v4(p_hi + o, hw[0], hw[1], hw[2], hw[3]);
+  st_shared_v4(p_lo + o, lw[0], lw[1], lw[2], lw[3]);
+  return sum;
+}
+
+// Scales `ncols` (a multiple of 32) TMEM columns of this thread's lane by a.
+__device__ __forceinline__ void tmem_scale(uint32_t taddr, int ncols, float a) {
+  for (int ch = 0; ch < ncols; ch += 32) {
+    float o[32];
+    tmem_ld32(taddr + ch, o);
+    uint32_t w[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(o[e] * a);
+    tmem_st32(taddr + ch, w);
+  }
+}
+
+// O / l of this thread's row, columns c0 .. c0 + ncols - 1, to bf16 (and
+// float32) global memory.
+__device__ __forceinline__ void store_o(uint32_t t_o, int c0, int ncols, float inv, bool valid,
+                                        __nv_bfloat16* O, float* O32, size_t orow) {
+  for (int ch = 0; ch < ncols; ch += 32) {
+    float o[32];
+    tmem_ld32(t_o + c0 + ch, o);
+    if (!valid) continue;
+    uint4* d4 = reinterpret_cast<uint4*>(O + orow + c0 + ch);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 w;
+      w.x = pack_bf16(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+      w.y = pack_bf16(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+      w.z = pack_bf16(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+      w.w = pack_bf16(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+      d4[q] = w;
+    }
+    if (O32) {
+      float4* d32 = reinterpret_cast<float4*>(O32 + orow + c0 + ch);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        d32[q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv,
+                             o[4 * q + 3] * inv);
+    }
+  }
+}
+
+// Keep bits of one block's row, set from two test groups: each accumulates
+// the bits of its own tiles a word at a time and ORs whole words into the
+// (zeroed) row.
+struct KeepBitsOr {
+  uint32_t* row;
+  uint32_t word;
+  int cur;
+  __device__ __forceinline__ void init(uint32_t* bits, size_t row_off) {
+    row = bits ? bits + row_off : nullptr;
+    word = 0;
+    cur = -1;
+  }
+  __device__ __forceinline__ void set(int j, bool kept) {
+    if (!row) return;
+    const int w = j >> 5;
+    if (w != cur) {
+      if (cur >= 0 && word) atomicOr(&row[cur], word);
+      cur = w;
+      word = 0;
+    }
+    if (kept) word |= 1u << (j & 31);
+  }
+  __device__ __forceinline__ void flush() {
+    if (row && cur >= 0 && word) atomicOr(&row[cur], word);
+    cur = -1;
+  }
+};
+
+template <bool VARLEN, bool DENSE>
 __global__ void __launch_bounds__(NT, 1)
     fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const Params p) {
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  using PL = Plan<DENSE>;
+  constexpr int NSK = PL::NSK, NPB = PL::NPB, SPER = PL::SPER;
+  constexpr uint32_t OFF_Q = PL::OFF_Q, OFF_K = PL::OFF_K, OFF_V = PL::OFF_V, OFF_P = PL::OFF_P,
+                     OFF_BAR = PL::OFF_BAR;
+  constexpr uint32_t REL_TX = 4 * PL::REL_LOCAL;  // bytes of rank 1's releases per tile
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base = smem_raw;
+  // 128-byte swizzled operands need 1024-byte aligned stages; both CTAs of a
+  // cluster have the same offset, so both leave here together if it is not
+  if (smem_u32(base) & 1023u) {
+    if (threadIdx.x == 0) record_layout_error(0x2f0);
+    return;
+  }
   Bars& bars = *reinterpret_cast<Bars*>(base + OFF_BAR);
   volatile int* abort = &bars.abort;
   const uint32_t sbase = smem_u32(base);
@@ -190,10 +436,12 @@ __global__ void __launch_bounds__(NT, 1)
   auto kpos = [&](int k) { return off + T * (k - koff); };
   // the CTA's block takes part in tile t iff the tile is not past its diagonal
   auto part = [&](int t) { return mine && ktop - t <= iX + koff; };
-  // PVs whose V the producers load without a request: the diagonal tiles,
-  // always kept (t = 0 for rank 1's block, t = 1 for rank 0's), or every
-  // tile when nothing is skipped.
+  // PVs whose V the producer loads without a request: the diagonal tiles,
+  // always kept and the first PVs (t = 0 for rank 1's block, t = 1 for rank
+  // 0's), or every tile when nothing is skipped.
   const int npre = p.never_skip ? ntiles : (hasB ? 2 : 1);
+  // S buffer barrier pair member of tile t
+  auto sg = [&](int t) { return t & PL::SGRP_MASK; };
 
   if (tid == 0) {
     mbar_init(smem_u32(&bars.q_full), 1);
@@ -201,20 +449,22 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_init(smem_u32(&bars.k_full[s]), 1);
       mbar_init(smem_u32(&bars.k_empty[s]), 1);
     }
-    for (int u = 0; u < NSLOT; ++u) {
-      mbar_init(smem_u32(&bars.s_full[u]), 1);
-      for (int r = 0; r < 2; ++r) {
-        mbar_init(smem_u32(&bars.dec_keep[u][r]), 1);
-        mbar_init(smem_u32(&bars.dec_skip[u][r]), 1);
+    for (int u = 0; u < NSLOT; ++u)
+      for (int g = 0; g < 2; ++g) {
+        mbar_init(smem_u32(&bars.s_full[u][g]), 1);
+        mbar_init(smem_u32(&bars.slot_free[u][g]), PL::REL_LOCAL + 1);
       }
-      mbar_init(smem_u32(&bars.slot_free[u]), 1);
-    }
+    for (int u = 0; u < RD; ++u)
+      for (int r = 0; r < 2; ++r) mbar_init(smem_u32(&bars.dec_full[u][r]), 1);
     for (int v = 0; v < NSV; ++v) {
       mbar_init(smem_u32(&bars.v_req[v]), 1);
       mbar_init(smem_u32(&bars.v_full[v]), 1);
       mbar_init(smem_u32(&bars.v_empty[v]), 1);
     }
-    mbar_init(smem_u32(&bars.pv_done), 1);
+    for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&bars.pv_done[b]), 1);
+    bars.dec_done = 0;
+    for (int f = 0; f < NFIN; ++f) bars.fin[f] = 0;
+    bars.n_kept = 0;
     bars.abort = 0;
     fence_mbar_init_cluster();
   }
@@ -229,46 +479,67 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t tmem = bars.tmem_slot;
   auto lead = [&](const void* x) { return mapa_rank(smem_u32(x), 0); };
 
-  if (warp == WARP_KPROD) {
-    // -------------------------------------------------------------- K producer
+  if (warp == WARP_PROD) {
+    // ----------------------------------------------------------- producer
+    // One thread serves two queues in one polling loop: the K halves of
+    // tiles 0, 1, ... as stages free up, and the V halves of the PVs in order
+    // (preloaded, or requested by the leader's PV issuer).
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
       if (leader) mbar_expect_tx(smem_u32(&bars.q_full), 2 * Q_BYTES);
       tma_load_3d_pair(sbase + OFF_Q, &tmQ, 0, yq0 + iX * T, zq, lead(&bars.q_full));
       tma_load_3d_pair(sbase + OFF_Q + QH_BYTES, &tmQ, 64, yq0 + iX * T, zq, lead(&bars.q_full));
-      for (int t = 0; t < ntiles; ++t) {
-        const int s = t % NSK;
-        if (t >= NSK && !mbar_wait(smem_u32(&bars.k_empty[s]), ((t / NSK) - 1) & 1, abort, 0x211))
-          break;
-        if (leader) mbar_expect_tx(smem_u32(&bars.k_full[s]), 2 * KH_BYTES);
-        const int row = yk0 + kpos(ktop - t) + 64 * (int)rank;
-        const uint32_t dst = sbase + OFF_K + s * KH_BYTES;
-        tma_load_3d_pair(dst, &tmK, 0, row, zkv, lead(&bars.k_full[s]));
-        tma_load_3d_pair(dst + KH_BLK, &tmK, 64, row, zkv, lead(&bars.k_full[s]));
-      }
-    }
-    __syncwarp();
-  } else if (warp == WARP_VPROD) {
-    // -------------------------------------------------------------- V producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmV);
-      for (int n = 0;; ++n) {
-        const int vs = n % NSV;
-        int j;
-        if (n < npre) {
-          j = ktop - n;  // PV n is tile n
-        } else {
-          if (!mbar_wait_cluster(smem_u32(&bars.v_req[vs]), ((n - npre) / NSV) & 1, abort, 0x212))
-            break;
-          j = *reinterpret_cast<volatile int*>(&bars.req_j[vs]);
-          if (j < 0) break;
+      int tk = 0;   // next K tile
+      int nv = 0;   // next V load (PV number)
+      int vj = -2;  // key block of V load nv once known (-1: stop, -2: not yet)
+      bool vdone = false;
+      unsigned long long t0 = globaltimer_ns();
+      while ((tk < ntiles || !vdone) && !*abort) {
+        bool progress = false;
+        if (tk < ntiles) {
+          const int s = tk % NSK;
+          if (tk < NSK || mbar_test(smem_u32(&bars.k_empty[s]), ((tk / NSK) - 1) & 1)) {
+            if (leader) mbar_expect_tx(smem_u32(&bars.k_full[s]), 2 * KH_BYTES);
+            const int row = yk0 + kpos(ktop - tk) + 64 * (int)rank;
+            const uint32_t dst = sbase + OFF_K + s * KH_BYTES;
+            tma_load_3d_pair(dst, &tmK, 0, row, zkv, lead(&bars.k_full[s]));
+            tma_load_3d_pair(dst + KH_BLK, &tmK, 64, row, zkv, lead(&bars.k_full[s]));
+            ++tk;
+            progress = true;
+          }
         }
-        if (n >= NSV && !mbar_wait(smem_u32(&bars.v_empty[vs]), ((n / NSV) - 1) & 1, abort, 0x213))
+        if (!vdone) {
+          const int vs = nv % NSV;
+          if (vj == -2) {
+            if (nv < npre) {
+              vj = ktop - nv;  // PV nv is tile nv
+            } else if (mbar_test_cluster(smem_u32(&bars.v_req[vs]), ((nv - npre) / NSV) & 1)) {
+              vj = *reinterpret_cast<volatile int*>(&bars.req_j[vs]);
+              if (vj < 0) vdone = true;
+              progress = true;
+            }
+          }
+          if (vj >= 0 &&
+              (nv < NSV || mbar_test(smem_u32(&bars.v_empty[vs]), ((nv / NSV) - 1) & 1))) {
+            if (leader) mbar_expect_tx(smem_u32(&bars.v_full[vs]), 2 * VH_BYTES);
+            tma_load_3d_pair(sbase + OFF_V + vs * VH_BYTES, &tmV, 64 * (int)rank, yk0 + kpos(vj),
+                             zkv, lead(&bars.v_full[vs]));
+            ++nv;
+            vj = -2;
+            progress = true;
+          }
+        }
+        if (progress) {
+          t0 = globaltimer_ns();
+        } else {
+          __nanosleep(32);  // idle: leave the scheduler to the test warps
+        }
+        if (!progress && globaltimer_ns() - t0 > kWaitLimitNs) {
+          if (atomicExch((int*)abort, 1) == 0) record_timeout(0x212);
           break;
-        if (leader) mbar_expect_tx(smem_u32(&bars.v_full[vs]), 2 * VH_BYTES);
-        tma_load_3d_pair(sbase + OFF_V + vs * VH_BYTES, &tmV, 64 * (int)rank, yk0 + kpos(j), zkv,
-                         lead(&bars.v_full[vs]));
+        }
       }
     }
     __syncwarp();
@@ -277,30 +548,46 @@ __global__ void __launch_bounds__(NT, 1)
     if (leader && lane == 0) {
       const int par = warp - WARP_QK0;
       const uint64_t dq = sdesc_sw128(sbase + OFF_Q, 16, 1024);
-      uint64_t dks[NSK];
-#pragma unroll
-      for (int s = 0; s < NSK; ++s) dks[s] = sdesc_sw128(sbase + OFF_K + s * KH_BYTES, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sbase + OFF_K, 16, 1024);
       bool ok = mbar_wait(smem_u32(&bars.q_full), 0, abort, 0x214);
       tc_fence_after();
       for (int t = par; ok && t < ntiles; t += 2) {
         const int u = t % NSLOT, s = t % NSK;
-        if (t >= NSLOT) {
-          ok = mbar_wait_spin(smem_u32(&bars.slot_free[u]), ((t - NSLOT) / NSLOT) & 1, abort, 0x215);
-          if (!ok) break;
-        }
+        // the tile's K and the decision ring usually are ready long before
+        // the S buffer: wait for them first, so that the buffer's release is
+        // the last event before the MMAs
         ok = mbar_wait(smem_u32(&bars.k_full[s]), (t / NSK) & 1, abort, 0x216);
         if (!ok) break;
+        // tile t's decisions go to ring entry t % RD: the PV issuer must have
+        // read that entry's previous tile (t - RD) first
+        if (t >= RD) {
+          ok = wait_counter(&bars.dec_done, t - RD + 1, abort, 0x21c);
+          if (!ok) break;
+        }
+        if (t >= NSLOT) {  // S of tile t - NSLOT read by both CTAs
+          const int tp = t - NSLOT;
+          const uint32_t fb = smem_u32(&bars.slot_free[u][sg(tp)]);
+          mbar_expect_tx(fb, REL_TX);
+          ok = mbar_wait_spin(fb, (tp / SPER) & 1, abort, 0x215);
+          if (!ok) break;
+        }
         tc_fence_after();
-        uint64_t dk = dks[0];
-#pragma unroll
-        for (int q = 1; q < NSK; ++q)
-          if (s == q) dk = dks[q];
+        const uint64_t dk = dk0 + (uint64_t)((s * KH_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_pair(tmem + u * 128, sdesc_kstep(dq, kk, QH_BYTES), sdesc_kstep(dk, kk, KH_BLK),
                    IDESC_QK, kk > 0, 0u, 0u);
-        commit_pair(smem_u32(&bars.s_full[u]), 3);
+        commit_pair(smem_u32(&bars.s_full[u][sg(t)]), 3);
         commit_pair(smem_u32(&bars.k_empty[s]), 3);
+      }
+      // the last NSLOT tiles' buffer releases have no later QK to wait for
+      // them: wait here, so that no store of rank 1 is still on its way to
+      // this CTA's shared memory when the kernel ends
+      for (int t = par; ok && t < ntiles; t += 2) {
+        if (t + NSLOT < ntiles) continue;
+        const uint32_t fb = smem_u32(&bars.slot_free[t % NSLOT][sg(t)]);
+        mbar_expect_tx(fb, REL_TX);
+        ok = mbar_wait(fb, (t / SPER) & 1, abort, 0x21d);
       }
     }
     __syncwarp();
@@ -310,64 +597,52 @@ __global__ void __launch_bounds__(NT, 1)
       uint64_t dvs[NSV];
 #pragma unroll
       for (int v = 0; v < NSV; ++v) dvs[v] = sdesc_sw128(sbase + OFF_V + v * VH_BYTES, VH_BYTES, 1024);
+      const uint64_t dp0 = sdesc_sw128(sbase + OFF_P, 16, 1024);
       int vcount = 0;
       bool ok = true;
-      // parity of the completed phases of dec_keep / dec_skip per slot and
-      // rank (bit 8 * rank)
-      uint32_t nkeep[NSLOT] = {0, 0, 0}, nskip[NSLOT] = {0, 0, 0};
       for (int t = 0; ok && t < ntiles; ++t) {
-        const int u = t % NSLOT;
-        int kr[2];
-        for (int r = 0; r < 2 && ok; ++r) {
-          const uint32_t bk = smem_u32(&bars.dec_keep[u][r]), bs = smem_u32(&bars.dec_skip[u][r]);
-          const uint32_t pk = (nkeep[u] >> (8 * r)) & 1u, ps = (nskip[u] >> (8 * r)) & 1u;
-          const unsigned long long t0 = globaltimer_ns();
-          while (true) {
-            if (mbar_test(bk, pk & 1)) { kr[r] = 1; nkeep[u] ^= 1u << (8 * r); break; }
-            if (mbar_test(bs, ps & 1)) { kr[r] = 0; nskip[u] ^= 1u << (8 * r); break; }
-            if (*abort || globaltimer_ns() - t0 > kWaitLimitNs) {
-              if (atomicExch((int*)abort, 1) == 0) record_timeout(0x217);
-              ok = false;
-              break;
-            }
-          }
-        }
+        const int u = t % RD;
+        const uint32_t ph = (t / RD) & 1;
+        mbar_expect_tx(smem_u32(&bars.dec_full[u][1]), 4);  // rank 1's decision word
+        ok = mbar_wait(smem_u32(&bars.dec_full[u][0]), ph, abort, 0x217) &&
+             mbar_wait(smem_u32(&bars.dec_full[u][1]), ph, abort, 0x21e);
         if (!ok) break;
-        const int k0 = kr[0], k1 = kr[1];
-        if (k0 | k1) {
-          const int vs = vcount % NSV;
-          if (vcount >= npre) {  // ask both V producers for tile t
-            for (uint32_t r = 0; r < 2; ++r) {
-              st_cluster_u32(mapa_rank(smem_u32(&bars.req_j[vs]), r), (uint32_t)(ktop - t));
-              mbar_arrive_cluster(mapa_rank(smem_u32(&bars.v_req[vs]), r));
-            }
+        const volatile int* dw = &bars.dec_word[u][0];
+        const int k0 = dw[0], k1 = dw[1];
+        // entry u is read: its next tile (t + RD) may be issued
+        *reinterpret_cast<volatile int*>(&bars.dec_done) = t + 1;
+        if (!(k0 | k1)) continue;
+        const int vs = vcount % NSV;
+        if (vcount >= npre) {  // ask both producers for tile t's V
+          for (uint32_t r = 0; r < 2; ++r) {
+            st_cluster_u32(mapa_rank(smem_u32(&bars.req_j[vs]), r), (uint32_t)(ktop - t));
+            mbar_arrive_cluster(mapa_rank(smem_u32(&bars.v_req[vs]), r));
           }
-          ok = mbar_wait_spin(smem_u32(&bars.v_full[vs]), (vcount / NSV) & 1, abort, 0x218);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t m0 = k0 ? 0u : 0xffffffffu, m1 = k1 ? 0u : 0xffffffffu;
-          uint64_t dv = dvs[0];
-#pragma unroll
-          for (int q = 1; q < NSV; ++q)
-            if (vs == q) dv = dvs[q];
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-#pragma unroll
-            for (int kk = 0; kk < T / 16; ++kk) {
-              const uint32_t a_t = tmem + u * 128 + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half;
-              mma_pair_ts(tmem + TMEM_O, a_t, dv + (uint64_t)((kk * 2048) >> 4), IDESC_PV, 1u, m0,
-                          m1);
-            }
-          }
-          commit_pair(smem_u32(&bars.v_empty[vs]), 3);
-          commit_pair(smem_u32(&bars.pv_done), (uint16_t)((k0 ? 1 : 0) | (k1 ? 2 : 0)));
-          commit_pair(smem_u32(&bars.slot_free[u]), 1);
-          ++vcount;
-        } else {
-          mbar_arrive(smem_u32(&bars.slot_free[u]));
         }
+        ok = mbar_wait_spin(smem_u32(&bars.v_full[vs]), (vcount / NSV) & 1, abort, 0x218);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t m0 = k0 ? 0u : 0xffffffffu, m1 = k1 ? 0u : 0xffffffffu;
+        uint64_t dv = dvs[0];
+#pragma unroll
+        for (int q = 1; q < NSV; ++q)
+          if (vs == q) dv = dvs[q];
+        // O += P_hi V + P_lo V over the pair (rows of a CTA that skipped
+        // masked); tile t's P is in buffer t % NPB
+        const int pb = t % NPB;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint64_t dp = dp0 + (uint64_t)(((pb * 2 + half) * P_BYTES) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < T / 16; ++kk)
+            mma_pair(tmem + TMEM_O, sdesc_kstep(dp, kk, QH_BYTES), dv + (uint64_t)((kk * 2048) >> 4),
+                     IDESC_PV, 1u, m0, m1);
+        }
+        commit_pair(smem_u32(&bars.v_empty[vs]), 3);
+        commit_pair(smem_u32(&bars.pv_done[pb]), (uint16_t)((k0 ? 1 : 0) | (k1 ? 2 : 0)));
+        ++vcount;
       }
-      // no further V requests: stop both V producers (a request for key block -1)
+      // no further V requests: stop both producers (a request for key block -1)
       if (vcount >= npre) {
         const int vs = vcount % NSV;
         for (uint32_t r = 0; r < 2; ++r) {
@@ -378,21 +653,40 @@ __global__ void __launch_bounds__(NT, 1)
     }
     __syncwarp();
   } else {
-    // ----------------------------------------------------- softmax / test (4 warps)
-    const int r = tid;  // 0..127
-    const int row = iX * T + r;  // row of the chunk; position off + row
+    // ------------------------------------------------ softmax / test (8 warps)
+    const int r = tid & (T - 1);  // row of the block = TMEM lane
+    const int g = tid >> 7;       // test group (tau > 0) or column half (tau = 0)
+    const int row = iX * T + r;   // row of the chunk; position off + row
     // (packed chunks: a row past the packed tensor is never written, whatever
     // the offsets say)
     const bool row_valid = mine && row < Lq && (!VARLEN || yq0 + row < p.total_q);
     const float thr = p.never_skip ? 0.f : (p.log2_tau - __log2f((float)(off + row + 1)));
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t t_o = tmem + lane_base + TMEM_O;
-    auto signal = [&](int u, int keep) {  // thread 0: this CTA's decision for slot u
-      mbar_arrive_remote(keep ? lead(&bars.dec_keep[u][rank]) : lead(&bars.dec_skip[u][rank]));
+    auto signal = [&](int t, int keep) {  // one thread: this CTA's decision for tile t
+      const int u = t % RD;
+      if (leader) {
+        *reinterpret_cast<volatile int*>(&bars.dec_word[u][0]) = keep;
+        mbar_arrive(smem_u32(&bars.dec_full[u][0]));
+      } else {
+        st_async_u32(lead(&bars.dec_word[u][1]), (uint32_t)keep, lead(&bars.dec_full[u][1]));
+      }
     };
+    auto release = [&](int t) {  // lane 0 of each warp: this warp has read tile t's S
+      const uint32_t b = smem_u32(&bars.slot_free[t % NSLOT][sg(t)]);
+      if (leader)
+        mbar_arrive_relaxed(b);
+      else
+        st_async_u32(lead(&bars.sink), 0u, mapa_rank(b, 0));
+    };
+    // trace row of this block: bit k of word k / 32 = key tile k kept
+    const int nw = VARLEN ? p.nw : (nb + 31) >> 5;
+    const size_t brow = (size_t)z * (VARLEN ? p.nbq_max : nb) + iX;
+    if (tid == 0 && mine && p.keep_bits)
+      for (int w = 0; w < nw; ++w) p.keep_bits[brow * nw + w] = 0u;
     // O starts at zero: every PV accumulates (a CTA's first PV may follow
-    // PVs of the peer's tiles).
-    {
+    // PVs of the peer's tiles)
+    if (g == 0) {
       uint32_t zero[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) zero[e] = 0u;
@@ -400,143 +694,235 @@ __global__ void __launch_bounds__(NT, 1)
       for (int ch = 0; ch < 4; ++ch) tmem_st32(t_o + ch * 32, zero);
       tc_fence_before();
     }
+    sync_256();  // O and the trace row zeroed before any decision leaves
+
     float m_ref = kNegInf, l = 0.f;
     // keep iff mraw * scale_log2 - m_ref - log2 l >= thr; cached as a raw
     // score bound, refreshed whenever (m_ref, l) change
     float bound_raw = kNegInf;
-    int n_kept = 0;
-    // trace row of this block: bit k of word k / 32 = key tile k kept
-    const int nw = VARLEN ? p.nw : (nb + 31) >> 5;
-    const size_t brow = (size_t)z * (VARLEN ? p.nbq_max : nb) + iX;
-    KeepBits kb;
-    kb.init(r == 0 && mine ? p.keep_bits : nullptr, brow * nw);
-    if (r == 0 && mine && p.keep_bits)
-      for (int w = (iX + koff) / 32 + 1; w < nw; ++w) p.keep_bits[brow * nw + w] = 0u;
-    softmax_sync();  // O zeroed by every thread before any decision leaves
 
-    for (int t = 0; t < ntiles; ++t) {
-      const int u = t % NSLOT;
-      // Wait for the tile's QK even when not taking part: the decision for
-      // slot u must not run ahead of the slot's previous use.
-      mbar_wait(smem_u32(&bars.s_full[u]), (t / NSLOT) & 1, abort, 0x219);
-      tc_fence_after();
-      if (!part(t)) {
-        if (r == 0) signal(u, 0);
-        continue;
-      }
-      const int j = ktop - t;  // key tile
-      const bool diag = (j == iX + koff);
-      const int lo = VARLEN ? max(0, -kpos(j)) : 0;  // columns below lo: no key
-      const uint32_t t_s = tmem + lane_base + u * 128;
-      // ---- row max of the tile (raw scores: the positive scale commutes)
-      const float mraw = (VARLEN && lo > 0) ? tmem_rowmax128_from(t_s, lo)
-                                            : tmem_rowmax128(t_s, diag, r);
-      const float mt = mraw * p.scale_log2;
-      int want = diag || p.never_skip;
-      if (!want && row_valid) want = mraw >= bound_raw;
-      tc_fence_before();
-      const int keep = vote_or(want);
-      kb.set(j, keep != 0);
-      if (!keep) {
-        if (r == 0) signal(u, 0);
-        continue;
-      }
-      // ---- kept tile ------------------------------------------------------
-      if (n_kept > 0) {  // this CTA's previous PV reads O
-        mbar_wait(smem_u32(&bars.pv_done), (n_kept - 1) & 1, abort, 0x21a);
+    if constexpr (!DENSE) {
+      // ---- two groups, alternate tiles (group g: tiles t = g, g + 2, ...)
+      KeepBitsOr kb;
+      kb.init(r == 0 && mine ? p.keep_bits : nullptr, brow * nw);
+      auto vote = [&](int pred) { return g == 0 ? vote_or_128<1>(pred) : vote_or_128<2>(pred); };
+      auto gsync = [&]() {
+        if (g == 0)
+          sync_128<1>();
+        else
+          sync_128<2>();
+      };
+      auto finalize = [&](int t) {  // one thread, after the group's decision for tile t
+        __threadfence_block();
+        *reinterpret_cast<volatile int*>(&bars.fin[t % NFIN]) = t + 1;
+      };
+      const uint32_t p_hi = sbase + OFF_P, p_lo = p_hi + P_BYTES;
+      for (int t = g; t < ntiles; t += 2) {
+        const int u = t % NSLOT;
+        // Wait for the tile's QK even when not taking part: this CTA's
+        // release of the slot must not run ahead of the slot's previous use.
+        mbar_wait(smem_u32(&bars.s_full[u][sg(t)]), (t / SPER) & 1, abort, 0x219);
         tc_fence_after();
-      }
-      const float m_new = fmaxf(m_ref, mt);
-      const bool first = (n_kept == 0);
-      const bool need = !first && (m_new > m_ref + kRescaleLog2);
-      if (first) {
-        m_ref = m_new;
-      } else if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? exp2f(m_ref - m_new) : 1.f;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          float o[32];
-          tmem_ld32(t_o + ch * 32, o);
-          uint32_t w[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(o[e] * alpha);
-          tmem_st32(t_o + ch * 32, w);
+        if (!part(t)) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) release(t);
+          if (r == 0) {
+            signal(t, 0);
+            finalize(t);
+          }
+          continue;
         }
-        if (need) {
-          l *= alpha;
+        // ---- this thread's S row into registers; the S buffer is free again
+        uint32_t v[128];
+        tmem_ld128(tmem + lane_base + u * 128, v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) release(t);
+        const int j = ktop - t;  // key tile
+        const bool diag = (j == iX + koff);
+        const int lo = VARLEN ? max(0, -kpos(j)) : 0;  // columns below lo: no key
+        const int hi = diag ? r : T - 1;                // columns past hi: masked
+        // ---- row max of the tile (raw scores: the positive scale commutes)
+        const float mraw = row_max128(v, hi, lo);
+        int keep = vote(diag || (row_valid && mraw >= bound_raw));
+        if (keep) {
+          // Every earlier tile must be final (the other group may have kept
+          // tile t - 1, or tile t - 3 after this group last looked): reload
+          // the running state and test again against the current bound.
+          if (t > 0) wait_counter(&bars.fin[(t - 1) % NFIN], t, abort, 0x21f);
+          __threadfence_block();
+          const int nk = *reinterpret_cast<volatile int*>(&bars.n_kept);
+          if (nk > 0) {
+            m_ref = bars.x.st.m[r];
+            l = bars.x.st.l[r];
+            bound_raw = (thr + m_ref + __log2f(l)) / p.scale_log2;
+          }
+          keep = vote(diag || (row_valid && mraw >= bound_raw));
+          if (keep) {
+            const float mt = mraw * p.scale_log2;
+            const float m_new = fmaxf(m_ref, mt);
+            const bool need = nk > 0 && (m_new > m_ref + kRescaleLog2);
+            float alpha = 1.f;
+            if (nk == 0) {
+              m_ref = m_new;
+            } else if (need) {
+              alpha = exp2f(m_ref - m_new);
+              m_ref = m_new;
+            }
+            // the previous kept tile's PV has read P and updated O
+            if (nk > 0) {
+              mbar_wait(smem_u32(&bars.pv_done[0]), (nk - 1) & 1, abort, 0x21a);
+              tc_fence_after();
+            }
+            // P = exp2(s2 - m_ref) as a bf16 pair hi + lo, 8 keys per store
+            float lsum = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 16; ++ch) {
+              float s8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) s8[e] = __uint_as_float(v[ch * 8 + e]);
+              lsum += p_chunk8(s8, ch * 8, hi, lo, p.scale_log2, m_ref, p_hi, p_lo, r);
+            }
+            if (__any_sync(0xffffffffu, need)) tmem_scale(t_o, 128, alpha);  // warp-collective
+            l = l * alpha + lsum;
+            bound_raw = (thr + m_ref + __log2f(l)) / p.scale_log2;
+            bars.x.st.m[r] = m_ref;
+            bars.x.st.l[r] = l;
+            fence_proxy_async_smem();  // P visible to the tensor cores
+            tc_fence_before();
+            gsync();  // every row's P, O rescale and state are in place
+            if (r == 0) {
+              *reinterpret_cast<volatile int*>(&bars.n_kept) = nk + 1;
+              signal(t, 1);
+              finalize(t);
+            }
+            kb.set(j, true);
+            continue;
+          }
+        }
+        kb.set(j, false);
+        if (r == 0) {
+          signal(t, 0);
+          finalize(t);
+        }
+      }
+      kb.flush();
+      sync_256();  // both groups are done: the state is the final one
+      const int nk = *reinterpret_cast<volatile int*>(&bars.n_kept);
+      if (mine && nk > 0) {
+        // ---- epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2 -------------
+        mbar_wait(smem_u32(&bars.pv_done[0]), (nk - 1) & 1, abort, 0x21b);
+        tc_fence_after();
+        m_ref = bars.x.st.m[r];
+        l = bars.x.st.l[r];
+        const size_t orow = VARLEN ? ((size_t)(yq0 + (row_valid ? row : 0)) * p.Hq + zq) * D
+                                   : ((size_t)z * p.L + (row_valid ? row : 0)) * D;
+        store_o(t_o, 64 * g, 64, 1.f / l, row_valid, p.O, p.O32, orow);
+        if (row_valid && g == 0) {
+          const size_t li = VARLEN ? (size_t)zq * p.total_q + yq0 + row : (size_t)z * p.L + row;
+          p.LSE[li] = (m_ref + __log2f(l)) * kLn2;
+        }
+        if (tid == 0 && p.kept_tiles) p.kept_tiles[brow] = nk;
+      }
+    } else {
+      // ---- tau = 0: every warp reads every tile, thread t holds columns
+      // 64 (t / 128) .. + 63 of its row; the halves meet through shared
+      // memory (row max before P, row sum after)
+      const int c0 = 64 * g;
+      const uint32_t t_oh = t_o + c0;
+      KeepBitsOr kb;
+      kb.init(tid == 0 && mine ? p.keep_bits : nullptr, brow * nw);
+      int pcnt[2] = {0, 0};  // this CTA's PVs per P buffer so far
+      auto wait_pbuf = [&](int b) {
+        if (pcnt[b] > 0) {
+          mbar_wait(smem_u32(&bars.pv_done[b]), (pcnt[b] - 1) & 1, abort, 0x21a);
+          tc_fence_after();
+        }
+      };
+      int n_kept = 0;
+      for (int t = 0; t < ntiles; ++t) {
+        const int u = t % NSLOT;
+        mbar_wait(smem_u32(&bars.s_full[u][sg(t)]), (t / SPER) & 1, abort, 0x219);
+        tc_fence_after();
+        if (!part(t)) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) release(t);
+          if (tid == 0) signal(t, 0);
+          continue;
+        }
+        float v[64];
+        tmem_ld64(tmem + lane_base + u * 128 + c0, v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) release(t);
+        const int j = ktop - t;
+        const bool diag = (j == iX + koff);
+        const int lo = VARLEN ? max(0, -kpos(j)) : 0;
+        const int hi = diag ? r : T - 1;
+        const float pmax = half_row_max(v, c0, hi, lo);
+        int want = diag || p.never_skip;
+        if (!want && row_valid) want = pmax >= bound_raw;
+        const int keep = vote_or_256(want);
+        kb.set(j, keep != 0);
+        if (!keep) {
+          if (tid == 0) signal(t, 0);
+          continue;
+        }
+        bars.x.half.max[g][r] = pmax;
+        sync_256();
+        const float mt = fmaxf(bars.x.half.max[0][r], bars.x.half.max[1][r]) * p.scale_log2;
+        const float m_new = fmaxf(m_ref, mt);
+        const bool first = (n_kept == 0);
+        const bool need = !first && (m_new > m_ref + kRescaleLog2);
+        float alpha = 1.f;
+        if (first) {
+          m_ref = m_new;
+        } else if (need) {
+          alpha = exp2f(m_ref - m_new);
           m_ref = m_new;
         }
-      }
-      // ---- P = exp2(s2 - m_ref) as hi + lo bf16 pairs over the S columns:
-      // each 32-column chunk holds 16 columns of P_hi and 16 of P_lo
-      float lsum = 0.f;
+        // P buffer t % NPB is free once this CTA's last PV that read it is done
+        const int pb = t % NPB;
+        wait_pbuf(pb);
+        const uint32_t p_hi = sbase + OFF_P + pb * 2 * P_BYTES, p_lo = p_hi + P_BYTES;
+        float lsum = 0.f;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        float sv[32];
-        tmem_ld32(t_s + ch * 32, sv);
-        uint32_t w[32];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int col = ch * 32 + e;
-          const float p0 = ((diag && col > r) || col < lo) ? 0.f
-                                                           : exp2f(sv[e] * p.scale_log2 - m_ref);
-          const float p1 = ((diag && col + 1 > r) || col + 1 < lo)
-                               ? 0.f
-                               : exp2f(sv[e + 1] * p.scale_log2 - m_ref);
-          lsum += p0 + p1;
-          const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-          const float2 hf = __bfloat1622float2(h);
-          w[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
-          w[16 + (e >> 1)] = pack_bf16(p0 - hf.x, p1 - hf.y);
+        for (int ch = 0; ch < 8; ++ch)
+          lsum += p_chunk8(&v[ch * 8], c0 + ch * 8, hi, lo, p.scale_log2, m_ref, p_hi, p_lo, r);
+        if (__any_sync(0xffffffffu, need)) {  // tcgen05.ld/st are warp-collective
+          // every earlier PV of this CTA has updated O before it is rescaled
+          if (NPB > 1) wait_pbuf(pb ^ 1);
+          tmem_scale(t_oh, 64, alpha);
         }
-        tmem_st32(t_s + ch * 32, w);
+        ++pcnt[pb];
+        bars.x.half.sum[g][r] = lsum;
+        fence_proxy_async_smem();  // P visible to the tensor cores
+        tc_fence_before();
+        sync_256();  // every row's P, O rescale and half sums are in place
+        if (tid == 0) signal(t, 1);
+        l = l * alpha + (bars.x.half.sum[0][r] + bars.x.half.sum[1][r]);
+        ++n_kept;
+        bound_raw = (thr + m_ref + __log2f(l)) / p.scale_log2;
       }
-      l += lsum;
-      ++n_kept;
-      bound_raw = (thr + m_ref + __log2f(l)) / p.scale_log2;
-      tc_fence_before();
-      softmax_sync();  // every row's P and O rescale are in TMEM
-      if (r == 0) signal(u, 1);
-    }
-    kb.flush();
-    if (mine && n_kept > 0) {
-      // ---- epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2 -----------------
-      mbar_wait(smem_u32(&bars.pv_done), (n_kept - 1) & 1, abort, 0x21b);
-      tc_fence_after();
-      const float inv = 1.f / l;
-      const size_t orow = VARLEN ? ((size_t)(yq0 + (row_valid ? row : 0)) * p.Hq + zq) * D
-                                 : ((size_t)z * p.L + (row_valid ? row : 0)) * D;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        float o[32];
-        tmem_ld32(t_o + ch * 32, o);
-        if (row_valid) {
-          uint4* d4 = reinterpret_cast<uint4*>(p.O + orow + ch * 32);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 w;
-            w.x = pack_bf16(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
-            w.y = pack_bf16(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
-            w.z = pack_bf16(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
-            w.w = pack_bf16(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
-            d4[q] = w;
-          }
-          if (p.O32) {
-            float4* d32 = reinterpret_cast<float4*>(p.O32 + orow + ch * 32);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              d32[q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv,
-                                   o[4 * q + 3] * inv);
-          }
+      kb.flush();
+      if (mine && n_kept > 0) {
+        for (int b = 0; b < NPB; ++b) wait_pbuf(b);
+        const size_t orow = VARLEN ? ((size_t)(yq0 + (row_valid ? row : 0)) * p.Hq + zq) * D
+                                   : ((size_t)z * p.L + (row_valid ? row : 0)) * D;
+        store_o(t_o, c0, 64, 1.f / l, row_valid, p.O, p.O32, orow);
+        if (row_valid && g == 0) {
+          const size_t li = VARLEN ? (size_t)zq * p.total_q + yq0 + row : (size_t)z * p.L + row;
+          p.LSE[li] = (m_ref + __log2f(l)) * kLn2;
         }
+        if (tid == 0 && p.kept_tiles) p.kept_tiles[brow] = n_kept;
       }
-      if (row_valid) {
-        const size_t li = VARLEN ? (size_t)zq * p.total_q + yq0 + row : (size_t)z * p.L + row;
-        p.LSE[li] = (m_ref + __log2f(l)) * kLn2;
-      }
-      if (r == 0 && p.kept_tiles) p.kept_tiles[brow] = n_kept;
     }
   }
+  // A CTA that gave up on a wait may still have copies or MMAs in flight:
+  // give them time to land before the CTA's shared memory and TMEM go.
+  if (*abort) drain_in_flight();
   // both CTAs finish every access to the other's shared memory and TMEM
   // before either frees TMEM or exits
   tc_fence_before();

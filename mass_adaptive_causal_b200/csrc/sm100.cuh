@@ -34,6 +34,11 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// Arrive with no memory ordering: for a signal that publishes no data (the
+// arriving thread's reads are already complete).
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -98,6 +103,35 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, vo
       if (atomicExch((int*)abort, 1) == 0) record_timeout(where);
       return false;
     }
+  }
+}
+
+// Bounded wait until a shared-memory counter written by another thread of
+// this CTA reaches `target` (a plain volatile poll: the counter carries no
+// data, it only gates).
+__device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatile int* abort,
+                                             unsigned int where) {
+  const volatile int* c = ctr;
+  if (*c >= target) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (*c >= target) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (atomicExch((int*)abort, 1) == 0) record_timeout(where);
+      return false;
+    }
+  }
+}
+
+// After a wait ran out, copies and MMAs this CTA issued earlier may still be
+// in flight; 20 microseconds lets them land before the CTA releases its
+// shared memory and TMEM.
+__device__ __forceinline__ void drain_in_flight() {
+  const unsigned long long t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < 20000ull) {
   }
 }
 
@@ -282,6 +316,16 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// Asynchronous 32-bit store into a peer CTA's shared memory whose arrival is
+// counted (4 bytes of transaction) on an mbarrier of that same CTA. The
+// storing thread does not wait for it; the receiver's mbarrier phase
+// completes only after the value has landed, so a waiter may read it then.
+__device__ __forceinline__ void st_async_u32(uint32_t remote_addr, uint32_t v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                   remote_addr),
+               "r"(v), "r"(remote_bar)
+               : "memory");
+}
 __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
@@ -295,6 +339,33 @@ __device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity)
       : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait on a local mbarrier whose arrivals may come from the peer CTA
+// (acquire at cluster scope); the thread may sleep inside try_wait, so a
+// warp that waits long does not take issue slots from its neighbours.
+__device__ __forceinline__ bool mbar_wait_cluster_sleep(uint32_t bar, uint32_t parity,
+                                                        volatile int* abort, unsigned int where) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (atomicExch((int*)abort, 1) == 0) record_timeout(where);
+      return false;
+    }
+  }
 }
 // Bounded wait on a local mbarrier whose arrivals may come from the peer CTA
 // (acquire at cluster scope); polls without suspending.
@@ -377,52 +448,6 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
       : "=r"(r[0]),"=r"(r[1]),"=r"(r[2]),"=r"(r[3]),"=r"(r[4]),"=r"(r[5]),"=r"(r[6]),"=r"(r[7]),"=r"(r[8]),"=r"(r[9]),"=r"(r[10]),"=r"(r[11]),"=r"(r[12]),"=r"(r[13]),"=r"(r[14]),"=r"(r[15]),"=r"(r[16]),"=r"(r[17]),"=r"(r[18]),"=r"(r[19]),"=r"(r[20]),"=r"(r[21]),"=r"(r[22]),"=r"(r[23]),"=r"(r[24]),"=r"(r[25]),"=r"(r[26]),"=r"(r[27]),"=r"(r[28]),"=r"(r[29]),"=r"(r[30]),"=r"(r[31]),"=r"(r[32]),"=r"(r[33]),"=r"(r[34]),"=r"(r[35]),"=r"(r[36]),"=r"(r[37]),"=r"(r[38]),"=r"(r[39]),"=r"(r[40]),"=r"(r[41]),"=r"(r[42]),"=r"(r[43]),"=r"(r[44]),"=r"(r[45]),"=r"(r[46]),"=r"(r[47]),"=r"(r[48]),"=r"(r[49]),"=r"(r[50]),"=r"(r[51]),"=r"(r[52]),"=r"(r[53]),"=r"(r[54]),"=r"(r[55]),"=r"(r[56]),"=r"(r[57]),"=r"(r[58]),"=r"(r[59]),"=r"(r[60]),"=r"(r[61]),"=r"(r[62]),"=r"(r[63]),"=r"(r[64]),"=r"(r[65]),"=r"(r[66]),"=r"(r[67]),"=r"(r[68]),"=r"(r[69]),"=r"(r[70]),"=r"(r[71]),"=r"(r[72]),"=r"(r[73]),"=r"(r[74]),"=r"(r[75]),"=r"(r[76]),"=r"(r[77]),"=r"(r[78]),"=r"(r[79]),"=r"(r[80]),"=r"(r[81]),"=r"(r[82]),"=r"(r[83]),"=r"(r[84]),"=r"(r[85]),"=r"(r[86]),"=r"(r[87]),"=r"(r[88]),"=r"(r[89]),"=r"(r[90]),"=r"(r[91]),"=r"(r[92]),"=r"(r[93]),"=r"(r[94]),"=r"(r[95]),"=r"(r[96]),"=r"(r[97]),"=r"(r[98]),"=r"(r[99]),"=r"(r[100]),"=r"(r[101]),"=r"(r[102]),"=r"(r[103]),"=r"(r[104]),"=r"(r[105]),"=r"(r[106]),"=r"(r[107]),"=r"(r[108]),"=r"(r[109]),"=r"(r[110]),"=r"(r[111]),"=r"(r[112]),"=r"(r[113]),"=r"(r[114]),"=r"(r[115]),"=r"(r[116]),"=r"(r[117]),"=r"(r[118]),"=r"(r[119]),"=r"(r[120]),"=r"(r[121]),"=r"(r[122]),"=r"(r[123]),"=r"(r[124]),"=r"(r[125]),"=r"(r[126]),"=r"(r[127])
       : "r"(taddr)
       : "memory");
-}
-
-// Row max over 128 TMEM columns of this thread's lane. With `diag`, columns
-// c > r are excluded (causal mask of the diagonal tile). One load, then eight
-// independent max chains so the reduction's latency is short.
-__device__ __forceinline__ float tmem_rowmax128(uint32_t taddr, bool diag, int r) {
-  uint32_t v[128];
-  tmem_ld128(taddr, v);
-  const float ninf = -__builtin_huge_valf();
-  float a[8];
-  if (!diag) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) a[k] = __uint_as_float(v[k]);
-#pragma unroll
-    for (int e = 8; e < 128; e += 16) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        a[k] = fmax3f(a[k], __uint_as_float(v[e + k]), __uint_as_float(v[e + 8 + k]));
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) a[k] = ninf;
-#pragma unroll
-    for (int e = 0; e < 128; e += 8) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], e + k > r ? ninf : __uint_as_float(v[e + k]));
-    }
-  }
-  return fmaxf(fmaxf(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5])), fmaxf(a[6], a[7]));
-}
-
-// Row max over TMEM columns lo .. 127 of this thread's lane (the columns
-// below lo are keys that do not exist).
-__device__ __forceinline__ float tmem_rowmax128_from(uint32_t taddr, int lo) {
-  uint32_t v[128];
-  tmem_ld128(taddr, v);
-  const float ninf = -__builtin_huge_valf();
-  float a[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) a[k] = ninf;
-#pragma unroll
-  for (int e = 0; e < 128; e += 8) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], e + k < lo ? ninf : __uint_as_float(v[e + k]));
-  }
-  return fmaxf(fmaxf(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5])), fmaxf(a[6], a[7]));
 }
 
 // Byte offset of the 16-byte chunk holding element (row, col) of a bf16
