@@ -28,9 +28,13 @@
 // tests against the running state it last saw: the bound
 // ln tau - ln Lq + m + ln l only grows as tiles are kept, so a tile below an
 // old bound is below the current one. A group that wants to keep a tile
-// first waits until every earlier tile is final, reloads the state the other
-// group may have advanced, tests again, and only then updates the state, so
-// the kept tiles are exactly those of the sequential rule. Each thread holds
+// first waits until every earlier tile is final, reloads the state if the
+// other group has kept a tile since it last looked, tests again, and only
+// then updates the state, so the kept tiles are exactly those of the
+// sequential rule. A skipped tile is marked final with one plain store that
+// also carries its group's keep count; only a kept tile publishes state, with
+// a release store of that count, so no fence sits on the skip path, which
+// nearly every tile takes. Each thread holds
 // its whole S row in registers and releases the S buffer right after the
 // TMEM load. At tau = 0 every tile is kept and the state is sequential, so
 // there the eight test warps instead split each row into two column halves.
@@ -168,11 +172,12 @@ struct Bars {
   int dec_word[RD][2];             // leader: 1 = keep, 0 = skip
   int sink;                        // leader: target of rank 1's buffer-release stores
   int dec_done;                    // leader: tiles whose decisions the PV issuer has read
-  // each CTA, between its two test groups: fin[t % NFIN] = t + 1 once tile t
-  // is final, n_kept = kept tiles so far, and the running (m, l) per row
-  // after the last kept tile
-  int fin[NFIN];
-  int n_kept;
+  // each CTA, between its two test groups. fin[t % NFIN]: tile t is final,
+  // written in one 8-byte store as (t + 1) | (kept tiles of its group so
+  // far) << 32; kcount[g]: group g's kept tiles, a release store after the
+  // group wrote the running (m, l) per row of its latest kept tile
+  unsigned long long fin[NFIN];
+  int kcount[2];
   union {
     struct {
       float m[T];
@@ -220,34 +225,6 @@ __device__ __forceinline__ void sync_128() {
   asm volatile("barrier.cta.sync %0, 128;" ::"n"(ID) : "memory");
 }
 __device__ __forceinline__ void sync_256() { asm volatile("barrier.cta.sync 3, 256;" ::: "memory"); }
-
-// Row max of a 128-column S row held in registers (raw scores). Columns past
-// `hi` (the causal mask of a diagonal tile) and below `lo` (keys that do not
-// exist) are excluded. Eight independent max chains.
-__device__ __forceinline__ float row_max128(const uint32_t (&v)[128], int hi, int lo) {
-  const float ninf = -__builtin_huge_valf();
-  float a[8];
-  if (hi >= T - 1 && lo <= 0) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) a[k] = __uint_as_float(v[k]);
-#pragma unroll
-    for (int e = 8; e < 128; e += 16) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        a[k] = fmax3f(a[k], __uint_as_float(v[e + k]), __uint_as_float(v[e + 8 + k]));
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) a[k] = ninf;
-#pragma unroll
-    for (int e = 0; e < 128; e += 8) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        a[k] = fmaxf(a[k], (e + k > hi || e + k < lo) ? ninf : __uint_as_float(v[e + k]));
-    }
-  }
-  return fmaxf(fmaxf(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5])), fmaxf(a[6], a[7]));
-}
 
 // The same over a 64-column half row whose tile columns are c0 + e.
 __device__ __forceinline__ float half_row_max(const float (&v)[64], int c0, int hi, int lo) {
@@ -463,8 +440,8 @@ __global__ void __launch_bounds__(NT, 1)
     }
     for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&bars.pv_done[b]), 1);
     bars.dec_done = 0;
-    for (int f = 0; f < NFIN; ++f) bars.fin[f] = 0;
-    bars.n_kept = 0;
+    for (int f = 0; f < NFIN; ++f) bars.fin[f] = 0ull;
+    bars.kcount[0] = bars.kcount[1] = 0;
     bars.abort = 0;
     fence_mbar_init_cluster();
   }
@@ -704,7 +681,7 @@ __global__ void __launch_bounds__(NT, 1)
     if constexpr (!DENSE) {
       // ---- two groups, alternate tiles (group g: tiles t = g, g + 2, ...)
       KeepBitsOr kb;
-      kb.init(r == 0 && mine ? p.keep_bits : nullptr, brow * nw);
+      kb.init(r == 64 && mine ? p.keep_bits : nullptr, brow * nw);
       auto vote = [&](int pred) { return g == 0 ? vote_or_128<1>(pred) : vote_or_128<2>(pred); };
       auto gsync = [&]() {
         if (g == 0)
@@ -712,9 +689,17 @@ __global__ void __launch_bounds__(NT, 1)
         else
           sync_128<2>();
       };
+      // kept tiles of this group, and of the other group as of the state
+      // held in (m_ref, l): the state is the latest unless the other group
+      // has kept a tile since
+      int k_own = 0, k_peer = 0;
+      // A tile's bookkeeping is spread over three warps of the group, since
+      // the group's next vote waits for its slowest warp: row 0 publishes
+      // the state, row 32 sends the decision, row 64 marks the tile final
+      // and keeps the trace bits.
       auto finalize = [&](int t) {  // one thread, after the group's decision for tile t
-        __threadfence_block();
-        *reinterpret_cast<volatile int*>(&bars.fin[t % NFIN]) = t + 1;
+        *reinterpret_cast<volatile unsigned long long*>(&bars.fin[t % NFIN]) =
+            ((unsigned long long)(uint32_t)k_own << 32) | (uint32_t)(t + 1);
       };
       const uint32_t p_hi = sbase + OFF_P, p_lo = p_hi + P_BYTES;
       for (int t = g; t < ntiles; t += 2) {
@@ -727,10 +712,8 @@ __global__ void __launch_bounds__(NT, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) release(t);
-          if (r == 0) {
-            signal(t, 0);
-            finalize(t);
-          }
+          if (r == 32) signal(t, 0);
+          if (r == 64) finalize(t);
           continue;
         }
         // ---- this thread's S row into registers; the S buffer is free again
@@ -746,20 +729,27 @@ __global__ void __launch_bounds__(NT, 1)
         // ---- row max of the tile (raw scores: the positive scale commutes)
         const float mraw = row_max128(v, hi, lo);
         int keep = vote(diag || (row_valid && mraw >= bound_raw));
-        if (keep) {
-          // Every earlier tile must be final (the other group may have kept
-          // tile t - 1, or tile t - 3 after this group last looked): reload
-          // the running state and test again against the current bound.
-          if (t > 0) wait_counter(&bars.fin[(t - 1) % NFIN], t, abort, 0x21f);
-          __threadfence_block();
-          const int nk = *reinterpret_cast<volatile int*>(&bars.n_kept);
-          if (nk > 0) {
-            m_ref = bars.x.st.m[r];
-            l = bars.x.st.l[r];
-            bound_raw = (thr + m_ref + __log2f(l)) / p.scale_log2;
+        if (__builtin_expect(keep, 0)) {
+          // Every earlier tile must be final: this group's are, and the other
+          // group's are once its tile t - 1 is (it finalizes in order). If it
+          // kept a tile since this group's state was current, its state is
+          // the latest: load it (acquire) and test again.
+          if (t > 0) {
+            const unsigned long long fw = wait_word64_lo(&bars.fin[(t - 1) % NFIN], t, abort, 0x21f);
+            const int kp = (int)(fw >> 32);
+            if (kp != k_peer) {
+              wait_acquire(&bars.kcount[g ^ 1], kp, abort, 0x220);
+              m_ref = bars.x.st.m[r];
+              l = bars.x.st.l[r];
+              bound_raw = (thr + m_ref + __log2f(l)) / p.scale_log2;
+              k_peer = kp;
+            }
+            // outside the branch, so that every thread of the group meets
+            // the barrier even if a timed-out wait left them disagreeing
+            keep = vote(diag || (row_valid && mraw >= bound_raw));
           }
-          keep = vote(diag || (row_valid && mraw >= bound_raw));
           if (keep) {
+            const int nk = k_own + k_peer;  // kept tiles before tile t
             const float mt = mraw * p.scale_log2;
             const float m_new = fmaxf(m_ref, mt);
             const bool need = nk > 0 && (m_new > m_ref + kRescaleLog2);
@@ -792,24 +782,22 @@ __global__ void __launch_bounds__(NT, 1)
             fence_proxy_async_smem();  // P visible to the tensor cores
             tc_fence_before();
             gsync();  // every row's P, O rescale and state are in place
-            if (r == 0) {
-              *reinterpret_cast<volatile int*>(&bars.n_kept) = nk + 1;
-              signal(t, 1);
-              finalize(t);
-            }
+            ++k_own;
+            if (r == 0) st_release_cta(&bars.kcount[g], k_own);  // publishes the state
+            if (r == 32) signal(t, 1);
+            if (r == 64) finalize(t);
             kb.set(j, true);
             continue;
           }
         }
         kb.set(j, false);
-        if (r == 0) {
-          signal(t, 0);
-          finalize(t);
-        }
+        if (r == 32) signal(t, 0);
+        if (r == 64) finalize(t);
       }
       kb.flush();
       sync_256();  // both groups are done: the state is the final one
-      const int nk = *reinterpret_cast<volatile int*>(&bars.n_kept);
+      const int nk = *reinterpret_cast<volatile int*>(&bars.kcount[0]) +
+                     *reinterpret_cast<volatile int*>(&bars.kcount[1]);
       if (mine && nk > 0) {
         // ---- epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2 -------------
         mbar_wait(smem_u32(&bars.pv_done[0]), (nk - 1) & 1, abort, 0x21b);

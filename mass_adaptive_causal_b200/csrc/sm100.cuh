@@ -126,6 +126,55 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatil
   }
 }
 
+// Release store / acquire load of a shared-memory word at CTA scope: the
+// writes a thread made (or saw through a CTA barrier) before the release are
+// visible to a thread whose acquire load reads the released value.
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+// Bounded wait until the acquire load of a shared counter reaches `target`.
+__device__ __forceinline__ bool wait_acquire(const int* ctr, int target, volatile int* abort,
+                                             unsigned int where) {
+  if (ld_acquire_cta(ctr) >= target) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (ld_acquire_cta(ctr) >= target) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (atomicExch((int*)abort, 1) == 0) record_timeout(where);
+      return false;
+    }
+  }
+}
+// Bounded wait until the low half of a shared 64-bit word (one 8-byte store
+// writes both halves) reaches `target`; returns the word (0 on a timeout).
+__device__ __forceinline__ unsigned long long wait_word64_lo(const unsigned long long* w, int target,
+                                                            volatile int* abort, unsigned int where) {
+  const volatile unsigned long long* c = w;
+  unsigned long long v = *c;
+  if ((int)(uint32_t)v >= target) return v;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i) {
+      v = *c;
+      if ((int)(uint32_t)v >= target) return v;
+    }
+    if (*abort) return 0ull;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (atomicExch((int*)abort, 1) == 0) record_timeout(where);
+      return 0ull;
+    }
+  }
+}
+
 // After a wait ran out, copies and MMAs this CTA issued earlier may still be
 // in flight; 20 microseconds lets them land before the CTA releases its
 // shared memory and TMEM.
@@ -151,6 +200,29 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+// Element-wise add of a shared-memory tile into global memory through a 3-D
+// tensor map (the add happens in L2, in the map's element type); one thread
+// issues it, and it is tracked as a bulk async-group of that thread. Rows
+// past the tensor's extent are not written.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int x,
+                                                  int y, int z) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// This thread's bulk groups have finished reading their shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// This thread's bulk groups have completed (global writes done).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ------------------------------ tcgen05 ------------------------------------
@@ -385,6 +457,42 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   }
 }
 
+// max of three floats (one instruction)
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Row max of a 128-column S row held in registers (raw scores). Columns past
+// `hi` (the causal mask of a diagonal tile) and below `lo` (keys that do not
+// exist) are excluded. Eight independent max chains, so the reduction costs
+// about eight dependent steps rather than sixty-four.
+__device__ __forceinline__ float row_max128(const uint32_t (&v)[128], int hi, int lo) {
+  const float ninf = -__builtin_huge_valf();
+  float a[8];
+  if (__builtin_expect(hi >= 127 && lo <= 0, 1)) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = __uint_as_float(v[k]);
+#pragma unroll
+    for (int e = 8; e < 128; e += 16) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        a[k] = fmax3f(a[k], __uint_as_float(v[e + k]), __uint_as_float(v[e + 8 + k]));
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = ninf;
+#pragma unroll
+    for (int e = 0; e < 128; e += 8) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        a[k] = fmaxf(a[k], (e + k > hi || e + k < lo) ? ninf : __uint_as_float(v[e + k]));
+    }
+  }
+  return fmaxf(fmaxf(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5])), fmaxf(a[6], a[7]));
+}
+
 // 32 consecutive f32 columns of this thread's TMEM lane (32x32b shape, x32),
 // waited for in the same statement so no register is read early.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -432,12 +540,6 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
       : "memory");
 #pragma unroll
   for (int e = 0; e < 64; ++e) v[e] = __uint_as_float(r[e]);
-}
-
-__device__ __forceinline__ float fmax3f(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
 }
 
 // All 128 columns of this thread's TMEM lane in one load (one wait).
