@@ -68,6 +68,24 @@ inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t Z
   return r == CUDA_SUCCESS;
 }
 
+// Float32 tensor [Z][rows][128] seen as 3-D (x = d, y = row, z = Z), box
+// 32 x 128 x 1 (128-byte rows), 128-byte swizzle: the backward's dQ
+// accumulator, target of bulk tensor reductions; rows past `rows` are not
+// written.
+inline bool make_map_f32_acc(CUtensorMap* m, void* base, uint64_t rows, uint64_t Z) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, rows, Z};
+  cuuint64_t strides[2] = {128 * 4, rows * 128 * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  memset(m, 0, sizeof(*m));
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Packed bf16 tensor [tokens][heads][128] seen as 3-D (x = d, y = token,
 // z = head), box 64 x box_rows x 1, 128-byte swizzle; tokens outside
 // [0, tokens) read as zero.
@@ -299,10 +317,11 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
                             void* dK, void* dV, int B, int Hq, int Hkv, int L, float scale,
                             float tau,
                             int32_t* kept, uint32_t* bits, cudaStream_t s) {
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mk64, mdq;
   const int Z = B * Hq, Zkv = B * Hkv;
   if (!make_map(&mq, Q, L, Z) || !make_map(&mk, K, L, Zkv) || !make_map(&mv, V, L, Zkv) ||
-      !make_map(&mdo, dO, L, Z))
+      !make_map(&mdo, dO, L, Z) || !make_map(&mk64, K, L, Zkv, 64) ||
+      !make_map_f32_acc(&mdq, w.dQacc, L, Z))
     return MALA_ERR_CUDA;
   const int nb = (L + bwd100::T - 1) / bwd100::T;
   const int never = tau == 0.f;
@@ -313,17 +332,30 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
     tp.LSE = LSE;
     tp.L = L;
     tp.nb = nb;
-    tp.npairs = (nb + 1) / 2;
+    tp.nclus = (nb + 3) / 4;
     tp.Hq = Hq;
     tp.G = Hq / Hkv;
     tp.scale_log2 = scale * kLog2e;
     tp.log2_tau = log2f(tau);
     tp.bits = tile_bits;
-    // every legal tile's scores are recomputed against the final LSE
+    // every legal tile's scores are recomputed against the final LSE, on
+    // CTA pairs of four query blocks (each CTA loads half of every key tile)
     MALA_CUDA_TRY(cudaFuncSetAttribute(bwdtest::test_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bwdtest::SMEM_BYTES));
-    bwdtest::test_kernel<<<dim3(tp.npairs, Z), bwdtest::NT, bwdtest::SMEM_BYTES, s>>>(mq, mk, tp);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * tp.nclus, Z, 1);
+    cfg.blockDim = dim3(bwdtest::NT, 1, 1);
+    cfg.dynamicSmemBytes = bwdtest::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    MALA_CUDA_TRY(cudaLaunchKernelEx(&cfg, bwdtest::test_kernel, mq, mk64, tp));
   } else if (bits) {
     const size_t nwords = (size_t)Z * nb * ((nb + 31) / 32);
     aux::lower_bits_kernel<<<blocks_for(nwords, 256, 4 * sm_count()), 256, 0, s>>>(bits, nb,
@@ -351,7 +383,7 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
                                      (int)bwd100::SMEM_BYTES));
   // one CTA per (key block, key/value head): dK_j, dV_j sum over its query heads
   bwd100::bwd_bf16_kernel<<<dim3(p.nb, Zkv), bwd100::NT, bwd100::SMEM_BYTES, s>>>(mq, mk, mv,
-                                                                                 mdo, p);
+                                                                                 mdo, mdq, p);
   const size_t n4 = (size_t)Z * L * 128 / 4;
   aux::convert_bf16_v4_kernel<<<blocks_for(n4, 256, 4 * sm_count()), 256, 0, s>>>(
       reinterpret_cast<const float4*>(w.dQacc), reinterpret_cast<uint2*>(dQ), n4);

@@ -24,8 +24,12 @@
 // Shared memory: K_j, V_j, Q_i, dO_i, P^T, dS^T (32 KB each, 128-byte
 // swizzle) + per-query LSE and D, and the list of kept query blocks.
 // dS goes to the tensor cores as a bf16 pair hi + lo (dQ sums rows of dS
-// that cancel); dQ_i is read back from TMEM (query rows in lanes) and added
-// with float4 atomics into a float32 workspace, converted afterwards.
+// that cancel); dQ_i is read back from TMEM (query rows in lanes) into a
+// float32 tile in the then free P^T and dS^T buffers and added into a
+// float32 workspace by four TMA bulk tensor reductions (the adds happen in
+// L2, a 16 KB block per instruction, instead of 4096 float4 atomics from the
+// threads), converted afterwards. The next tile's first MMA waits until the
+// reductions have read the tile.
 #pragma once
 
 #include "sm100.cuh"
@@ -94,7 +98,7 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, uint32_t tadd
 __global__ void __launch_bounds__(NT, 1)
     bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                    const Params p) {
+                    const __grid_constant__ CUtensorMap tmdQ, const Params p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -269,6 +273,9 @@ __global__ void __launch_bounds__(NT, 1)
       }
       mma_commit(bar_mma);
       mma_pend = true;
+      // the previous tile's dQ reduction has read its staging tile (the P^T
+      // and dS^T buffers this tile writes next)
+      bulk_wait_read_all();
     }
     if (mbar_wait(bar_mma, ph_mma, abort, 0x203)) {
       ph_mma ^= 1;
@@ -417,22 +424,24 @@ __global__ void __launch_bounds__(NT, 1)
         q_pend = true;
       }
       ++kept_count;
-      // ---- dQ_i rows (lane = query `row`, this thread's 64 of d) added into
-      // the float32 workspace; tcgen05.ld is warp-collective: every lane
-      // loads, only valid rows add.
-      const int q = i * T + row;
-      float4* dst = reinterpret_cast<float4*>(p.dQacc + ((size_t)z * p.L + (q < p.L ? q : 0)) * D +
-                                              half * 64);
+      // ---- dQ_i (lane = query `row`, this thread's 64 of d) into a float32
+      // staging tile in the P^T and dS^T buffers (free now, 64 KB
+      // contiguous): four blocks of 32 columns, 128 rows of 128 bytes with
+      // the 128-byte swizzle of the reduction's tensor map. Thread 0 adds it
+      // into the workspace with one bulk reduction per block after the
+      // tile's last barrier; rows past L are not written.
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float v[32];
         tmem_ld32(t_st + c * 32, v);
-        if (q < p.L) {
+        const uint32_t blk = pta + (uint32_t)(2 * half + c) * 16384u + (uint32_t)row * 128u;
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            atomicAdd(dst + c * 8 + e, make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]));
-        }
+        for (int q = 0; q < 8; ++q)
+          st_shared_v4(blk + ((uint32_t)(q ^ (row & 7)) << 4), __float_as_uint(v[4 * q]),
+                       __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]),
+                       __float_as_uint(v[4 * q + 3]));
       }
+      fence_proxy_async_smem();  // the staging tile visible to the bulk copy
     }
     if (has_next) {
       if (half == 0)
@@ -446,6 +455,11 @@ __global__ void __launch_bounds__(NT, 1)
     // the next tile once every thread is here
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) {
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) tma_reduce_add_3d(&tmdQ, pta + cb * 16384u, cb * 32, i * T, z);
+      bulk_commit_group();
+    }
     }
   }
   if (tid == 0 && p.kept_tiles) p.kept_tiles[(size_t)z * p.nb + j] = kept_count - kept_before;
@@ -454,6 +468,7 @@ __global__ void __launch_bounds__(NT, 1)
   // kept; anything on the error path) land before the CTA releases its
   // shared memory and TMEM
   if (tid == 0) {
+    bulk_wait_all();  // every dQ reduction of this CTA has landed
     if (kv_pend) mbar_settle(bar_kv, 0);
     if (!ok) {
       if (q_pend) mbar_settle(bar_q, ph_q);
