@@ -630,6 +630,133 @@ def tau_study(args):
 
 
 # ---------------------------------------------------------------------------
+# matched-work policy study (matched_8k): at the per-block tile budget of the
+# rule's own GPU keep set, other allocations of the same number of tiles are
+# compared by the dense probability mass they leave out and by their output
+# error against dense attention (MassAlloc Attention; jaehun.me review,
+# "Matched-work study", Table 1; agihunt.info summary, matched-work paragraph)
+# ---------------------------------------------------------------------------
+# calibration draws of the head-position policy: sequence indices
+# CAL_SEQ0 + H k + h of the same config (independent streams, never a
+# benchmarked sequence)
+CAL_SEQ0 = 500
+N_CAL = 2
+POLICIES = ("mala", "position_static", "head_position_static", "per_instance_oracle")
+
+
+def bf16_round(a):
+    """float64 -> nearest bfloat16 -> float64 (the inputs the kernels see)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).double().numpy()
+
+
+def dense_row_tile_mass(Q, K, tile, scale):
+    """Host float64 analysis: dense causal softmax probabilities P (L, L) of
+    one slice and, per row r and key tile j, the probability row r puts on
+    tile j's keys (L, nb)."""
+    L = Q.shape[0]
+    S = (Q @ K.T) * scale
+    S[np.arange(L)[None, :] > np.arange(L)[:, None]] = -np.inf
+    S -= S.max(axis=1, keepdims=True)
+    P = np.exp(S)
+    P /= P.sum(axis=1, keepdims=True)
+    nb = (L + tile - 1) // tile
+    Pp = np.zeros((L, nb * tile))
+    Pp[:, :L] = P
+    return P, Pp.reshape(L, nb, tile).sum(axis=2)
+
+
+def block_mass(row_mass, tile):
+    """(L, nb) per-row tile mass -> (nb, nb) summed over each query block."""
+    L, nb = row_mass.shape
+    pad = np.zeros((nb * tile, nb))
+    pad[:L] = row_mass
+    return pad.reshape(nb, tile, nb).sum(axis=1)
+
+
+def position_static_keep(counts):
+    """Per query block i: the diagonal tile, the first (sink) tile, then the
+    nearest earlier tiles, counts[i] of them; the same for every input."""
+    nb = len(counts)
+    keep = np.zeros((nb, nb), np.uint8)
+    for i in range(nb):
+        order = [i] + ([0] if i > 0 else []) + list(range(i - 1, 0, -1))
+        keep[i, order[:counts[i]]] = 1
+    return keep
+
+
+def top_keep(score, counts):
+    """Per query block i: the counts[i] legal tiles of largest score."""
+    nb = len(counts)
+    keep = np.zeros((nb, nb), np.uint8)
+    for i in range(nb):
+        order = np.argsort(-score[i, :i + 1], kind="stable")
+        keep[i, order[:counts[i]]] = 1
+    return keep
+
+
+def restricted_output(P, V, keep, tile):
+    """Softmax restricted to the kept tiles, times V, and the per-row mass
+    left out."""
+    L = P.shape[0]
+    blk = np.arange(L) // tile
+    Pk = np.where(keep[blk][:, blk].astype(bool), P, 0.0)
+    kept = Pk.sum(axis=1)
+    return (Pk @ V) / kept[:, None], 1.0 - kept
+
+
+def policy_study(args):
+    """One JSON line: per allocation policy, the mean omitted mass and the
+    output rel-L2 against dense attention, on matched_8k (8 heads, L=8192),
+    each policy given the rule's per-block tile counts from mala_fwd's keep
+    bits. Dense probabilities are host float64 analysis of the bf16 inputs."""
+    import torch
+    import mass_adaptive_causal_b200 as mala
+    torch.cuda.set_device(0)
+    cfg = synth.CONFIGS["matched_8k"]
+    L, H, d, tile = cfg.L, cfg.H, cfg.d, cfg.tile
+    scale = 1.0 / np.sqrt(d)
+    x = synth.prefill_inputs(cfg, with_grad=False)
+    host = {n: bf16_round(x[n]) for n in ("Q", "K", "V")}
+    dev = {n: torch.from_numpy(host[n]).to(torch.bfloat16).cuda() for n in host}
+    O, LSE, kept, bits = mala.mala_fwd(dev["Q"], dev["K"], dev["V"], tau=1.0, trace=True)
+    mala.mala_check()
+    nb = (L + tile - 1) // tile
+    keep_gpu = mala.unpack_bits(bits, nb)
+    O_gpu = O.float().cpu().numpy()
+    u = synth.unit_vector(cfg.config_seed, d)
+    acc = {n: {"omitted_mass_mean": 0.0, "out_rel_l2": 0.0} for n in POLICIES}
+    kernel_err = 0.0
+    t0 = time.time()
+    for h in range(H):
+        Q, K, V = host["Q"][0, h], host["K"][0, h], host["V"][0, h]
+        P, rm = dense_row_tile_mass(Q, K, tile, scale)
+        cal = np.zeros((nb, nb))
+        for k in range(N_CAL):
+            sq = synth.prefill_sequence(cfg.config_seed, CAL_SEQ0 + H * k + h, L, d, cfg.rho,
+                                        cfg.n_pairs, u, with_grad=False)
+            _, rmc = dense_row_tile_mass(bf16_round(sq["Q"]), bf16_round(sq["K"]), tile, scale)
+            cal += block_mass(rmc, tile)
+        kg = keep_gpu[0, h]
+        counts = kg.sum(axis=1)
+        keeps = {"mala": kg, "position_static": position_static_keep(counts),
+                 "head_position_static": top_keep(cal, counts),
+                 "per_instance_oracle": top_keep(block_mass(rm, tile), counts)}
+        O_dense = P @ V
+        nrm = np.linalg.norm(O_dense)
+        for name, kp in keeps.items():
+            assert np.array_equal(kp.sum(axis=1), counts)
+            Oz, om = restricted_output(P, V, kp, tile)
+            acc[name]["omitted_mass_mean"] += om.mean() / H
+            acc[name]["out_rel_l2"] += np.linalg.norm(Oz - O_dense) / nrm / H
+        kernel_err += np.linalg.norm(O_gpu[0, h] - O_dense) / nrm / H
+    print(json.dumps({"study": "matched_work", "workload": "matched_8k", "heads": H, "L": L,
+                      "slots_per_query": retained_pairs(bits, L, tile) / (H * L),
+                      "policies": acc, "mala_kernel_out_rel_l2": kernel_err,
+                      "calibration_draws": N_CAL, "host_seconds": time.time() - t0}), flush=True)
+
+
+# ---------------------------------------------------------------------------
 # per-workload report: configurations 0-2 (the tiny float32 case, the
 # matched-work shape and the length sweep), each at tau=1 and tau=0
 # ---------------------------------------------------------------------------
@@ -795,13 +922,16 @@ def main():
     ap.add_argument("--tau", type=float, default=1.0, help="tau of --profile")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the per-workload report of configurations 0-2")
-    ap.add_argument("--study", choices=["tau"], default=None,
-                    help="tau sweep: slots, omitted mass and error against dense, one JSON line")
+    ap.add_argument("--study", choices=["tau", "policy"], default=None,
+                    help="tau: sweep of tau (slots, omitted mass, error against dense); policy: "
+                         "matched-work allocation policies on matched_8k; one JSON line each")
     args = ap.parse_args()
     if args.profile:
         return profile_case(args)
     if args.study == "tau":
         return tau_study(args)
+    if args.study == "policy":
+        return policy_study(args)
     args.warmup = max(3, args.warmup)
 
     rank = int(os.environ.get("RANK", "0"))
