@@ -289,15 +289,29 @@ __global__ void __launch_bounds__(NT, 1)
     {
       // P^T row (key `row`) over this thread's 64 queries, fp32 kept for dS
       float pr[T / 2];
+      // an interior tile (below the diagonal, every query row < L) masks nothing
+      const bool interior = !diag && (i + 1) * T <= p.L;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float s[32];
         tmem_ld32(t_st + c * 32, s);
+        const float4* l4 = reinterpret_cast<const float4*>(lse_c + half * 64 + c * 32);
+        if (interior) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int qc = half * 64 + c * 32 + e;
-          const bool legal = (!diag || qc >= row) && (i * T + qc) < p.L;
-          pr[c * 32 + e] = legal ? exp2f(s[e] * p.scale_log2 - lse_c[qc]) : 0.f;
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 lv = l4[e4];
+            pr[c * 32 + 4 * e4 + 0] = ex2_approx(s[4 * e4 + 0] * p.scale_log2 - lv.x);
+            pr[c * 32 + 4 * e4 + 1] = ex2_approx(s[4 * e4 + 1] * p.scale_log2 - lv.y);
+            pr[c * 32 + 4 * e4 + 2] = ex2_approx(s[4 * e4 + 2] * p.scale_log2 - lv.z);
+            pr[c * 32 + 4 * e4 + 3] = ex2_approx(s[4 * e4 + 3] * p.scale_log2 - lv.w);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int qc = half * 64 + c * 32 + e;
+            const bool legal = (!diag || qc >= row) && (i * T + qc) < p.L;
+            pr[c * 32 + e] = legal ? ex2_approx(s[e] * p.scale_log2 - lse_c[qc]) : 0.f;
+          }
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -359,15 +373,18 @@ __global__ void __launch_bounds__(NT, 1)
       for (int c = 0; c < 2; ++c) {
         float dp[32];
         tmem_ld32(t_dpt + c * 32, dp);
+        // D of the tile's query columns half * 64 + c * 32 + ..., four at a time
+        const float4* d4 = reinterpret_cast<const float4*>(dd_c + half * 64 + c * 32);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t whi[4], wlo[4];
+          const float4 da = d4[2 * q], db = d4[2 * q + 1];
+          const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
             const int lc = c * 32 + q * 8 + e;  // this thread's column
-            const int qc = half * 64 + lc;      // the tile's query column
-            const float a = pr[lc] * (dp[q * 8 + e] - dd_c[qc]) * p.scale;
-            const float b = pr[lc + 1] * (dp[q * 8 + e + 1] - dd_c[qc + 1]) * p.scale;
+            const float a = pr[lc] * (dp[q * 8 + e] - dv[e]) * p.scale;
+            const float b = pr[lc + 1] * (dp[q * 8 + e + 1] - dv[e + 1]) * p.scale;
             const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
             const float2 hf = __bfloat1622float2(h);
             whi[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);

@@ -207,19 +207,6 @@ __device__ __forceinline__ int vote_or_128(int pred) {
       : "memory");
   return (int)out;
 }
-// OR-vote over the 256 test threads on named barrier 3.
-__device__ __forceinline__ int vote_or_256(int pred) {
-  uint32_t out;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "barrier.cta.red.or.pred po, 3, 256, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}\n"
-      : "=r"(out)
-      : "r"(pred)
-      : "memory");
-  return (int)out;
-}
 template <int ID>
 __device__ __forceinline__ void sync_128() {
   asm volatile("barrier.cta.sync %0, 128;" ::"n"(ID) : "memory");
@@ -256,8 +243,10 @@ __device__ __forceinline__ float half_row_max(const float (&v)[64], int c0, int 
 }
 
 // P = exp2(s * scale_log2 - m) for 8 keys (tile columns col0 .. col0 + 7,
-// masked ones 0) as a bf16 pair hi + lo, stored into row r of the swizzled
-// P buffers; returns the 8 values' float sum.
+// masked ones 0; MASKED = false: the tile has no masked column) as a bf16
+// pair hi + lo, stored into row r of the swizzled P buffers; returns the 8
+// values' float sum.
+template <bool MASKED>
 __device__ __forceinline__ float p_chunk8(const float* s, int col0, int hi, int lo, float scale_log2,
                                           float m, uint32_t p_hi, uint32_t p_lo, int r) {
   uint32_t hw[4], lw[4];
@@ -265,9 +254,10 @@ __device__ __forceinline__ float p_chunk8(const float* s, int col0, int hi, int 
 #pragma unroll
   for (int e = 0; e < 8; e += 2) {
     const int col = col0 + e;
-    const bool x0 = col > hi || col < lo, x1 = col + 1 > hi || col + 1 < lo;
-    const float p0 = x0 ? 0.f : exp2f(s[e] * scale_log2 - m);
-    const float p1 = x1 ? 0.f : exp2f(s[e + 1] * scale_log2 - m);
+    const bool x0 = MASKED && (col > hi || col < lo);
+    const bool x1 = MASKED && (col + 1 > hi || col + 1 < lo);
+    const float p0 = x0 ? 0.f : ex2_approx(s[e] * scale_log2 - m);
+    const float p1 = x1 ? 0.f : ex2_approx(s[e + 1] * scale_log2 - m);
     sum += p0 + p1;
     const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
     const float2 hf = __bfloat1622float2(hb);
@@ -772,7 +762,7 @@ __global__ void __launch_bounds__(NT, 1)
               float s8[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) s8[e] = __uint_as_float(v[ch * 8 + e]);
-              lsum += p_chunk8(s8, ch * 8, hi, lo, p.scale_log2, m_ref, p_hi, p_lo, r);
+              lsum += p_chunk8<true>(s8, ch * 8, hi, lo, p.scale_log2, m_ref, p_hi, p_lo, r);
             }
             if (__any_sync(0xffffffffu, need)) tmem_scale(t_o, 128, alpha);  // warp-collective
             l = l * alpha + lsum;
@@ -850,14 +840,9 @@ __global__ void __launch_bounds__(NT, 1)
         const int lo = VARLEN ? max(0, -kpos(j)) : 0;
         const int hi = diag ? r : T - 1;
         const float pmax = half_row_max(v, c0, hi, lo);
-        int want = diag || p.never_skip;
-        if (!want && row_valid) want = pmax >= bound_raw;
-        const int keep = vote_or_256(want);
-        kb.set(j, keep != 0);
-        if (!keep) {
-          if (tid == 0) signal(t, 0);
-          continue;
-        }
+        // this instantiation runs only with tau = 0: every legal tile is
+        // kept, so there is nothing to vote on
+        kb.set(j, true);
         bars.x.half.max[g][r] = pmax;
         sync_256();
         const float mt = fmaxf(bars.x.half.max[0][r], bars.x.half.max[1][r]) * p.scale_log2;
@@ -876,9 +861,17 @@ __global__ void __launch_bounds__(NT, 1)
         wait_pbuf(pb);
         const uint32_t p_hi = sbase + OFF_P + pb * 2 * P_BYTES, p_lo = p_hi + P_BYTES;
         float lsum = 0.f;
+        if (diag || lo > 0) {
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          lsum += p_chunk8(&v[ch * 8], c0 + ch * 8, hi, lo, p.scale_log2, m_ref, p_hi, p_lo, r);
+          for (int ch = 0; ch < 8; ++ch)
+            lsum += p_chunk8<true>(&v[ch * 8], c0 + ch * 8, hi, lo, p.scale_log2, m_ref, p_hi,
+                                   p_lo, r);
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            lsum += p_chunk8<false>(&v[ch * 8], c0 + ch * 8, hi, lo, p.scale_log2, m_ref, p_hi,
+                                    p_lo, r);
+        }
         if (__any_sync(0xffffffffu, need)) {  // tcgen05.ld/st are warp-collective
           // every earlier PV of this CTA has updated O before it is rescaled
           if (NPB > 1) wait_pbuf(pb ^ 1);
@@ -892,7 +885,6 @@ __global__ void __launch_bounds__(NT, 1)
         if (tid == 0) signal(t, 1);
         l = l * alpha + (bars.x.half.sum[0][r] + bars.x.half.sum[1][r]);
         ++n_kept;
-        bound_raw = (thr + m_ref + __log2f(l)) / p.scale_log2;
       }
       kb.flush();
       if (mine && n_kept > 0) {

@@ -457,6 +457,15 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   }
 }
 
+// 2^x by the hardware's approximate exponential (PTX ex2.approx.ftz.f32:
+// relative error near 2^-22, subnormal results flushed to zero), one
+// instruction; the per-element exponentials of P use it.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // max of three floats (one instruction)
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   float d;
