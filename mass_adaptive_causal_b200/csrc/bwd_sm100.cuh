@@ -47,7 +47,7 @@ constexpr uint32_t TILE_BYTES = T * D * 2;
 constexpr uint32_t HALF_BYTES = T * 64 * 2;
 constexpr int LIST_CHUNK = 1024;  // query blocks listed per round
 constexpr int LIST_ROUNDS = LIST_CHUNK / NT;
-constexpr uint32_t SMEM_BYTES = 6 * TILE_BYTES + 1024 /*align*/ + 2048 /*LSE, D*/ + 64 /*bars*/ +
+constexpr uint32_t SMEM_BYTES = 6 * TILE_BYTES + 1024 /*align*/ + 2048 /*LSE, D*/ + 128 /*bars*/ +
                                 LIST_CHUNK * 4 + LIST_ROUNDS * NWARP * 4;
 constexpr uint32_t TMEM_COLS = 512;
 // S^T, dP^T: A = K_j or V_j (K-major over d), B = Q_i or dO_i (K-major over d)
@@ -113,9 +113,9 @@ __global__ void __launch_bounds__(NT, 1)
   float* lse_s = reinterpret_cast<float*>(base + 6 * TILE_BYTES);  // [2][128]
   float* dd_s = lse_s + 2 * T;                                      // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(dd_s + 2 * T);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* list = reinterpret_cast<int*>(bars + 8);  // [LIST_CHUNK]
+  int* list = reinterpret_cast<int*>(bars + 16);  // [LIST_CHUNK]
   int* wcount = list + LIST_CHUNK;               // [LIST_ROUNDS][NWARP]
 
   const int tid = threadIdx.x;
@@ -133,13 +133,21 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t bar_kv = smem_u32(&bars[0]);
   const uint32_t bar_q = smem_u32(&bars[1]);
   const uint32_t bar_do = smem_u32(&bars[2]);
-  const uint32_t bar_mma = smem_u32(&bars[3]);
+  // one completion per tile each: S^T; dP^T and dV; dK; dQ (a commit
+  // covers every earlier MMA of the issuing thread)
+  const uint32_t bar_s = smem_u32(&bars[3]);
+  const uint32_t bar_dv = smem_u32(&bars[4]);
+  const uint32_t bar_dk = smem_u32(&bars[5]);
+  const uint32_t bar_dq = smem_u32(&bars[6]);
 
   if (tid == 0) {
     mbar_init(bar_kv, 1);
     mbar_init(bar_q, 1);
     mbar_init(bar_do, 1);
-    mbar_init(bar_mma, 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_dv, 1);
+    mbar_init(bar_dk, 1);
+    mbar_init(bar_dq, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -169,8 +177,15 @@ __global__ void __launch_bounds__(NT, 1)
   }
   // Phases and copies/MMAs in flight; thread 0 issues every copy and MMA,
   // so its own view is the one that the exit path settles.
-  uint32_t ph_q = 0, ph_do = 0, ph_mma = 0;
+  uint32_t ph_q = 0, ph_do = 0, ph_s = 0, ph_dv = 0, ph_dk = 0, ph_dq = 0;
   bool kv_pend = true, q_pend = false, do_pend = false, mma_pend = false;
+  uint32_t pend_bar = 0, pend_ph = 0;  // thread 0: the last barrier committed
+  auto commit = [&](uint32_t bar, uint32_t ph) {
+    mma_commit(bar);
+    pend_bar = bar;
+    pend_ph = ph;
+    mma_pend = true;
+  };
   bool kv_ready = false;
   int kept_count = 0;
   int tcount = 0;  // tiles done by this CTA: picks the LSE / D buffer
@@ -262,7 +277,8 @@ __global__ void __launch_bounds__(NT, 1)
       ok = false;
     }
     if (__syncthreads_or(!ok)) { ok = false; break; }
-    // ---- S^T = K_j Q_i^T -----------------------------------------------------
+    // ---- S^T = K_j Q_i^T; then dP^T = V_j dO_i^T, which needs no P and runs
+    // while the threads form P
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
@@ -271,15 +287,26 @@ __global__ void __launch_bounds__(NT, 1)
         mma_bf16(tmem, sdesc_sw128(ka + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024),
                  IDESC_KQ, kk > 0);
       }
-      mma_commit(bar_mma);
-      mma_pend = true;
+      commit(bar_s, ph_s);
+      if (mbar_wait(bar_do, ph_do, abort, 0x204)) {
+        ph_do ^= 1;
+        do_pend = false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          mma_bf16(tmem + 128, sdesc_sw128(va + off, 16, 1024), sdesc_sw128(da + off, 16, 1024),
+                   IDESC_KQ, kk > 0);
+        }
+      } else {
+        ok = false;
+      }
       // the previous tile's dQ reduction has read its staging tile (the P^T
       // and dS^T buffers this tile writes next)
       bulk_wait_read_all();
     }
-    if (mbar_wait(bar_mma, ph_mma, abort, 0x203)) {
-      ph_mma ^= 1;
-      mma_pend = false;
+    if (mbar_wait(bar_s, ph_s, abort, 0x203)) {
+      ph_s ^= 1;
     } else {
       ok = false;
     }
@@ -323,22 +350,10 @@ __global__ void __launch_bounds__(NT, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      if (mbar_wait(bar_do, ph_do, abort, 0x204)) {
-        ph_do ^= 1;
-        do_pend = false;
-      } else {
-        ok = false;
-      }
-      if (__syncthreads_or(!ok)) { ok = false; break; }
-      // ---- dP^T = V_j dO_i^T ; dV += P^T dO_i ---------------------------------
+      __syncthreads();
+      // ---- dV += P^T dO_i --------------------------------------------------------
       if (tid == 0) {
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          mma_bf16(tmem + 128, sdesc_sw128(va + off, 16, 1024), sdesc_sw128(da + off, 16, 1024),
-                   IDESC_KQ, kk > 0);
-        }
 #pragma unroll
         for (int kk = 0; kk < T / 16; ++kk) {
           const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
@@ -346,12 +361,10 @@ __global__ void __launch_bounds__(NT, 1)
                    sdesc_sw128(da + kk * 2048, HALF_BYTES, 1024), IDESC_ACC,
                    (kept_count > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar_mma);
-        mma_pend = true;
+        commit(bar_dv, ph_dv);
       }
-      if (mbar_wait(bar_mma, ph_mma, abort, 0x205)) {
-        ph_mma ^= 1;
-        mma_pend = false;
+      if (mbar_wait(bar_dv, ph_dv, abort, 0x205)) {  // dP^T and dV done
+        ph_dv ^= 1;
       } else {
         ok = false;
       }
@@ -398,7 +411,9 @@ __global__ void __launch_bounds__(NT, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
-      // ---- dK += (hi + lo)^T Q_i ; dQ_i = (hi + lo) K_j (into the S^T columns)
+      // ---- dK += (hi + lo)^T Q_i, then dQ_i = (hi + lo) K_j (into the S^T
+      // columns); once dK is done Q_i is free and the next tile's Q loads
+      // while the dQ products run
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
@@ -412,6 +427,7 @@ __global__ void __launch_bounds__(NT, 1)
                      (kept_count > 0 || part > 0 || kk > 0) ? 1u : 0u);
           }
         }
+        commit(bar_dk, ph_dk);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
           const uint32_t src = part == 0 ? sta : pta;
@@ -422,24 +438,27 @@ __global__ void __launch_bounds__(NT, 1)
                      (part > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        mma_commit(bar_mma);
-        mma_pend = true;
+        commit(bar_dq, ph_dq);
+        if (mbar_wait(bar_dk, ph_dk, abort, 0x207)) {
+          ph_dk ^= 1;
+          if (has_next) {  // Q_i has been read
+            mbar_expect_tx(bar_q, TILE_BYTES);
+            tma_load_3d(qa, &tmQ, 0, inext * T, z, bar_q);
+            tma_load_3d(qa + HALF_BYTES, &tmQ, 64, inext * T, z, bar_q);
+            q_pend = true;
+          }
+        } else {
+          ok = false;
+        }
       }
-      if (mbar_wait(bar_mma, ph_mma, abort, 0x206)) {
-        ph_mma ^= 1;
-        mma_pend = false;
+      if (mbar_wait(bar_dq, ph_dq, abort, 0x206)) {
+        ph_dq ^= 1;
+        mma_pend = false;  // every MMA of the tile has completed
       } else {
         ok = false;
       }
       if (__syncthreads_or(!ok)) { ok = false; break; }
       tc_fence_after();
-      // Q_i has been read: the next tile's Q goes into its buffer now
-      if (tid == 0 && has_next) {
-        mbar_expect_tx(bar_q, TILE_BYTES);
-        tma_load_3d(qa, &tmQ, 0, inext * T, z, bar_q);
-        tma_load_3d(qa + HALF_BYTES, &tmQ, 64, inext * T, z, bar_q);
-        q_pend = true;
-      }
       ++kept_count;
       // ---- dQ_i (lane = query `row`, this thread's 64 of d) into a float32
       // staging tile in the P^T and dS^T buffers (free now, 64 KB
@@ -490,7 +509,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (!ok) {
       if (q_pend) mbar_settle(bar_q, ph_q);
       if (do_pend) mbar_settle(bar_do, ph_do);
-      if (mma_pend) mbar_settle(bar_mma, ph_mma);
+      if (mma_pend) mbar_settle(pend_bar, pend_ph);
     }
   }
 
