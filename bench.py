@@ -300,10 +300,13 @@ def count_launches(fn):
     import torch
     from torch.profiler import ProfilerActivity, profile
     torch.cuda.synchronize()
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        fn()
-        torch.cuda.synchronize()
-    names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    try:
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            fn()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    except Exception:  # no activity trace (e.g. another CUPTI client such as ncu)
+        return None, []
     ours = [n for n in names if any(k in n for k in ("fwd2::", "bwd100::", "bwdtest::", "dec::",
                                                           "aux::", "simt::"))]
     return len(ours), sorted(set(n.split("(")[0] for n in ours))
@@ -1021,7 +1024,8 @@ def main():
         "decode_kept_tile_frac": work["decode_kept_tiles"] / work["decode_tiles"],
         "roofline": roof, "roofline_bwd": roof_bwd, "roofline_decode": roof_dec,
         "clocks": clocks,
-        "gpu_launches": args.steps * work["launches_per_step"],
+        "gpu_launches": (args.steps * work["launches_per_step"]
+                         if work["launches_per_step"] is not None else None),
         "gpu_launches_per_step": work["launches_per_step"], "kernels": work["kernels"],
     }
     if dense is not None:

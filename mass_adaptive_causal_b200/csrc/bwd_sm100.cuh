@@ -191,6 +191,29 @@ __global__ void __launch_bounds__(NT, 1)
   int tcount = 0;  // tiles done by this CTA: picks the LSE / D buffer
   bool ok = true;
   const int nw = (p.nb + 31) >> 5;
+  // The diagonal block (first query head) is nearly always the column's
+  // first kept tile: its Q, dO, LSE and D are fetched now, beside K_j and
+  // V_j, so the first tile does not wait for them after the listing. If the
+  // first kept tile is another block, that tile lets these copies land
+  // before it fetches its own into the same buffers.
+  {
+    const int q = j * T + row;
+    const bool qv = q < p.L;
+    if (half == 0)
+      lse_s[row] = qv ? p.LSE[(size_t)zq0 * p.L + q] * kLog2e : 0.f;
+    else
+      dd_s[row] = qv ? p.Dterm[(size_t)zq0 * p.L + q] : 0.f;
+    if (tid == 0) {
+      mbar_expect_tx(bar_q, TILE_BYTES);
+      tma_load_3d(qa, &tmQ, 0, j * T, zq0, bar_q);
+      tma_load_3d(qa + HALF_BYTES, &tmQ, 64, j * T, zq0, bar_q);
+      mbar_expect_tx(bar_do, TILE_BYTES);
+      tma_load_3d(da, &tmdO, 0, j * T, zq0, bar_do);
+      tma_load_3d(da + HALF_BYTES, &tmdO, 64, j * T, zq0, bar_do);
+      q_pend = do_pend = true;
+    }
+  }
+  bool spec = true;  // the diagonal's copies are still unclaimed
 
   for (int hg = 0; hg < p.G && ok; ++hg) {
   const int z = zq0 + hg;  // query head: Q_i, dO_i, LSE, D, dQ, the keep bits
@@ -239,6 +262,26 @@ __global__ void __launch_bounds__(NT, 1)
     const int inext = has_next ? list[li + 1] : 0;
     float* lse_c = lse_s + (tcount & 1) * T;
     float* dd_c = dd_s + (tcount & 1) * T;
+    if (spec) {
+      spec = false;
+      if (hg == 0 && i == j) {
+        prefetched = true;  // the diagonal's copies (and LSE, D) are this tile's
+      } else {
+        if (mbar_wait(bar_q, ph_q, abort, 0x208)) {
+          ph_q ^= 1;
+        } else {
+          ok = false;
+        }
+        if (tid == 0) {
+          if (mbar_wait(bar_do, ph_do, abort, 0x209)) {
+            ph_do ^= 1;
+          } else {
+            ok = false;
+          }
+        }
+        if (tid == 0) q_pend = do_pend = false;
+      }
+    }
     if (!prefetched) {
       const int q = i * T + row;
       const bool qv = q < p.L;
@@ -506,11 +549,10 @@ __global__ void __launch_bounds__(NT, 1)
   if (tid == 0) {
     bulk_wait_all();  // every dQ reduction of this CTA has landed
     if (kv_pend) mbar_settle(bar_kv, 0);
-    if (!ok) {
-      if (q_pend) mbar_settle(bar_q, ph_q);
-      if (do_pend) mbar_settle(bar_do, ph_do);
-      if (mma_pend) mbar_settle(pend_bar, pend_ph);
-    }
+    // (also the diagonal's copies when no tile was kept)
+    if (q_pend) mbar_settle(bar_q, ph_q);
+    if (do_pend) mbar_settle(bar_do, ph_do);
+    if (!ok && mma_pend) mbar_settle(pend_bar, pend_ph);
   }
 
   // ---- epilogue: dK_j (warps 0-3), dV_j (warps 4-7) in bf16; zero if no

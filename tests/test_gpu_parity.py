@@ -175,6 +175,26 @@ def test_bf16_small_fwd_bwd(L, tau):
     cov.require(0.5)
 
 
+def test_bf16_backward_column_starting_below_its_diagonal():
+    """On random inputs at tau = 32 some key columns fail the backward's test
+    on their diagonal tile while later query blocks keep them, so a column's
+    first kept tile is not the diagonal one (the work pass then drops its
+    early copies of the diagonal block): the gradients still follow the
+    oracle."""
+    rng = np.random.default_rng(11)
+    L, tau = 2048, 32.0
+    arrs = [rng.standard_normal((1, 2, L, 128)) for _ in range(4)]
+    t = {n: dev_tensor(a, torch.bfloat16) for n, a in zip(("Q", "K", "V", "dO"), arrs)}
+    outs = run_bf16_prefill(t, tau)
+    nb = oracle.n_blocks(L, 128)
+    gb = mala.unpack_bits(outs[8][0], nb)  # (heads, nb, nb) backward keep bits
+    assert sum(1 for h in range(2) for j in range(nb) if gb[h, j, j] == 0 and gb[h, j + 1:, j].any()) > 0
+    cov = Coverage(f"column below its diagonal tau={tau}")
+    for h in range(2):
+        check_bf16_slice(t, outs, 0, h, tau, cov)
+    cov.require(0.5)
+
+
 @pytest.mark.parametrize("L", [1000])
 def test_bf16_chain_without_float32_output(L):
     """Backward with D from the bf16 output (no float32 copy)."""
