@@ -140,7 +140,8 @@ int mala_varlen_trace_words(int max_seqlen_q, int max_seqlen_k);
 /* Bytes of device workspace mala_bwd needs: the row terms D (float32
  * [B][H][L]), the float32 dQ accumulator [B][H][L][d] and the per-tile keep
  * bits of the backward's test pass (B*H*nb*ceil(nb/32) words for nb =
- * ceil(L/64)), each rounded up to 256 bytes. */
+ * ceil(L/64)), each rounded up to 256 bytes, and 256 bytes for the work
+ * pass's column counter. */
 size_t mala_bwd_workspace_bytes(int B, int H, int L, int d);
 
 /*

@@ -232,6 +232,7 @@ struct BwdWorkspace {
   float* D;
   float* dQacc;
   uint32_t* bits;  // per-tile keep bits of the test pass (sized for 64-row tiles)
+  int* counter;    // the work pass's column counter
 };
 inline size_t bwd_bits_words(size_t Z, size_t L) {
   const size_t nb = (L + 63) / 64;
@@ -239,7 +240,7 @@ inline size_t bwd_bits_words(size_t Z, size_t L) {
 }
 inline size_t bwd_ws_bytes(size_t Z, size_t L, size_t d) {
   return round256(Z * L * sizeof(float)) + round256(Z * L * d * sizeof(float)) +
-         round256(bwd_bits_words(Z, L) * sizeof(uint32_t));
+         round256(bwd_bits_words(Z, L) * sizeof(uint32_t)) + 256;
 }
 inline BwdWorkspace bwd_ws_carve(void* ws, size_t Z, size_t L, size_t d) {
   BwdWorkspace w;
@@ -249,6 +250,8 @@ inline BwdWorkspace bwd_ws_carve(void* ws, size_t Z, size_t L, size_t d) {
   w.dQacc = reinterpret_cast<float*>(c);
   c += round256(Z * L * d * sizeof(float));
   w.bits = reinterpret_cast<uint32_t*>(c);
+  c += round256(bwd_bits_words(Z, L) * sizeof(uint32_t));
+  w.counter = reinterpret_cast<int*>(c);
   return w;
 }
 
@@ -378,12 +381,18 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
+  p.Zkv = Zkv;
+  p.item_counter = w.counter;
+  aux::zero_u32_kernel<<<1, 32, 0, s>>>(reinterpret_cast<uint32_t*>(w.counter), 1);
   MALA_CUDA_TRY(cudaFuncSetAttribute(bwd100::bwd_bf16_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)bwd100::SMEM_BYTES));
-  // one CTA per (key block, key/value head): dK_j, dV_j sum over its query heads
-  bwd100::bwd_bf16_kernel<<<dim3(p.nb, Zkv), bwd100::NT, bwd100::SMEM_BYTES, s>>>(mq, mk, mv,
-                                                                                 mdo, mdq, p);
+  // persistent: one CTA per SM takes (key block, key/value head) columns in
+  // turn; dK_j, dV_j sum over the column's query heads
+  const int ncols = p.nb * Zkv;
+  const int nsm = sm_count();
+  bwd100::bwd_bf16_kernel<<<ncols < nsm ? ncols : nsm, bwd100::NT, bwd100::SMEM_BYTES, s>>>(
+      mq, mk, mv, mdo, mdq, p);
   const size_t n4 = (size_t)Z * L * 128 / 4;
   aux::convert_bf16_v4_kernel<<<blocks_for(n4, 256, 4 * sm_count()), 256, 0, s>>>(
       reinterpret_cast<const float4*>(w.dQacc), reinterpret_cast<uint2*>(dQ), n4);

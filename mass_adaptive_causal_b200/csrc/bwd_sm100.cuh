@@ -11,8 +11,9 @@
 //   P = exp(S - LSE), dV_j += P^T dO_i, dP = dO_i V_j^T, dS = P o (dP - D),
 //   dK_j += scale dS^T Q_i, dQ_i += scale dS K_j.
 //
-// CTA (256 threads) = one key block j: it lists the kept query blocks
-// i >= j of its column of the bit matrix, then for each: loads Q_i and dO_i
+// Persistent CTAs (256 threads, one per SM) take key columns (key block j
+// of a key/value head) in turn. Per column a CTA lists the kept query
+// blocks i >= j of its column of the bit matrix, then for each: loads Q_i and dO_i
 // (the next kept block's while the current one is worked on), recomputes
 // S^T = K_j Q_i^T with keys in TMEM lanes, and accumulates dK_j, dV_j in
 // TMEM. Threads t and t + 128 own TMEM lane t mod 128 and split the 128
@@ -71,6 +72,8 @@ struct Params {
   int32_t* kept_tiles;   // [B * Hq][nb]
   const uint32_t* bits;  // [B * Hq][nb][nw] from the test pass
   int Hq, Hkv, G;        // query heads, key/value heads, G = Hq / Hkv
+  int Zkv;               // B * Hkv
+  int* item_counter;     // zeroed before the launch: columns handed out past the first
 };
 
 // Row of a TMEM accumulator (this thread's lane) -> bf16 global row. Every
@@ -126,10 +129,13 @@ __global__ void __launch_bounds__(NT, 1)
   // of the tile (a key for S^T / dP^T, a query for dQ), half = which 64.
   const int row = tid & (T - 1);
   const int half = warp >> 2;
-  const int j = blockIdx.x;   // key block 0 has the most query blocks: first
-  const int zkv = blockIdx.y;  // (b, key/value head): K_j, V_j, dK_j, dV_j
-  // dK_j and dV_j sum over the G query heads that share this key/value head
-  const int zq0 = (zkv / p.Hkv) * p.Hq + (zkv % p.Hkv) * p.G;
+  // Columns c = zkv * nb + j (key block j of key/value head zkv), key blocks
+  // ascending within a head. The first gridDim.x columns go one to a CTA;
+  // after that a CTA takes the next column from a counter, so CTAs that run
+  // together work on neighbouring key blocks of one head (their kept query
+  // blocks, and the dQ rows they add into, mostly coincide and stay in L2).
+  const int n_items = p.nb * p.Zkv;
+  int* item_slot = reinterpret_cast<int*>(tmem_slot + 2);
   const uint32_t bar_kv = smem_u32(&bars[0]);
   const uint32_t bar_q = smem_u32(&bars[1]);
   const uint32_t bar_do = smem_u32(&bars[2]);
@@ -166,19 +172,10 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t t_dk = tmem + lane_base + 256;
   const uint32_t t_dv = tmem + lane_base + 384;
 
-  // K_j, V_j: waited for before the first product, so the load overlaps the
-  // listing of the kept query blocks
-  if (tid == 0) {
-    mbar_expect_tx(bar_kv, 2 * TILE_BYTES);
-    tma_load_3d(ka, &tmK, 0, j * T, zkv, bar_kv);
-    tma_load_3d(ka + HALF_BYTES, &tmK, 64, j * T, zkv, bar_kv);
-    tma_load_3d(va, &tmV, 0, j * T, zkv, bar_kv);
-    tma_load_3d(va + HALF_BYTES, &tmV, 64, j * T, zkv, bar_kv);
-  }
   // Phases and copies/MMAs in flight; thread 0 issues every copy and MMA,
   // so its own view is the one that the exit path settles.
   uint32_t ph_q = 0, ph_do = 0, ph_s = 0, ph_dv = 0, ph_dk = 0, ph_dq = 0;
-  bool kv_pend = true, q_pend = false, do_pend = false, mma_pend = false;
+  bool kv_pend = false, q_pend = false, do_pend = false, mma_pend = false;
   uint32_t pend_bar = 0, pend_ph = 0;  // thread 0: the last barrier committed
   auto commit = [&](uint32_t bar, uint32_t ph) {
     mma_commit(bar);
@@ -186,33 +183,51 @@ __global__ void __launch_bounds__(NT, 1)
     pend_ph = ph;
     mma_pend = true;
   };
-  bool kv_ready = false;
-  int kept_count = 0;
   int tcount = 0;  // tiles done by this CTA: picks the LSE / D buffer
+  uint32_t ph_kv = 0;
   bool ok = true;
   const int nw = (p.nb + 31) >> 5;
-  // The diagonal block (first query head) is nearly always the column's
-  // first kept tile: its Q, dO, LSE and D are fetched now, beside K_j and
-  // V_j, so the first tile does not wait for them after the listing. If the
-  // first kept tile is another block, that tile lets these copies land
-  // before it fetches its own into the same buffers.
-  {
+  // Loads of column c that need no listing: K_j, V_j and, since the diagonal
+  // block (first query head) is nearly always the column's first kept tile,
+  // its Q, dO, LSE and D (LSE and D into buffer tcount & 1). A column whose
+  // first kept tile is another block lets these copies land before it fetches
+  // its own into the same buffers.
+  auto issue_column_loads = [&](int c) {
+    const int j = c % p.nb, zkv = c / p.nb;
+    const int zq0 = (zkv / p.Hkv) * p.Hq + (zkv % p.Hkv) * p.G;
     const int q = j * T + row;
     const bool qv = q < p.L;
     if (half == 0)
-      lse_s[row] = qv ? p.LSE[(size_t)zq0 * p.L + q] * kLog2e : 0.f;
+      lse_s[(tcount & 1) * T + row] = qv ? p.LSE[(size_t)zq0 * p.L + q] * kLog2e : 0.f;
     else
-      dd_s[row] = qv ? p.Dterm[(size_t)zq0 * p.L + q] : 0.f;
+      dd_s[(tcount & 1) * T + row] = qv ? p.Dterm[(size_t)zq0 * p.L + q] : 0.f;
     if (tid == 0) {
+      mbar_expect_tx(bar_kv, 2 * TILE_BYTES);
+      tma_load_3d(ka, &tmK, 0, j * T, zkv, bar_kv);
+      tma_load_3d(ka + HALF_BYTES, &tmK, 64, j * T, zkv, bar_kv);
+      tma_load_3d(va, &tmV, 0, j * T, zkv, bar_kv);
+      tma_load_3d(va + HALF_BYTES, &tmV, 64, j * T, zkv, bar_kv);
       mbar_expect_tx(bar_q, TILE_BYTES);
       tma_load_3d(qa, &tmQ, 0, j * T, zq0, bar_q);
       tma_load_3d(qa + HALF_BYTES, &tmQ, 64, j * T, zq0, bar_q);
       mbar_expect_tx(bar_do, TILE_BYTES);
       tma_load_3d(da, &tmdO, 0, j * T, zq0, bar_do);
       tma_load_3d(da + HALF_BYTES, &tmdO, 64, j * T, zq0, bar_do);
-      q_pend = do_pend = true;
+      kv_pend = q_pend = do_pend = true;
     }
-  }
+  };
+  int col = blockIdx.x;
+  if (col < n_items) issue_column_loads(col);
+  while (col < n_items && ok) {
+  const int j = col % p.nb;    // key block
+  const int zkv = col / p.nb;  // (b, key/value head): K_j, V_j, dK_j, dV_j
+  // dK_j and dV_j sum over the G query heads that share this key/value head
+  const int zq0 = (zkv / p.Hkv) * p.Hq + (zkv % p.Hkv) * p.G;
+  // the next column, taken now so that its loads can start as soon as this
+  // column's last products have read the buffers
+  if (tid == 0) *item_slot = (int)gridDim.x + atomicAdd(p.item_counter, 1);
+  bool kv_ready = false;
+  int kept_count = 0;
   bool spec = true;  // the diagonal's copies are still unclaimed
 
   for (int hg = 0; hg < p.G && ok; ++hg) {
@@ -306,7 +321,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (q < p.L) next_val = (half == 0 ? p.LSE : p.Dterm)[(size_t)z * p.L + q];
     }
     if (!kv_ready) {
-      if (mbar_wait(bar_kv, 0, abort, 0x201)) {
+      if (mbar_wait(bar_kv, ph_kv, abort, 0x201)) {
         kv_pend = false;
       } else {
         ok = false;
@@ -543,17 +558,26 @@ __global__ void __launch_bounds__(NT, 1)
   }
   if (tid == 0 && p.kept_tiles) p.kept_tiles[(size_t)z * p.nb + j] = kept_count - kept_before;
   }
-  // thread 0's copies and MMAs still in flight (K_j, V_j when no tile was
-  // kept; anything on the error path) land before the CTA releases its
-  // shared memory and TMEM
-  if (tid == 0) {
-    bulk_wait_all();  // every dQ reduction of this CTA has landed
-    if (kv_pend) mbar_settle(bar_kv, 0);
-    // (also the diagonal's copies when no tile was kept)
-    if (q_pend) mbar_settle(bar_q, ph_q);
-    if (do_pend) mbar_settle(bar_do, ph_do);
-    if (!ok && mma_pend) mbar_settle(pend_bar, pend_ph);
+  // The column's buffers are free: its last products have completed (or it
+  // kept no tile). Copies still unclaimed -- K_j, V_j and the diagonal's
+  // when no tile was kept -- land first; then the next column's loads start
+  // while this one writes dK_j, dV_j.
+  if (!kv_ready) {
+    if (!mbar_wait(bar_kv, ph_kv, abort, 0x20a)) ok = false;
   }
+  ph_kv ^= 1;
+  if (spec) {
+    if (!mbar_wait(bar_q, ph_q, abort, 0x20b)) ok = false;
+    ph_q ^= 1;
+    if (tid == 0) {
+      if (!mbar_wait(bar_do, ph_do, abort, 0x20c)) ok = false;
+      ph_do ^= 1;
+    }
+  }
+  if (tid == 0) kv_pend = q_pend = do_pend = false;
+  __syncthreads();  // item_slot written; every thread past its column's loads
+  const int next = *item_slot;
+  if (ok && next < n_items) issue_column_loads(next);
 
   // ---- epilogue: dK_j (warps 0-3), dV_j (warps 4-7) in bf16; zero if no
   // tile was kept (TMEM loads are warp-collective: all lanes load, valid key
@@ -570,6 +594,21 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = zero;
     }
+  }
+  // dK, dV read out of TMEM before the next column's products overwrite them
+  tc_fence_before();
+  if (__syncthreads_or(!ok)) ok = false;
+  tc_fence_after();
+  col = next;
+  }
+  // thread 0's copies and MMAs still in flight (anything on the error path)
+  // land before the CTA releases its shared memory and TMEM
+  if (tid == 0) {
+    bulk_wait_all();  // every dQ reduction of this CTA has landed
+    if (kv_pend) mbar_settle(bar_kv, ph_kv);
+    if (q_pend) mbar_settle(bar_q, ph_q);
+    if (do_pend) mbar_settle(bar_do, ph_do);
+    if (!ok && mma_pend) mbar_settle(pend_bar, pend_ph);
   }
   tc_fence_before();
   __syncthreads();

@@ -74,7 +74,8 @@ def test_bwd_and_decode_argument_checks(lib):
     need = lib.mala_bwd_workspace_bytes(1, 2, 1000, 128)
     r256 = lambda x: ((x + 255) // 256) * 256
     nb64 = (1000 + 63) // 64
-    assert need == r256(2 * 1000 * 4) + r256(2 * 1000 * 128 * 4) + r256(2 * nb64 * ((nb64 + 31) // 32) * 4)
+    assert need == (r256(2 * 1000 * 4) + r256(2 * 1000 * 128 * 4)
+                    + r256(2 * nb64 * ((nb64 + 31) // 32) * 4) + 256)  # + the column counter
     args = [v] * 11
     assert lib.mala_bwd(*args, need - 1, 1, 2, 2, 1000, 128, 1, 1.0, 128, 0.0, None, None, None) == 1
     assert lib.mala_bwd(*args, need, 1, 2, 2, 1000, 128, 1, -0.5, 128, 0.0, None, None, None) == 1
