@@ -102,11 +102,14 @@ template <bool DENSE>
 struct Plan {
   static constexpr int NSK = DENSE ? 2 : 6;  // even: one stage's tiles share an issuer
   static constexpr int NPB = DENSE ? 2 : 1;  // P buffers, tile t uses t % NPB
-  // S buffer u's full / free barriers come in pairs, one per test group: tile
-  // t uses pair member t % 2 (DENSE: member 0 only, every warp reads every
-  // tile), so each barrier's phases are waited for in order by one consumer
-  static constexpr int SGRP_MASK = DENSE ? 0 : 1;
-  static constexpr int SPER = DENSE ? 3 : 6;            // tiles between uses of one barrier
+  // S buffer u's full / free barriers come in pairs: tile t uses pair member
+  // t % 2, so each barrier serves every sixth tile. Then one test group
+  // (DENSE: every test warp) consumes its phases, and one QK issuer (even or
+  // odd tiles) arms, waits for or commits them, in order; with one barrier
+  // per buffer the two issuers would take alternate phases, and one could
+  // arm a phase while the other's earlier phase was still pending.
+  static constexpr int SGRP_MASK = 1;
+  static constexpr int SPER = 6;                        // tiles between uses of one barrier
   static constexpr uint32_t REL_LOCAL = DENSE ? 8 : 4;  // releasing warps per CTA and tile
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
