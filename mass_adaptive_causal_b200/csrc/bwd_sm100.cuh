@@ -12,11 +12,13 @@
 //   dK_j += scale dS^T Q_i, dQ_i += scale dS K_j.
 //
 // Persistent CTAs (256 threads, one per SM) take key columns (key block j
-// of a key/value head) in turn. Per column a CTA lists the kept query
-// blocks i >= j of its column of the bit matrix, then for each: loads Q_i and dO_i
-// (the next kept block's while the current one is worked on), recomputes
-// S^T = K_j Q_i^T with keys in TMEM lanes, and accumulates dK_j, dV_j in
-// TMEM. Threads t and t + 128 own TMEM lane t mod 128 and split the 128
+// of a key/value head) in turn; a column's K_j, V_j and diagonal block load
+// while the previous column writes its dK, dV. Per column a CTA lists the
+// kept query blocks i >= j of its column of the bit matrix, then for each:
+// S^T = K_j Q_i^T (keys in TMEM lanes) with dP^T = V_j dO_i^T behind it, P,
+// dV, dS, then dK and dQ, each stage on its own barrier; the next kept
+// block's dO loads once dP^T and dV have read the current one, its Q once dK
+// has. dK_j, dV_j accumulate in TMEM. Threads t and t + 128 own TMEM lane t mod 128 and split the 128
 // columns of each accumulator into halves, so the elementwise work of a
 // tile (P, dS, the dQ readout) is spread over 8 warps:
 //   TMEM [  0,128): S^T, later reused for dQ_i = dS K_j
@@ -192,15 +194,22 @@ __global__ void __launch_bounds__(NT, 1)
   // its Q, dO, LSE and D (LSE and D into buffer tcount & 1). A column whose
   // first kept tile is another block lets these copies land before it fetches
   // its own into the same buffers.
-  auto issue_column_loads = [&](int c) {
+  auto column_row_term = [&](int c) {  // this thread's LSE (half 0) or D of the diagonal block
     const int j = c % p.nb, zkv = c / p.nb;
     const int zq0 = (zkv / p.Hkv) * p.Hq + (zkv % p.Hkv) * p.G;
     const int q = j * T + row;
-    const bool qv = q < p.L;
+    if (q >= p.L) return 0.f;
+    return half == 0 ? p.LSE[(size_t)zq0 * p.L + q] * kLog2e : p.Dterm[(size_t)zq0 * p.L + q];
+  };
+  auto store_row_term = [&](float v) {
     if (half == 0)
-      lse_s[(tcount & 1) * T + row] = qv ? p.LSE[(size_t)zq0 * p.L + q] * kLog2e : 0.f;
+      lse_s[(tcount & 1) * T + row] = v;
     else
-      dd_s[(tcount & 1) * T + row] = qv ? p.Dterm[(size_t)zq0 * p.L + q] : 0.f;
+      dd_s[(tcount & 1) * T + row] = v;
+  };
+  auto issue_column_copies = [&](int c) {
+    const int j = c % p.nb, zkv = c / p.nb;
+    const int zq0 = (zkv / p.Hkv) * p.Hq + (zkv % p.Hkv) * p.G;
     if (tid == 0) {
       mbar_expect_tx(bar_kv, 2 * TILE_BYTES);
       tma_load_3d(ka, &tmK, 0, j * T, zkv, bar_kv);
@@ -217,15 +226,20 @@ __global__ void __launch_bounds__(NT, 1)
     }
   };
   int col = blockIdx.x;
-  if (col < n_items) issue_column_loads(col);
+  if (col < n_items) {
+    issue_column_copies(col);
+    store_row_term(column_row_term(col));
+  }
   while (col < n_items && ok) {
   const int j = col % p.nb;    // key block
   const int zkv = col / p.nb;  // (b, key/value head): K_j, V_j, dK_j, dV_j
   // dK_j and dV_j sum over the G query heads that share this key/value head
   const int zq0 = (zkv / p.Hkv) * p.Hq + (zkv % p.Hkv) * p.G;
   // the next column, taken now so that its loads can start as soon as this
-  // column's last products have read the buffers
-  if (tid == 0) *item_slot = (int)gridDim.x + atomicAdd(p.item_counter, 1);
+  // column's last products have read the buffers (the value is first needed
+  // at the column's end, so the counter's round trip is not waited for here)
+  int fetched = 0;
+  if (tid == 0) fetched = (int)gridDim.x + atomicAdd(p.item_counter, 1);
   bool kv_ready = false;
   int kept_count = 0;
   bool spec = true;  // the diagonal's copies are still unclaimed
@@ -574,10 +588,20 @@ __global__ void __launch_bounds__(NT, 1)
       ph_do ^= 1;
     }
   }
-  if (tid == 0) kv_pend = q_pend = do_pend = false;
+  if (tid == 0) {
+    kv_pend = q_pend = do_pend = false;
+    *item_slot = fetched;
+  }
   __syncthreads();  // item_slot written; every thread past its column's loads
   const int next = *item_slot;
-  if (ok && next < n_items) issue_column_loads(next);
+  const bool more = ok && next < n_items;
+  // the next column's copies start now; its LSE / D are loaded now and stored
+  // after the epilogue, which does not wait for them
+  float next_term = 0.f;
+  if (more) {
+    issue_column_copies(next);
+    next_term = column_row_term(next);
+  }
 
   // ---- epilogue: dK_j (warps 0-3), dV_j (warps 4-7) in bf16; zero if no
   // tile was kept (TMEM loads are warp-collective: all lanes load, valid key
@@ -595,6 +619,7 @@ __global__ void __launch_bounds__(NT, 1)
       for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = zero;
     }
   }
+  if (more) store_row_term(next_term);
   // dK, dV read out of TMEM before the next column's products overwrite them
   tc_fence_before();
   if (__syncthreads_or(!ok)) ok = false;
