@@ -356,18 +356,6 @@ __device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(m0), "r"(m1)
       : "memory");
 }
-// D (+)= A[tmem] * B[smem] over the pair (A: each CTA's own TMEM rows).
-__device__ __forceinline__ void mma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate, uint32_t m0,
-                                            uint32_t m1) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5, %6, %6, %6, %6}, p;"
-      "\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(m0), "r"(m1)
-      : "memory");
-}
 // Arrive once, when the issuing thread's prior MMAs complete, on the mbarrier
 // at this shared-memory offset in every CTA of `cta_mask` (bit r = rank r).
 __device__ __forceinline__ void commit_pair(uint32_t bar, uint16_t cta_mask) {
@@ -382,11 +370,6 @@ __device__ __forceinline__ void commit_pair(uint32_t bar, uint16_t cta_mask) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar)
                : "memory");
-}
-// Arrive on an mbarrier given by cluster address with the default (CTA
-// scope) semantics: no cluster-wide fence, for signals that carry no data.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 // Asynchronous 32-bit store into a peer CTA's shared memory whose arrival is
 // counted (4 bytes of transaction) on an mbarrier of that same CTA. The
@@ -412,51 +395,6 @@ __device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity)
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait on a local mbarrier whose arrivals may come from the peer CTA
-// (acquire at cluster scope); the thread may sleep inside try_wait, so a
-// warp that waits long does not take issue slots from its neighbours.
-__device__ __forceinline__ bool mbar_wait_cluster_sleep(uint32_t bar, uint32_t parity,
-                                                        volatile int* abort, unsigned int where) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      if (atomicExch((int*)abort, 1) == 0) record_timeout(where);
-      return false;
-    }
-  }
-}
-// Bounded wait on a local mbarrier whose arrivals may come from the peer CTA
-// (acquire at cluster scope); polls without suspending.
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort, unsigned int where) {
-  if (mbar_test_cluster(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_test_cluster(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      if (atomicExch((int*)abort, 1) == 0) record_timeout(where);
-      return false;
-    }
-  }
-}
-
 // 2^x by the hardware's approximate exponential (PTX ex2.approx.ftz.f32:
 // relative error near 2^-22, subnormal results flushed to zero), one
 // instruction; the per-element exponentials of P use it.
