@@ -320,11 +320,12 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
                             void* dK, void* dV, int B, int Hq, int Hkv, int L, float scale,
                             float tau,
                             int32_t* kept, uint32_t* bits, cudaStream_t s) {
-  CUtensorMap mq, mk, mv, mdo, mk64, mdq;
+  CUtensorMap mq, mk, mv, mdo, mk64, mdq, mdk, mdv;
   const int Z = B * Hq, Zkv = B * Hkv;
   if (!make_map(&mq, Q, L, Z) || !make_map(&mk, K, L, Zkv) || !make_map(&mv, V, L, Zkv) ||
       !make_map(&mdo, dO, L, Z) || !make_map(&mk64, K, L, Zkv, 64) ||
-      !make_map_f32_acc(&mdq, w.dQacc, L, Z))
+      !make_map_f32_acc(&mdq, w.dQacc, L, Z) || !make_map(&mdk, dK, L, Zkv) ||
+      !make_map(&mdv, dV, L, Zkv))
     return MALA_ERR_CUDA;
   const int nb = (L + bwd100::T - 1) / bwd100::T;
   const int never = tau == 0.f;
@@ -392,7 +393,7 @@ inline mala_status bwd_bf16(const void* Q, const void* K, const void* V, const v
   const int ncols = p.nb * Zkv;
   const int nsm = sm_count();
   bwd100::bwd_bf16_kernel<<<ncols < nsm ? ncols : nsm, bwd100::NT, bwd100::SMEM_BYTES, s>>>(
-      mq, mk, mv, mdo, mdq, p);
+      mq, mk, mv, mdo, mdq, mdk, mdv, p);
   const size_t n4 = (size_t)Z * L * 128 / 4;
   aux::convert_bf16_v4_kernel<<<blocks_for(n4, 256, 4 * sm_count()), 256, 0, s>>>(
       reinterpret_cast<const float4*>(w.dQacc), reinterpret_cast<uint2*>(dQ), n4);

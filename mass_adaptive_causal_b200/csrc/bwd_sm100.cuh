@@ -26,13 +26,13 @@
 //   TMEM [256,384): dK_j accumulator      TMEM [384,512): dV_j accumulator
 // Shared memory: K_j, V_j, Q_i, dO_i, P^T, dS^T (32 KB each, 128-byte
 // swizzle) + per-query LSE and D, and the list of kept query blocks.
-// dS goes to the tensor cores as a bf16 pair hi + lo (dQ sums rows of dS
-// that cancel); dQ_i is read back from TMEM (query rows in lanes) into a
-// float32 tile in the then free P^T and dS^T buffers and added into a
-// float32 workspace by four TMA bulk tensor reductions (the adds happen in
-// L2, a 16 KB block per instruction, instead of 4096 float4 atomics from the
-// threads), converted afterwards. The next tile's first MMA waits until the
-// reductions have read the tile.
+// dS goes to the dQ product as a bf16 pair hi + lo (dQ sums rows of dS
+// that cancel), to the dK product as hi alone; dQ_i is read back from TMEM
+// (query rows in lanes) into a float32 tile in the then free P^T and dS^T
+// buffers and added into a float32 workspace by four TMA bulk tensor
+// reductions (the adds happen in L2, a 16 KB block per instruction, instead
+// of 4096 float4 atomics from the threads), converted afterwards. The next
+// tile forms its P while the reductions read the tile and stores P after.
 #pragma once
 
 #include "sm100.cuh"
@@ -46,6 +46,10 @@ constexpr int T = 128;
 constexpr int D = 128;
 constexpr int NT = 256;
 constexpr int NWARP = NT / 32;
+// The thread that issues the bulk copies out of shared memory (dQ
+// reductions, dK / dV stores) and owns their bulk async-groups; thread 0
+// issues the loads and MMAs.
+constexpr int BULK_TID = 32;
 constexpr uint32_t TILE_BYTES = T * D * 2;
 constexpr uint32_t HALF_BYTES = T * 64 * 2;
 constexpr int LIST_CHUNK = 1024;  // query blocks listed per round
@@ -78,32 +82,28 @@ struct Params {
   int* item_counter;     // zeroed before the launch: columns handed out past the first
 };
 
-// Row of a TMEM accumulator (this thread's lane) -> bf16 global row. Every
-// lane of the warp must call it (tcgen05.ld is warp-collective); `store`
-// masks the global write.
-__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, uint32_t taddr, bool store) {
+// Row `row` of a TMEM accumulator (this thread's lane, 128 columns) -> bf16
+// row of a 128 x 128 shared tile in the two 64-column halves and 128-byte
+// swizzle of the bf16 tensor maps. Every lane of the warp must call it
+// (tcgen05.ld is warp-collective).
+__device__ __forceinline__ void stage_row_bf16(uint32_t dst, int row, uint32_t taddr) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     float v[32];
     tmem_ld32(taddr + c * 32, v);
-    if (!store) continue;
-    uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint4 w;
-      w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-      w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-      w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-      w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-      d4[q] = w;
-    }
+    for (int q = 0; q < 4; ++q)
+      st_shared_v4(dst + sw128_chunk_off(row, c * 32 + q * 8, T), pack_bf16(v[8 * q + 0], v[8 * q + 1]),
+                   pack_bf16(v[8 * q + 2], v[8 * q + 3]), pack_bf16(v[8 * q + 4], v[8 * q + 5]),
+                   pack_bf16(v[8 * q + 6], v[8 * q + 7]));
   }
 }
 
 __global__ void __launch_bounds__(NT, 1)
     bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                    const __grid_constant__ CUtensorMap tmdQ, const Params p) {
+                    const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmdK,
+                    const __grid_constant__ CUtensorMap tmdV, const Params p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -373,9 +373,6 @@ __global__ void __launch_bounds__(NT, 1)
       } else {
         ok = false;
       }
-      // the previous tile's dQ reduction has read its staging tile (the P^T
-      // and dS^T buffers this tile writes next)
-      bulk_wait_read_all();
     }
     if (mbar_wait(bar_s, ph_s, abort, 0x203)) {
       ph_s ^= 1;
@@ -412,13 +409,17 @@ __global__ void __launch_bounds__(NT, 1)
             pr[c * 32 + e] = legal ? ex2_approx(s[e] * p.scale_log2 - lse_c[qc]) : 0.f;
           }
         }
+      }
+      // P is formed while the previous tile's dQ reductions read their
+      // staging tile (the P^T and dS^T buffers); it is stored once they have
+      if (tid == BULK_TID) bulk_wait_read_all();
+      __syncthreads();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int q0 = c * 32 + q * 8;
-          st_shared_v4(pta + sw128_chunk_off(row, half * 64 + q0, T),
-                       pack_bf16(pr[q0], pr[q0 + 1]), pack_bf16(pr[q0 + 2], pr[q0 + 3]),
-                       pack_bf16(pr[q0 + 4], pr[q0 + 5]), pack_bf16(pr[q0 + 6], pr[q0 + 7]));
-        }
+      for (int q = 0; q < 8; ++q) {
+        const int q0 = q * 8;
+        st_shared_v4(pta + sw128_chunk_off(row, half * 64 + q0, T),
+                     pack_bf16(pr[q0], pr[q0 + 1]), pack_bf16(pr[q0 + 2], pr[q0 + 3]),
+                     pack_bf16(pr[q0 + 4], pr[q0 + 5]), pack_bf16(pr[q0 + 6], pr[q0 + 7]));
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -483,21 +484,18 @@ __global__ void __launch_bounds__(NT, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
-      // ---- dK += (hi + lo)^T Q_i, then dQ_i = (hi + lo) K_j (into the S^T
-      // columns); once dK is done Q_i is free and the next tile's Q loads
-      // while the dQ products run
+      // ---- dK += hi^T Q_i, then dQ_i = (hi + lo) K_j (into the S^T columns);
+      // once dK is done Q_i is free and the next tile's Q loads while the dQ
+      // products run. dK sums over queries, where dS has no cancelling
+      // structure: the single rounding of hi leaves it within ~2e-3 (rel-L2).
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const uint32_t src = part == 0 ? sta : pta;
-#pragma unroll
-          for (int kk = 0; kk < T / 16; ++kk) {
-            const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            mma_bf16(tmem + 256, sdesc_sw128(src + aoff, 16, 1024),
-                     sdesc_sw128(qa + kk * 2048, HALF_BYTES, 1024), IDESC_ACC,
-                     (kept_count > 0 || part > 0 || kk > 0) ? 1u : 0u);
-          }
+        for (int kk = 0; kk < T / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          mma_bf16(tmem + 256, sdesc_sw128(sta + aoff, 16, 1024),
+                   sdesc_sw128(qa + kk * 2048, HALF_BYTES, 1024), IDESC_ACC,
+                   (kept_count > 0 || kk > 0) ? 1u : 0u);
         }
         commit(bar_dk, ph_dk);
 #pragma unroll
@@ -563,7 +561,7 @@ __global__ void __launch_bounds__(NT, 1)
     // the next tile once every thread is here
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
+    if (tid == BULK_TID) {
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) tma_reduce_add_3d(&tmdQ, pta + cb * 16384u, cb * 32, i * T, z);
       bulk_commit_group();
@@ -592,6 +590,9 @@ __global__ void __launch_bounds__(NT, 1)
     kv_pend = q_pend = do_pend = false;
     *item_slot = fetched;
   }
+  // the epilogue stages dK_j, dV_j in the P^T and dS^T buffers once the last
+  // tile's dQ reductions have read them
+  if (tid == BULK_TID) bulk_wait_read_all();
   __syncthreads();  // item_slot written; every thread past its column's loads
   const int next = *item_slot;
   const bool more = ok && next < n_items;
@@ -603,17 +604,19 @@ __global__ void __launch_bounds__(NT, 1)
     next_term = column_row_term(next);
   }
 
-  // ---- epilogue: dK_j (warps 0-3), dV_j (warps 4-7) in bf16; zero if no
-  // tile was kept (TMEM loads are warp-collective: all lanes load, valid key
-  // rows store)
+  // ---- epilogue: dK_j (warps 0-3) into the P^T buffer, dV_j (warps 4-7)
+  // into the dS^T buffer as bf16 tiles, written out by four bulk tensor
+  // stores (rows past L are not written) that run under the next column's
+  // first products; the next tile stores its P once they have read the
+  // buffers. A column that kept no tile writes zero rows directly.
   const int key = j * T + row;
   if (ok) {
-    __nv_bfloat16* dst =
-        (half == 0 ? p.dK : p.dV) + ((size_t)zkv * p.L + (key < p.L ? key : 0)) * D;
     if (kept_count > 0) {
       tc_fence_after();
-      store_row_bf16(dst, half == 0 ? t_dk : t_dv, key < p.L);
+      stage_row_bf16(half == 0 ? pta : sta, row, half == 0 ? t_dk : t_dv);
+      fence_proxy_async_smem();  // the staged tiles visible to the bulk stores
     } else if (key < p.L) {
+      __nv_bfloat16* dst = (half == 0 ? p.dK : p.dV) + ((size_t)zkv * p.L + key) * D;
       uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = zero;
@@ -624,12 +627,19 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_before();
   if (__syncthreads_or(!ok)) ok = false;
   tc_fence_after();
+  if (ok && kept_count > 0 && tid == BULK_TID) {
+    tma_store_3d(&tmdK, pta, 0, j * T, zkv);
+    tma_store_3d(&tmdK, pta + HALF_BYTES, 64, j * T, zkv);
+    tma_store_3d(&tmdV, sta, 0, j * T, zkv);
+    tma_store_3d(&tmdV, sta + HALF_BYTES, 64, j * T, zkv);
+    bulk_commit_group();
+  }
   col = next;
   }
   // thread 0's copies and MMAs still in flight (anything on the error path)
   // land before the CTA releases its shared memory and TMEM
+  if (tid == BULK_TID) bulk_wait_all();  // every dQ reduction and dK / dV store has landed
   if (tid == 0) {
-    bulk_wait_all();  // every dQ reduction of this CTA has landed
     if (kv_pend) mbar_settle(bar_kv, ph_kv);
     if (q_pend) mbar_settle(bar_q, ph_q);
     if (do_pend) mbar_settle(bar_do, ph_do);
