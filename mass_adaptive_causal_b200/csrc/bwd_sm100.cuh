@@ -16,16 +16,19 @@
 // while the previous column writes its dK, dV. Per column a CTA lists the
 // kept query blocks i >= j of its column of the bit matrix, then for each:
 // S^T = K_j Q_i^T (keys in TMEM lanes) with dP^T = V_j dO_i^T behind it, P,
-// dV, dS, then dK and dQ, each stage on its own barrier; the next kept
-// block's dO loads once dP^T and dV have read the current one, its Q once dK
-// has. dK_j, dV_j accumulate in TMEM. Threads t and t + 128 own TMEM lane t mod 128 and split the 128
-// columns of each accumulator into halves, so the elementwise work of a
-// tile (P, dS, the dQ readout) is spread over 8 warps:
-//   TMEM [  0,128): S^T, later reused for dQ_i = dS K_j
-//   TMEM [128,256): dP^T = V_j dO_i^T
+// dV, dS, then dK and dQ, each stage on its own barrier. Q alternates
+// between two buffers and loads two tiles ahead, as each tile's dK product
+// frees its buffer; the next tile's S^T is issued right behind the tile's dQ
+// product, so the tensor cores compute it while the threads read dQ out; the
+// next dO loads once dP^T and dV have read the current one. dK_j, dV_j accumulate in TMEM. Threads t and
+// t + 128 own TMEM lane t mod 128 and split the 128 columns of each
+// accumulator into halves, so the elementwise work of a tile (P, dS, the dQ
+// readout) is spread over 8 warps:
+//   TMEM [  0,128): S^T = K_j Q_i^T
+//   TMEM [128,256): dP^T = V_j dO_i^T, later reused for dQ_i = dS K_j
 //   TMEM [256,384): dK_j accumulator      TMEM [384,512): dV_j accumulator
-// Shared memory: K_j, V_j, Q_i, dO_i, P^T, dS^T (32 KB each, 128-byte
-// swizzle) + per-query LSE and D, and the list of kept query blocks.
+// Shared memory: K_j, V_j, Q_i (two), dO_i, P^T, dS^T (32 KB each, 128-byte
+// swizzle) + per-query LSE and D, and the kept blocks as a bit mask.
 // dS goes to the dQ product as a bf16 pair hi + lo (dQ sums rows of dS
 // that cancel), to the dK product as hi alone; dQ_i is read back from TMEM
 // (query rows in lanes) into a float32 tile in the then free P^T and dS^T
@@ -54,8 +57,10 @@ constexpr uint32_t TILE_BYTES = T * D * 2;
 constexpr uint32_t HALF_BYTES = T * 64 * 2;
 constexpr int LIST_CHUNK = 1024;  // query blocks listed per round
 constexpr int LIST_ROUNDS = LIST_CHUNK / NT;
-constexpr uint32_t SMEM_BYTES = 6 * TILE_BYTES + 1024 /*align*/ + 2048 /*LSE, D*/ + 128 /*bars*/ +
-                                LIST_CHUNK * 4 + LIST_ROUNDS * NWARP * 4;
+constexpr int MASK_WORDS = LIST_CHUNK / 32;
+// K, V, Q (two buffers), dO, P^T, dS^T; LSE and D (two buffers each); the
+// barriers; the kept-block masks (two)
+constexpr uint32_t SMEM_BYTES = 7 * TILE_BYTES + 2048 + 128 + 2 * MASK_WORDS * 4;
 constexpr uint32_t TMEM_COLS = 512;
 // S^T, dP^T: A = K_j or V_j (K-major over d), B = Q_i or dO_i (K-major over d)
 constexpr uint32_t IDESC_KQ = idesc_bf16(128, 128, false, false);
@@ -104,24 +109,29 @@ __global__ void __launch_bounds__(NT, 1)
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmdK,
                     const __grid_constant__ CUtensorMap tmdV, const Params p) {
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base = smem_raw;
+  // 128-byte swizzled tiles need a 1024-byte aligned base
+  if (smem_u32(base) & 1023u) {
+    if (threadIdx.x == 0) record_layout_error(0x2f2);
+    return;
+  }
   const uint32_t ka = smem_u32(base);
   const uint32_t va = ka + TILE_BYTES;
-  const uint32_t qa = ka + 2 * TILE_BYTES;
-  const uint32_t da = ka + 3 * TILE_BYTES;   // dO_i
-  const uint32_t pta = ka + 4 * TILE_BYTES;  // P^T
-  const uint32_t sta = ka + 5 * TILE_BYTES;  // dS^T
+  // Q_i of the CTA's tiles alternate between two buffers (tile count parity),
+  // so the next tile's Q loads a whole tile ahead
+  const uint32_t qa0 = ka + 2 * TILE_BYTES;
+  const uint32_t da = ka + 4 * TILE_BYTES;   // dO_i
+  const uint32_t pta = ka + 5 * TILE_BYTES;  // P^T
+  const uint32_t sta = ka + 6 * TILE_BYTES;  // dS^T
   // per-query LSE * log2(e) and D, two buffers each: the next kept tile's
   // values land in one while the current tile reads the other
-  float* lse_s = reinterpret_cast<float*>(base + 6 * TILE_BYTES);  // [2][128]
+  float* lse_s = reinterpret_cast<float*>(base + 7 * TILE_BYTES);  // [2][128]
   float* dd_s = lse_s + 2 * T;                                      // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(dd_s + 2 * T);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* list = reinterpret_cast<int*>(bars + 16);  // [LIST_CHUNK]
-  int* wcount = list + LIST_CHUNK;               // [LIST_ROUNDS][NWARP]
+  uint32_t* kmask = reinterpret_cast<uint32_t*>(bars + 16);  // [2][MASK_WORDS]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -139,23 +149,26 @@ __global__ void __launch_bounds__(NT, 1)
   const int n_items = p.nb * p.Zkv;
   int* item_slot = reinterpret_cast<int*>(tmem_slot + 2);
   const uint32_t bar_kv = smem_u32(&bars[0]);
-  const uint32_t bar_q = smem_u32(&bars[1]);
-  const uint32_t bar_do = smem_u32(&bars[2]);
+  const uint32_t bar_q0 = smem_u32(&bars[1]);  // Q buffer b: bar_q0 + 8 b
+  const uint32_t bar_do = smem_u32(&bars[3]);
   // one completion per tile each: S^T; dP^T and dV; dK; dQ (a commit
   // covers every earlier MMA of the issuing thread)
-  const uint32_t bar_s = smem_u32(&bars[3]);
-  const uint32_t bar_dv = smem_u32(&bars[4]);
-  const uint32_t bar_dk = smem_u32(&bars[5]);
-  const uint32_t bar_dq = smem_u32(&bars[6]);
+  const uint32_t bar_s = smem_u32(&bars[4]);
+  const uint32_t bar_dv = smem_u32(&bars[5]);
+  const uint32_t bar_dk = smem_u32(&bars[6]);
+  const uint32_t bar_dq = smem_u32(&bars[7]);
+  const uint32_t bar_fin = smem_u32(&bars[8]);  // the exit's wait for every MMA
 
   if (tid == 0) {
     mbar_init(bar_kv, 1);
-    mbar_init(bar_q, 1);
+    mbar_init(bar_q0, 1);
+    mbar_init(bar_q0 + 8, 1);
     mbar_init(bar_do, 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_dv, 1);
     mbar_init(bar_dk, 1);
     mbar_init(bar_dq, 1);
+    mbar_init(bar_fin, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -169,29 +182,25 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const uint32_t t_st = tmem + lane_base + half * 64;         // S^T, then dQ
-  const uint32_t t_dpt = tmem + lane_base + 128 + half * 64;  // dP^T
+  const uint32_t t_st = tmem + lane_base + half * 64;         // S^T
+  const uint32_t t_dpt = tmem + lane_base + 128 + half * 64;  // dP^T, then dQ
   const uint32_t t_dk = tmem + lane_base + 256;
   const uint32_t t_dv = tmem + lane_base + 384;
 
-  // Phases and copies/MMAs in flight; thread 0 issues every copy and MMA,
-  // so its own view is the one that the exit path settles.
-  uint32_t ph_q = 0, ph_do = 0, ph_s = 0, ph_dv = 0, ph_dk = 0, ph_dq = 0;
-  bool kv_pend = false, q_pend = false, do_pend = false, mma_pend = false;
-  uint32_t pend_bar = 0, pend_ph = 0;  // thread 0: the last barrier committed
-  auto commit = [&](uint32_t bar, uint32_t ph) {
-    mma_commit(bar);
-    pend_bar = bar;
-    pend_ph = ph;
-    mma_pend = true;
-  };
-  int tcount = 0;  // tiles done by this CTA: picks the LSE / D buffer
+  // Phases and copies in flight; thread 0 issues every copy and MMA, so its
+  // own view is the one that the exit path settles. Only thread 0 waits on
+  // the Q barriers: bit b of ph_qm / q_pendm is Q buffer b's.
+  uint32_t ph_qm = 0, ph_do = 0, ph_s = 0, ph_dv = 0, ph_dk = 0, ph_dq = 0;
+  uint32_t q_pendm = 0;
+  bool kv_pend = false, do_pend = false;
+  int tcount = 0;  // tiles done by this CTA: picks the Q and the LSE / D buffers
+  int nlist = 0;   // listings done by this CTA: picks the mask buffer
   uint32_t ph_kv = 0;
   bool ok = true;
   const int nw = (p.nb + 31) >> 5;
   // Loads of column c that need no listing: K_j, V_j and, since the diagonal
   // block (first query head) is nearly always the column's first kept tile,
-  // its Q, dO, LSE and D (LSE and D into buffer tcount & 1). A column whose
+  // its Q, dO, LSE and D (into buffers tcount & 1). A column whose
   // first kept tile is another block lets these copies land before it fetches
   // its own into the same buffers.
   auto column_row_term = [&](int c) {  // this thread's LSE (half 0) or D of the diagonal block
@@ -216,13 +225,16 @@ __global__ void __launch_bounds__(NT, 1)
       tma_load_3d(ka + HALF_BYTES, &tmK, 64, j * T, zkv, bar_kv);
       tma_load_3d(va, &tmV, 0, j * T, zkv, bar_kv);
       tma_load_3d(va + HALF_BYTES, &tmV, 64, j * T, zkv, bar_kv);
-      mbar_expect_tx(bar_q, TILE_BYTES);
-      tma_load_3d(qa, &tmQ, 0, j * T, zq0, bar_q);
-      tma_load_3d(qa + HALF_BYTES, &tmQ, 64, j * T, zq0, bar_q);
+      const int b = tcount & 1;
+      const uint32_t qb = qa0 + b * TILE_BYTES, bq = bar_q0 + 8 * b;
+      mbar_expect_tx(bq, TILE_BYTES);
+      tma_load_3d(qb, &tmQ, 0, j * T, zq0, bq);
+      tma_load_3d(qb + HALF_BYTES, &tmQ, 64, j * T, zq0, bq);
       mbar_expect_tx(bar_do, TILE_BYTES);
       tma_load_3d(da, &tmdO, 0, j * T, zq0, bar_do);
       tma_load_3d(da + HALF_BYTES, &tmdO, 64, j * T, zq0, bar_do);
-      kv_pend = q_pend = do_pend = true;
+      kv_pend = do_pend = true;
+      q_pendm |= 1u << b;
     }
   };
   int col = blockIdx.x;
@@ -248,10 +260,12 @@ __global__ void __launch_bounds__(NT, 1)
   const int z = zq0 + hg;  // query head: Q_i, dO_i, LSE, D, dQ, the keep bits
   const int kept_before = kept_count;
   for (int i0 = j; i0 < p.nb && ok; i0 += LIST_CHUNK) {
-    // ---- list the kept query blocks i in [i0, i0 + LIST_CHUNK), ascending:
-    // every bit word is loaded first, then one barrier orders the counts
+    // ---- the kept query blocks i in [i0, i0 + LIST_CHUNK) as a bit mask,
+    // bit b of word m for block i0 + 32 m + b (every bit word is loaded
+    // first, then one barrier publishes the mask); every thread walks it in
+    // ascending order. Two masks: a thread still walking the previous one
+    // is at most one listing behind.
     bool fk[LIST_ROUNDS];
-    unsigned bal[LIST_ROUNDS];
 #pragma unroll
     for (int k = 0; k < LIST_ROUNDS; ++k) {
       const int i = i0 + k * NT + tid;
@@ -260,55 +274,62 @@ __global__ void __launch_bounds__(NT, 1)
           (in && !p.never_skip) ? p.bits[((size_t)z * p.nb + i) * nw + (j >> 5)] : 0u;
       fk[k] = in && (p.never_skip || ((w >> (j & 31)) & 1u));
     }
+    uint32_t* msk = kmask + (nlist & 1) * MASK_WORDS;
+    ++nlist;
 #pragma unroll
     for (int k = 0; k < LIST_ROUNDS; ++k) {
-      bal[k] = __ballot_sync(0xffffffffu, fk[k]);
-      if (lane == 0) wcount[k * NWARP + warp] = __popc(bal[k]);
+      const unsigned bal = __ballot_sync(0xffffffffu, fk[k]);
+      if (lane == 0) msk[k * NWARP + warp] = bal;
     }
     __syncthreads();
-    int n_list = 0;
-#pragma unroll
-    for (int k = 0; k < LIST_ROUNDS; ++k) {
-      int off = n_list, tot = 0;
-#pragma unroll
-      for (int w = 0; w < NWARP; ++w) {
-        const int c = wcount[k * NWARP + w];
-        off += w < warp ? c : 0;
-        tot += c;
+    int mw = -1;
+    uint32_t rem = 0u;
+    auto next_block = [&]() -> int {  // the next kept block, -1 past the last
+      while (rem == 0u) {
+        if (++mw >= MASK_WORDS) return -1;
+        rem = msk[mw];
       }
-      if (fk[k]) list[off + __popc(bal[k] & ((1u << lane) - 1u))] = i0 + k * NT + tid;
-      n_list += tot;
-    }
-    __syncthreads();
-    // Within a list, tile li + 1's Q, dO, LSE and D are fetched while tile li
-    // is still being worked on: dO once the dP / dV products have read it,
-    // Q once the dK / dQ products have, LSE and D into the other buffer.
-    // Threads 0-127 move the LSE of query `row`, threads 128-255 its D.
+      const int bit = __ffs(rem) - 1;
+      rem &= rem - 1u;
+      return i0 + 32 * mw + bit;
+    };
+    // Within a list, tile n + 2's Q loads into tile n's Q buffer once tile
+    // n's dK product has read it, and tile n + 1's S^T is issued behind tile
+    // n's dQ product; tile n + 1's dO loads once tile n's dP / dV products
+    // have read the buffer, its LSE and D into the other buffer. Threads
+    // 0-127 move the LSE of query `row`, threads 128-255 its D.
+    int cur = next_block();
+    int nxt = cur >= 0 ? next_block() : -1;
+    int nxt2 = nxt >= 0 ? next_block() : -1;
+    bool s_ready = false;  // thread 0: this tile's S^T was issued by the previous tile
+    bool first = true;     // the list's first tile
     bool prefetched = false;
-    for (int li = 0; li < n_list && ok; ++li) {
-    const int i = list[li];
-    const bool has_next = li + 1 < n_list;
-    const int inext = has_next ? list[li + 1] : 0;
-    float* lse_c = lse_s + (tcount & 1) * T;
-    float* dd_c = dd_s + (tcount & 1) * T;
+    for (; cur >= 0 && ok; cur = nxt, nxt = nxt2, nxt2 = nxt2 >= 0 ? next_block() : -1) {
+    const int i = cur;
+    const bool has_next = nxt >= 0;
+    const int inext = has_next ? nxt : 0;
+    const int qb = tcount & 1;  // this tile's Q buffer; the next tile's is qb ^ 1
+    const uint32_t qc = qa0 + qb * TILE_BYTES, qn = qa0 + (qb ^ 1) * TILE_BYTES;
+    const uint32_t bar_qc = bar_q0 + 8 * qb, bar_qn = bar_q0 + 8 * (qb ^ 1);
+    float* lse_c = lse_s + qb * T;
+    float* dd_c = dd_s + qb * T;
     if (spec) {
       spec = false;
       if (hg == 0 && i == j) {
         prefetched = true;  // the diagonal's copies (and LSE, D) are this tile's
-      } else {
-        if (mbar_wait(bar_q, ph_q, abort, 0x208)) {
-          ph_q ^= 1;
+      } else if (tid == 0) {  // they land before this block's go into the buffers
+        if (mbar_wait(bar_qc, (ph_qm >> qb) & 1u, abort, 0x208)) {
+          ph_qm ^= 1u << qb;
+          q_pendm &= ~(1u << qb);
         } else {
           ok = false;
         }
-        if (tid == 0) {
-          if (mbar_wait(bar_do, ph_do, abort, 0x209)) {
-            ph_do ^= 1;
-          } else {
-            ok = false;
-          }
+        if (mbar_wait(bar_do, ph_do, abort, 0x209)) {
+          ph_do ^= 1;
+          do_pend = false;
+        } else {
+          ok = false;
         }
-        if (tid == 0) q_pend = do_pend = false;
       }
     }
     if (!prefetched) {
@@ -319,15 +340,26 @@ __global__ void __launch_bounds__(NT, 1)
       else
         dd_c[row] = qv ? p.Dterm[(size_t)z * p.L + q] : 0.f;
       if (tid == 0) {
-        mbar_expect_tx(bar_q, TILE_BYTES);
-        tma_load_3d(qa, &tmQ, 0, i * T, z, bar_q);
-        tma_load_3d(qa + HALF_BYTES, &tmQ, 64, i * T, z, bar_q);
+        mbar_expect_tx(bar_qc, TILE_BYTES);
+        tma_load_3d(qc, &tmQ, 0, i * T, z, bar_qc);
+        tma_load_3d(qc + HALF_BYTES, &tmQ, 64, i * T, z, bar_qc);
         mbar_expect_tx(bar_do, TILE_BYTES);
         tma_load_3d(da, &tmdO, 0, i * T, z, bar_do);
         tma_load_3d(da + HALF_BYTES, &tmdO, 64, i * T, z, bar_do);
-        q_pend = do_pend = true;
+        q_pendm |= 1u << qb;
+        do_pend = true;
       }
     }
+    // the list's second tile's Q into the other buffer, whose last readers
+    // (the previous tile's S^T and dK products) have completed; later tiles'
+    // Q load two tiles ahead, as each tile's dK product frees its buffer
+    if (tid == 0 && first && has_next) {
+      mbar_expect_tx(bar_qn, TILE_BYTES);
+      tma_load_3d(qn, &tmQ, 0, inext * T, z, bar_qn);
+      tma_load_3d(qn + HALF_BYTES, &tmQ, 64, inext * T, z, bar_qn);
+      q_pendm |= 1u << (qb ^ 1);
+    }
+    first = false;
     // next tile's LSE or D: loaded now, stored once this tile is done
     float next_val = 0.f;
     if (has_next) {
@@ -342,24 +374,26 @@ __global__ void __launch_bounds__(NT, 1)
       }
       kv_ready = true;
     }
-    if (mbar_wait(bar_q, ph_q, abort, 0x202)) {
-      ph_q ^= 1;
-      q_pend = false;
-    } else {
-      ok = false;
-    }
-    if (__syncthreads_or(!ok)) { ok = false; break; }
-    // ---- S^T = K_j Q_i^T; then dP^T = V_j dO_i^T, which needs no P and runs
-    // while the threads form P
+    // ---- S^T = K_j Q_i^T, unless the previous tile issued it; then
+    // dP^T = V_j dO_i^T, which needs no P and runs while the threads form P
+    // (the previous tile has read its dQ out of these columns)
     if (tid == 0) {
-      tc_fence_after();
+      if (!s_ready) {
+        if (mbar_wait(bar_qc, (ph_qm >> qb) & 1u, abort, 0x202)) {
+          ph_qm ^= 1u << qb;
+          q_pendm &= ~(1u << qb);
+          tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-        mma_bf16(tmem, sdesc_sw128(ka + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024),
-                 IDESC_KQ, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+            mma_bf16(tmem, sdesc_sw128(ka + off, 16, 1024), sdesc_sw128(qc + off, 16, 1024),
+                     IDESC_KQ, kk > 0);
+          }
+          mma_commit(bar_s);
+        } else {
+          ok = false;
+        }
       }
-      commit(bar_s, ph_s);
       if (mbar_wait(bar_do, ph_do, abort, 0x204)) {
         ph_do ^= 1;
         do_pend = false;
@@ -434,7 +468,7 @@ __global__ void __launch_bounds__(NT, 1)
                    sdesc_sw128(da + kk * 2048, HALF_BYTES, 1024), IDESC_ACC,
                    (kept_count > 0 || kk > 0) ? 1u : 0u);
         }
-        commit(bar_dv, ph_dv);
+        mma_commit(bar_dv);
       }
       if (mbar_wait(bar_dv, ph_dv, abort, 0x205)) {  // dP^T and dV done
         ph_dv ^= 1;
@@ -484,38 +518,58 @@ __global__ void __launch_bounds__(NT, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
-      // ---- dK += hi^T Q_i, then dQ_i = (hi + lo) K_j (into the S^T columns);
-      // once dK is done Q_i is free and the next tile's Q loads while the dQ
-      // products run. dK sums over queries, where dS has no cancelling
-      // structure: the single rounding of hi leaves it within ~2e-3 (rel-L2).
+      // ---- dK += hi^T Q_i, then dQ_i = (hi + lo) K_j into the dP^T columns
+      // (read into the threads by now), then the next tile's S^T into the
+      // S^T columns (P has been formed), its Q having landed meanwhile. dK
+      // sums over queries, where dS has no cancelling structure: the single
+      // rounding of hi leaves it within ~2e-3 (rel-L2).
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < T / 16; ++kk) {
           const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
           mma_bf16(tmem + 256, sdesc_sw128(sta + aoff, 16, 1024),
-                   sdesc_sw128(qa + kk * 2048, HALF_BYTES, 1024), IDESC_ACC,
+                   sdesc_sw128(qc + kk * 2048, HALF_BYTES, 1024), IDESC_ACC,
                    (kept_count > 0 || kk > 0) ? 1u : 0u);
         }
-        commit(bar_dk, ph_dk);
+        mma_commit(bar_dk);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
           const uint32_t src = part == 0 ? sta : pta;
 #pragma unroll
           for (int kk = 0; kk < T / 16; ++kk) {
-            mma_bf16(tmem, sdesc_sw128(src + kk * 2048, HALF_BYTES, 1024),
+            mma_bf16(tmem + 128, sdesc_sw128(src + kk * 2048, HALF_BYTES, 1024),
                      sdesc_sw128(ka + kk * 2048, HALF_BYTES, 1024), IDESC_DQ,
                      (part > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        commit(bar_dq, ph_dq);
+        mma_commit(bar_dq);
+        s_ready = false;
+        if (has_next) {
+          if (mbar_wait(bar_qn, (ph_qm >> (qb ^ 1)) & 1u, abort, 0x20d)) {
+            ph_qm ^= 1u << (qb ^ 1);
+            q_pendm &= ~(1u << (qb ^ 1));
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+              mma_bf16(tmem, sdesc_sw128(ka + off, 16, 1024), sdesc_sw128(qn + off, 16, 1024),
+                       IDESC_KQ, kk > 0);
+            }
+            mma_commit(bar_s);
+            s_ready = true;
+          } else {
+            ok = false;
+          }
+        }
+        // the dK product has read Q_i: the tile after next loads into qc
         if (mbar_wait(bar_dk, ph_dk, abort, 0x207)) {
           ph_dk ^= 1;
-          if (has_next) {  // Q_i has been read
-            mbar_expect_tx(bar_q, TILE_BYTES);
-            tma_load_3d(qa, &tmQ, 0, inext * T, z, bar_q);
-            tma_load_3d(qa + HALF_BYTES, &tmQ, 64, inext * T, z, bar_q);
-            q_pend = true;
+          if (nxt2 >= 0) {
+            mbar_expect_tx(bar_qc, TILE_BYTES);
+            tma_load_3d(qc, &tmQ, 0, nxt2 * T, z, bar_qc);
+            tma_load_3d(qc + HALF_BYTES, &tmQ, 64, nxt2 * T, z, bar_qc);
+            q_pendm |= 1u << qb;
           }
         } else {
           ok = false;
@@ -523,7 +577,6 @@ __global__ void __launch_bounds__(NT, 1)
       }
       if (mbar_wait(bar_dq, ph_dq, abort, 0x206)) {
         ph_dq ^= 1;
-        mma_pend = false;  // every MMA of the tile has completed
       } else {
         ok = false;
       }
@@ -539,7 +592,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float v[32];
-        tmem_ld32(t_st + c * 32, v);
+        tmem_ld32(t_dpt + c * 32, v);
         const uint32_t blk = pta + (uint32_t)(2 * half + c) * 16384u + (uint32_t)row * 128u;
 #pragma unroll
         for (int q = 0; q < 8; ++q)
@@ -578,22 +631,27 @@ __global__ void __launch_bounds__(NT, 1)
     if (!mbar_wait(bar_kv, ph_kv, abort, 0x20a)) ok = false;
   }
   ph_kv ^= 1;
-  if (spec) {
-    if (!mbar_wait(bar_q, ph_q, abort, 0x20b)) ok = false;
-    ph_q ^= 1;
-    if (tid == 0) {
-      if (!mbar_wait(bar_do, ph_do, abort, 0x20c)) ok = false;
-      ph_do ^= 1;
-    }
+  if (spec && tid == 0) {
+    const int b = tcount & 1;
+    if (!mbar_wait(bar_q0 + 8 * b, (ph_qm >> b) & 1u, abort, 0x20b)) ok = false;
+    ph_qm ^= 1u << b;
+    if (!mbar_wait(bar_do, ph_do, abort, 0x20c)) ok = false;
+    ph_do ^= 1;
   }
   if (tid == 0) {
-    kv_pend = q_pend = do_pend = false;
+    // with every wait met nothing is in flight: the column's last tile loads
+    // no next Q, and the diagonal's copies were claimed or waited for
+    if (ok) {
+      kv_pend = do_pend = false;
+      q_pendm = 0u;
+    }
     *item_slot = fetched;
   }
   // the epilogue stages dK_j, dV_j in the P^T and dS^T buffers once the last
   // tile's dQ reductions have read them
   if (tid == BULK_TID) bulk_wait_read_all();
-  __syncthreads();  // item_slot written; every thread past its column's loads
+  // item_slot written; every thread past its column's loads
+  if (__syncthreads_or(!ok)) ok = false;
   const int next = *item_slot;
   const bool more = ok && next < n_items;
   // the next column's copies start now; its LSE / D are loaded now and stored
@@ -637,13 +695,16 @@ __global__ void __launch_bounds__(NT, 1)
   col = next;
   }
   // thread 0's copies and MMAs still in flight (anything on the error path)
-  // land before the CTA releases its shared memory and TMEM
+  // land before the CTA releases its shared memory and TMEM: one last commit
+  // covers every MMA it issued
   if (tid == BULK_TID) bulk_wait_all();  // every dQ reduction and dK / dV store has landed
   if (tid == 0) {
     if (kv_pend) mbar_settle(bar_kv, ph_kv);
-    if (q_pend) mbar_settle(bar_q, ph_q);
+    if (q_pendm & 1u) mbar_settle(bar_q0, ph_qm & 1u);
+    if (q_pendm & 2u) mbar_settle(bar_q0 + 8, (ph_qm >> 1) & 1u);
     if (do_pend) mbar_settle(bar_do, ph_do);
-    if (!ok && mma_pend) mbar_settle(pend_bar, pend_ph);
+    mma_commit(bar_fin);
+    mbar_settle(bar_fin, 0);
   }
   tc_fence_before();
   __syncthreads();
