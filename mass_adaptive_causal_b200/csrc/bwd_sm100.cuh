@@ -61,6 +61,7 @@ constexpr int MASK_WORDS = LIST_CHUNK / 32;
 // K, V, Q (two buffers), dO, P^T, dS^T; LSE and D (two buffers each); the
 // barriers; the kept-block masks (two)
 constexpr uint32_t SMEM_BYTES = 7 * TILE_BYTES + 2048 + 128 + 2 * MASK_WORDS * 4;
+static_assert(SMEM_BYTES <= 227 * 1024, "the work pass must fit one CTA's shared memory");
 constexpr uint32_t TMEM_COLS = 512;
 // S^T, dP^T: A = K_j or V_j (K-major over d), B = Q_i or dO_i (K-major over d)
 constexpr uint32_t IDESC_KQ = idesc_bf16(128, 128, false, false);
@@ -187,9 +188,10 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t t_dk = tmem + lane_base + 256;
   const uint32_t t_dv = tmem + lane_base + 384;
 
-  // Phases and copies in flight; thread 0 issues every copy and MMA, so its
-  // own view is the one that the exit path settles. Only thread 0 waits on
-  // the Q barriers: bit b of ph_qm / q_pendm is Q buffer b's.
+  // Phases and copies in flight; thread 0 issues every load and MMA, so its
+  // own view is the one that the exit path settles (the bulk copies out of
+  // shared memory are BULK_TID's). Only thread 0 waits on the Q barriers:
+  // bit b of ph_qm / q_pendm is Q buffer b's.
   uint32_t ph_qm = 0, ph_do = 0, ph_s = 0, ph_dv = 0, ph_dk = 0, ph_dq = 0;
   uint32_t q_pendm = 0;
   bool kv_pend = false, do_pend = false;
