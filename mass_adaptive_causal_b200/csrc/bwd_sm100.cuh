@@ -58,9 +58,10 @@ constexpr uint32_t HALF_BYTES = T * 64 * 2;
 constexpr int LIST_CHUNK = 1024;  // query blocks listed per round
 constexpr int LIST_ROUNDS = LIST_CHUNK / NT;
 constexpr int MASK_WORDS = LIST_CHUNK / 32;
+static_assert(MASK_WORDS == LIST_ROUNDS * NWARP, "one mask word per warp and listing round");
 // K, V, Q (two buffers), dO, P^T, dS^T; LSE and D (two buffers each); the
-// barriers; the kept-block masks (two)
-constexpr uint32_t SMEM_BYTES = 7 * TILE_BYTES + 2048 + 128 + 2 * MASK_WORDS * 4;
+// barriers; the kept-block masks and their per-warp nonzero-word bits (two)
+constexpr uint32_t SMEM_BYTES = 7 * TILE_BYTES + 2048 + 128 + 2 * (MASK_WORDS + NWARP) * 4;
 static_assert(SMEM_BYTES <= 227 * 1024, "the work pass must fit one CTA's shared memory");
 constexpr uint32_t TMEM_COLS = 512;
 // S^T, dP^T: A = K_j or V_j (K-major over d), B = Q_i or dO_i (K-major over d)
@@ -133,6 +134,7 @@ __global__ void __launch_bounds__(NT, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint32_t* kmask = reinterpret_cast<uint32_t*>(bars + 16);  // [2][MASK_WORDS]
+  uint32_t* knz = kmask + 2 * MASK_WORDS;                     // [2][NWARP]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -277,18 +279,36 @@ __global__ void __launch_bounds__(NT, 1)
       fk[k] = in && (p.never_skip || ((w >> (j & 31)) & 1u));
     }
     uint32_t* msk = kmask + (nlist & 1) * MASK_WORDS;
+    uint32_t* wnz = knz + (nlist & 1) * NWARP;  // bit k: this warp's word of round k is nonzero
     ++nlist;
+    uint32_t nzbits = 0u;
 #pragma unroll
     for (int k = 0; k < LIST_ROUNDS; ++k) {
       const unsigned bal = __ballot_sync(0xffffffffu, fk[k]);
       if (lane == 0) msk[k * NWARP + warp] = bal;
+      nzbits |= (bal != 0u ? 1u : 0u) << k;
     }
+    if (lane == 0) wnz[warp] = nzbits;
     __syncthreads();
+    // bit m: mask word m is nonzero, so the walk goes from one kept block's
+    // word to the next without reading the empty words between them
+    uint32_t nzw = 0u;
+#pragma unroll
+    for (int w = 0; w < NWARP; ++w) {
+      const uint32_t b = wnz[w];
+#pragma unroll
+      for (int k = 0; k < LIST_ROUNDS; ++k) nzw |= ((b >> k) & 1u) << (k * NWARP + w);
+    }
     int mw = -1;
     uint32_t rem = 0u;
     auto next_block = [&]() -> int {  // the next kept block, -1 past the last
       while (rem == 0u) {
-        if (++mw >= MASK_WORDS) return -1;
+        const uint32_t ahead = mw >= MASK_WORDS - 1 ? 0u : nzw & (~0u << (mw + 1));
+        if (ahead == 0u) {
+          mw = MASK_WORDS;
+          return -1;
+        }
+        mw = __ffs(ahead) - 1;
         rem = msk[mw];
       }
       const int bit = __ffs(rem) - 1;
